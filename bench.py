@@ -1,0 +1,444 @@
+#!/usr/bin/env python
+"""MoE layer forward benchmark: routed tokens/s on B200, with the roofline.
+
+One step = one whole layer forward (route, dispatch, grouped expert FFN,
+shared expert, combine) over one batch of synthetic input already resident
+in HBM.  Default workload: the Mixtral-style prefill layer (T=4096,
+hidden 4096, intermediate 14336, 8 experts, top-2, SwiGLU, bf16).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+Multi-GPU (torchrun, one rank per GPU): every rank runs an independent
+replica on its own batch (the layer has no exchange step without a capacity
+limit), so the job's throughput is N * T / (slowest rank's step time).
+``--impl reference`` times the CPU oracle (the plain float64 statement of the
+layer) on the host cores instead, on a bounded token sample per step.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "MoE layer fwd routed tokens/s on 1 B200; % of tensor/HBM roofline"
+UNIT = "tokens/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=30)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="mixtral_prefill")
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-sample", type=int, default=0, help="tokens in the oracle sample (0 = auto)")
+    return ap.parse_args()
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as fh:
+            p = json.load(fh)
+        return p, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ---------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines: list[str] = []
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (FileNotFoundError, OSError):
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.15)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        if self.thread:
+            self.thread.join(timeout=2)
+        sm, mx, power, reasons = [], [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx.append(float(parts[2]))
+                power.append(float(parts[3]))
+            except ValueError:
+                continue
+            for nm, val in zip(names, parts[5:9]):
+                if val.lower() == "active":
+                    reasons.add(nm)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "power_w_max": max(power) if power else None, "samples": len(sm),
+                "reasons": sorted(reasons)}
+
+
+# ---------------------------------------------------------------- cost model
+
+def layer_costs(w, R: int, touched: int) -> dict:
+    """Algorithmic FLOP and bytes of the layer and of each expert GEMM.
+
+    R = routed rows kept after the capacity cut, touched = experts with at
+    least one row.  Counts the work the method must do (the touched experts'
+    weights read once, x in, out written) and not the buffers it chooses."""
+    es = 4 if w.dtype == "f32" else 2
+    glu = 2 if w.act == "swiglu" else 1
+    if w.weight_format == "q4_affine_g64":
+        wbytes_per_elem = 0.5
+        scale_bytes = lambda n, k: n * (k // 64) * 4       # bf16 scale + bias per group
+    else:
+        wbytes_per_elem = es
+        scale_bytes = lambda n, k: 0
+    w1 = touched * (glu * (w.F * w.d * wbytes_per_elem + scale_bytes(w.F, w.d)))
+    w3 = touched * (w.d * w.F * wbytes_per_elem + scale_bytes(w.d, w.F))
+    f1 = 2.0 * R * w.d * w.F * glu
+    f2 = 2.0 * R * w.F * w.d
+    fs = 6.0 * w.T * w.d * w.shared_F if w.shared_F else 0.0
+    sbytes = 3 * w.d * w.shared_F * es if w.shared_F else 0
+    router = 2.0 * w.T * w.d * w.E
+    flops = f1 + f2 + fs + router
+    xbytes = w.T * w.d * es
+    layer_bytes = w1 + w3 + sbytes + 2 * xbytes + w.E * w.d * 4
+    return dict(flops=flops, bytes=layer_bytes,
+                ffn1=dict(flops=f1, bytes=w1 + R * w.d * es + R * w.F * es),
+                ffn2=dict(flops=f2, bytes=w3 + R * w.F * es + R * w.d * es))
+
+
+def source_hash(path: str) -> str:
+    with open(path, "rb") as fh:
+        return hashlib.sha256(fh.read()).hexdigest()[:16]
+
+
+def recorded_traffic(kernel_file: str, workload: str):
+    """DRAM bytes per launch of the dominant kernel from the committed ncu
+    summary, if it was taken on the current source of that kernel."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as fh:
+        rec = json.load(fh)
+    ent = rec.get(workload)
+    if not ent or ent.get("source_sha256_16") != source_hash(kernel_file):
+        return None
+    return ent.get("dram_bytes_per_launch")
+
+
+# ---------------------------------------------------------------- CPU oracle arm
+
+def oracle_sample_run(w, inp, n_tokens: int, seed: int = 0):
+    """Route every token and evaluate the experts on a seeded sample of
+    ``n_tokens`` tokens with the CPU oracle.  Returns (seconds, tokens, result)."""
+    import numpy as np
+    from mixture_experts_layer_41_b200.inputs import to_host
+    from oracle import moe_oracle as O
+
+    rng = np.random.default_rng(seed)
+    toks = np.sort(rng.choice(w.T, size=min(n_tokens, w.T), replace=False))
+    host = {k: to_host(v) for k, v in inp.items() if v is not None}
+
+    def experts(e):
+        out = {}
+        for key in ("w1", "w2", "w3", "q1", "q2", "q3", "s1", "s2", "s3", "b1", "b2", "b3"):
+            if key in host:
+                out[key] = host[key][e]
+        return out
+
+    shared = {k: host[k] for k in ("ws1", "ws2", "ws3")} if w.shared_F else None
+    t0 = time.perf_counter()
+    res = O.layer_forward(host["x"], host["w_router"], experts, top_k=w.k, act=w.act,
+                          capacity_factor=w.capacity_factor, router=w.router, norm=w.norm_topk_prob,
+                          routed_scaling=w.routed_scaling, n_group=w.n_group, topk_group=w.topk_group,
+                          expert_bias=host.get("expert_bias"), logit_bias=host.get("logit_bias"),
+                          shared=shared, aux_alpha=w.aux_alpha, tokens=toks)
+    return time.perf_counter() - t0, toks, res
+
+
+def blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:  # noqa: BLE001
+        return os.cpu_count() or 1
+
+
+def auto_sample(w) -> int:
+    # about 10-30 s of oracle work on a few dozen host cores
+    per_tok = 6.0 * w.d * w.F * w.k
+    n = int(4e11 / max(per_tok, 1.0))
+    return max(8, min(w.T, n, 256))
+
+
+def run_reference(args):
+    import torch
+    from mixture_experts_layer_41_b200.inputs import make_inputs, workload
+
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    w = workload(args.workload)
+    inp = make_inputs(w, seed=args.seed, device="cpu")
+    n = args.cpu_sample or max(4, auto_sample(w) // 8)
+    for _ in range(args.warmup):
+        oracle_sample_run(w, inp, n, seed=args.seed)
+    times = []
+    for i in range(args.steps):
+        dt, toks, _ = oracle_sample_run(w, inp, n, seed=args.seed + i)
+        times.append(dt)
+    sec = statistics.mean(times)
+    value = len(toks) / sec
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": sec * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, "T": w.T, "d": w.d, "F": w.F, "E": w.E, "top_k": w.k},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+                         "sample": f"route all {w.T} tokens, expert MLPs on {len(toks)} sampled tokens per step"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------- GPU arm
+
+def run_ours(args):
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    from mixture_experts_layer_41_b200 import _lib as L
+    from mixture_experts_layer_41_b200 import api
+    from mixture_experts_layer_41_b200.inputs import make_inputs, workload
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.gpus != world and world > 1:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE {world}")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    w = workload(args.workload)
+    inp = make_inputs(w, seed=args.seed + rank, device=dev)
+    wf = "q4_affine_g64" if w.weight_format == "q4_affine_g64" else w.dtype
+    cfg = api.make_config(num_tokens=w.T, hidden=w.d, intermediate=w.F, num_experts=w.E, top_k=w.k,
+                          router=w.router, norm_topk_prob=w.norm_topk_prob,
+                          routed_scaling=w.routed_scaling if w.router == "sigmoid_group" else 1.0,
+                          n_group=w.n_group, topk_group=w.topk_group, capacity_factor=w.capacity_factor,
+                          act=w.act, act_dtype=w.dtype, weight_dtype=wf, shared_intermediate=w.shared_F,
+                          aux_alpha=w.aux_alpha)
+    weights = {k: inp[k] for k in ("w1", "w2", "w3", "s1", "s2", "s3", "b1", "b2", "b3", "ws1", "ws2", "ws3")
+               if inp.get(k) is not None}
+    for i in "123":
+        if inp.get("q" + i) is not None:
+            weights["w" + i] = inp["q" + i]
+    bias = inp["logit_bias"] if w.router == "softmax_topk" else inp["expert_bias"]
+    layer = api.MoELayer(cfg, inp["w_router"], weights, router_bias=bias, device=dev)
+    x = inp["x"]
+    stream = torch.cuda.current_stream()
+
+    # warm-up
+    for _ in range(args.warmup):
+        layer.forward(x)
+    torch.cuda.synchronize()
+    st = layer.status()
+    if st != 0:
+        raise SystemExit(f"device status {st}: {api.moe_status_string(st)}")
+
+    # timed region: K whole-layer steps, phase events recorded on the launching stream
+    K = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(L.MOE_PHASE_COUNT)] for _ in range(K)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(local) if rank == 0 or world == 1 else None
+    barrier()
+    torch.cuda.synchronize()
+    if sampler:
+        sampler.start()
+        time.sleep(0.3)
+    start.record(stream)
+    for i in range(K):
+        api.moe_set_phase_events(ev[i])
+        layer.forward(x)
+    end.record(stream)
+    torch.cuda.synchronize()
+    api.moe_set_phase_events(None)
+    barrier()
+    clocks = sampler.stop() if sampler else None
+    ms = start.elapsed_time(end) / K
+    phases = {}
+    names = ["route", "permute", "ffn1", "ffn2", "shared", "combine"]
+    for p, nm in enumerate(names, start=1):
+        phases[nm] = statistics.mean(ev[i][p - 1].elapsed_time(ev[i][p]) for i in range(K))
+    ms_t = torch.tensor([ms], device=dev)
+    if world > 1:
+        dist.all_reduce(ms_t, op=dist.ReduceOp.MAX)
+    ms_max = float(ms_t.item())
+
+    # routing outcome of the timed steps (identical every step)
+    kept = layer.o.kept_counts.cpu().numpy()
+    R = int(kept.sum())
+    touched = int((kept > 0).sum())
+    dropped = int(layer.o.dropped[0].item())
+    aux_raw, aux = api.moe_aux_loss(cfg, layer.o.kept_counts.cpu(), layer.o.prob_sum.cpu())
+
+    # e2e: the same layer through moe_forward_host with pinned host buffers
+    dt = x.dtype
+    x_host = x.cpu().pin_memory()
+    out_host = torch.empty((w.T, w.d), dtype=dt).pin_memory()
+    kc_host = torch.empty(w.E, dtype=torch.int32).pin_memory()
+    ps_host = torch.empty(w.E, dtype=torch.float32).pin_memory()
+    dr_host = torch.empty(4, dtype=torch.int32).pin_memory()
+    for _ in range(max(2, args.warmup // 2)):
+        api.moe_forward_host(cfg, x_host, inp["w_router"], bias, weights, out_host, kc_host, ps_host, dr_host,
+                             layer.ws)
+    torch.cuda.synchronize()
+    barrier()
+    e_s, e_e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e_s.record(stream)
+    for _ in range(K):
+        api.moe_forward_host(cfg, x_host, inp["w_router"], bias, weights, out_host, kc_host, ps_host, dr_host,
+                             layer.ws)
+    e_e.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e_s.elapsed_time(e_e) / K
+    e2e_t = torch.tensor([e2e_ms], device=dev)
+    if world > 1:
+        dist.all_reduce(e2e_t, op=dist.ReduceOp.MAX)
+    e2e_ms = float(e2e_t.item())
+    h2d = x_host.numel() * x_host.element_size()
+    d2h = out_host.numel() * out_host.element_size() + 2 * 4 * w.E + 4
+    same = torch.equal(out_host.view(torch.int16) if dt == torch.bfloat16 else out_host,
+                       layer.o.out.cpu().view(torch.int16) if dt == torch.bfloat16 else layer.o.out.cpu())
+
+    peaks, peak_src = load_peaks()
+    costs = layer_costs(w, R, touched)
+    tensor_peak = peaks["bf16_tflops"] * 1e12          # burst: kernels timed back to back, < 1 s
+    hbm_peak = peaks["hbm_gbs"] * 1e9
+    # dominant kernel: the longer expert GEMM phase
+    dom = "ffn1" if phases["ffn1"] >= phases["ffn2"] else "ffn2"
+    dk = costs[dom]
+    t_dom = phases[dom] * 1e-3
+    t_tensor, t_hbm = dk["flops"] / tensor_peak, dk["bytes"] / hbm_peak
+    kernel_file = os.path.join(ROOT, "mixture_experts_layer_41_b200", "csrc",
+                               "ffn_q4.cu" if w.weight_format == "q4_affine_g64" else
+                               ("ffn_simt.cu" if w.dtype == "f32" else "ffn_tc.cu"))
+    traffic = recorded_traffic(kernel_file, f"{w.name}:{dom}")
+    if t_tensor >= t_hbm and w.weight_format == "dense" and w.dtype == "bf16":
+        roof = {"bound": "tensor", "achieved": dk["flops"] / t_dom / 1e12, "peak": peaks["bf16_tflops"],
+                "unit": "TFLOP/s"}
+    else:
+        roof = {"bound": "hbm", "achieved": dk["bytes"] / t_dom / 1e9, "peak": peaks["hbm_gbs"], "unit": "GB/s"}
+    roof["frac"] = roof["achieved"] / roof["peak"]
+    roof["traffic"] = traffic
+    roof["kernel"] = {"ffn1": "grouped expert GEMM, phase 1 (gate/up or in)",
+                      "ffn2": "grouped expert GEMM, phase 2 (down or out)"}[dom]
+    roof["peak_source"] = f"{peak_src} ({'burst' if roof['bound'] == 'tensor' else 'copy'})"
+    roof["algorithmic"] = {"flop_per_launch": dk["flops"], "bytes_per_launch": dk["bytes"],
+                           "ms_per_launch": phases[dom]}
+    t_layer_roof = max(costs["flops"] / tensor_peak, costs["bytes"] / hbm_peak)
+
+    per_gpu = w.T / (ms_max * 1e-3)
+    line = {
+        "metric": METRIC, "value": per_gpu * world, "unit": UNIT, "n_gpus": world, "steps": K,
+        "warmup": args.warmup, "ms_per_step": ms_max, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16" if w.dtype == "bf16" else w.dtype, "data": "synthetic",
+        "config": {"workload": w.name, "T": w.T, "d": w.d, "F": w.F, "E": w.E, "top_k": w.k, "act": w.act,
+                   "router": w.router, "capacity_factor": w.capacity_factor or None,
+                   "weights": w.weight_format, "shared_F": w.shared_F, "parallelism": f"replicas x{world}",
+                   "l2": "inputs larger than L2: every step streams all touched expert weights "
+                         f"({costs['bytes'] / 1e9:.2f} GB) from HBM"},
+        "roofline": roof,
+        "layer_roofline": {"frac": t_layer_roof / (ms_max * 1e-3), "roof_ms": t_layer_roof * 1e3,
+                           "flop": costs["flops"], "bytes": costs["bytes"],
+                           "tflops": costs["flops"] / (ms_max * 1e-3) / 1e12},
+        "phases_ms": {k: round(v, 4) for k, v in phases.items()},
+        "routing": {"rows": R, "touched_experts": touched, "dropped": dropped, "aux_raw": aux_raw, "aux": aux},
+        "e2e": {"value": world * w.T / (e2e_ms * 1e-3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms, "matches_device_out": bool(same)},
+        "gpu_launches": K * (8 + (2 if w.shared_F else 0)),
+        "clocks": clocks,
+    }
+
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        n = args.cpu_sample or auto_sample(w)
+        host_inp = {k: v for k, v in inp.items()}
+        sec, toks, res = oracle_sample_run(w, host_inp, n, seed=args.seed)
+        got = layer.o.out.float().cpu().numpy().astype(np.float64)[toks]
+        ref = res["out"][toks]
+        err = float(np.abs(got - ref).max() / max(np.abs(ref).max(), 1e-30))
+        line["cpu_baseline"] = {"value": len(toks) / sec, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+                                "sample": f"route all {w.T} tokens + expert MLPs of {len(toks)} seeded tokens "
+                                          f"({sec:.1f} s)"}
+        line["parity_on_sample"] = {"tokens": int(len(toks)), "rel_err": err,
+                                    "tol": 1e-5 if w.dtype == "f32" else 2e-2,
+                                    "ok": err <= (1e-5 if w.dtype == "f32" else 2e-2)}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    args = parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,172 @@
+// Shared definitions of the MoE library: workspace layout, device status
+// codes and small device helpers.  Internal to the library.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+#include <stddef.h>
+
+#include "../../include/moe.h"
+
+namespace moe {
+
+// ---------------------------------------------------------------- tiling constants
+constexpr int kRouteTokens = 32;      // tokens per router block
+constexpr int kRouteThreads = 256;
+constexpr int kPermTokens = 256;      // tokens per dispatch count block
+constexpr int kMaxExperts = 256;
+constexpr int kMaxTopK = 32;
+constexpr int kMaxGroups = 32;
+
+// ---------------------------------------------------------------- device status
+// The first word of the workspace holds 0 or the code of the first failure a
+// kernel recorded (atomicCAS from 0).
+enum DeviceStatus : int {
+  kDevOk = 0,
+  kDevBadExpertId = 1,       // dispatch: topk id outside [0, E)
+  kDevDuplicateId = 2,       // dispatch: a token names the same expert twice
+  kDevTimeoutProducer = 10,  // grouped GEMM: TMA producer waited too long
+  kDevTimeoutMma = 11,       // grouped GEMM: MMA issuer waited too long
+  kDevTimeoutEpilogue = 12,  // grouped GEMM: epilogue waited too long
+  kDevTimeoutDrain = 13,     // grouped GEMM: in-flight work did not drain after an abort
+  kDevBadOffsets = 20,       // grouped FFN: expert_offsets not 0-based / non-decreasing / in range
+};
+
+__device__ __forceinline__ void record_status(int *status, int code) {
+  atomicCAS(status, 0, code);
+}
+
+// ---------------------------------------------------------------- workspace
+struct WsLayout {
+  size_t status;       // int32[64]
+  size_t route_part;   // double[nb_route][E]
+  size_t blk_counts;   // int32[nb_perm][E]
+  size_t blk_base;     // int32[nb_perm][E]
+  size_t local_rank;   // int32[T*k]
+  size_t offsets;      // int32[E+1]
+  size_t perm_token;   // int32[T*k]
+  size_t perm_w;       // float[T*k]
+  size_t slot_row;     // int32[T*k]
+  size_t topk_ids;     // int32[T*k]
+  size_t topk_w;       // float[T*k]
+  size_t raw_counts;   // int32[E]
+  size_t kept_counts;  // int32[E]
+  size_t prob_sum;     // float[E]
+  size_t dropped;      // int32[1]
+  size_t x_perm;       // act[T*k][d]
+  size_t h;            // act[T*k][F]   (grouped FFN intermediate)
+  size_t y_perm;       // act[T*k][d]
+  size_t shared_h;     // act[T][Fs]
+  size_t shared_out;   // act[T][d]
+  size_t x_stage;      // act[T][d]   (moe_forward_host)
+  size_t out_stage;    // act[T][d]
+  size_t total;
+};
+
+inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+inline size_t act_size(const moe_config &c) { return c.act_dtype == MOE_F32 ? 4 : 2; }
+
+inline int route_blocks(const moe_config &c) {
+  return (c.num_tokens + kRouteTokens - 1) / kRouteTokens;
+}
+inline int perm_blocks(const moe_config &c) {
+  return (c.num_tokens + kPermTokens - 1) / kPermTokens;
+}
+
+inline WsLayout ws_layout(const moe_config &c) {
+  WsLayout L{};
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    size_t here = off;
+    off = align_up(off + bytes, 256);
+    return here;
+  };
+  const size_t T = (size_t)c.num_tokens, E = (size_t)c.num_experts, K = (size_t)c.top_k;
+  const size_t d = (size_t)c.hidden, F = (size_t)c.intermediate;
+  const size_t Fs = (size_t)(c.shared_intermediate > 0 ? c.shared_intermediate : 0);
+  const size_t es = act_size(c);
+  const size_t slots = T * K;
+  L.status = take(256);
+  L.route_part = take(sizeof(double) * route_blocks(c) * E);
+  L.blk_counts = take(sizeof(int32_t) * perm_blocks(c) * E);
+  L.blk_base = take(sizeof(int32_t) * perm_blocks(c) * E);
+  L.local_rank = take(sizeof(int32_t) * slots);
+  L.offsets = take(sizeof(int32_t) * (E + 1));
+  L.perm_token = take(sizeof(int32_t) * slots);
+  L.perm_w = take(sizeof(float) * slots);
+  L.slot_row = take(sizeof(int32_t) * slots);
+  L.topk_ids = take(sizeof(int32_t) * slots);
+  L.topk_w = take(sizeof(float) * slots);
+  L.raw_counts = take(sizeof(int32_t) * E);
+  L.kept_counts = take(sizeof(int32_t) * E);
+  L.prob_sum = take(sizeof(float) * E);
+  L.dropped = take(sizeof(int32_t));
+  L.x_perm = take(es * slots * d);
+  L.h = take(es * slots * F);
+  L.y_perm = take(es * slots * d);
+  L.shared_h = take(es * T * Fs);
+  L.shared_out = take(Fs ? es * T * d : 0);
+  L.x_stage = take(es * T * d);
+  L.out_stage = take(es * T * d);
+  L.total = off;
+  return L;
+}
+
+template <typename P>
+inline P *ws_ptr(void *ws, size_t off) {
+  return reinterpret_cast<P *>(static_cast<char *>(ws) + off);
+}
+
+// ---------------------------------------------------------------- device helpers
+__device__ __forceinline__ float bf16_to_f32(uint16_t b) {
+  return __uint_as_float(((uint32_t)b) << 16);
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t *>(&v);
+}
+
+// ---------------------------------------------------------------- launchers (one per kernel file)
+cudaError_t launch_route(const moe_config &c, const void *x, const float *w_router,
+                         const float *router_bias, int32_t *topk_ids, float *topk_w,
+                         double *route_part, float *prob_sum, cudaStream_t s);
+
+cudaError_t launch_permute(const moe_config &c, const void *x, const int32_t *topk_ids,
+                           const float *topk_w, int64_t capacity, int32_t *expert_offsets,
+                           int32_t *perm_token, float *perm_w, int32_t *slot_row, void *x_perm,
+                           int32_t *raw_counts, int32_t *kept_counts, int32_t *dropped,
+                           int32_t *blk_counts, int32_t *blk_base, int32_t *local_rank,
+                           int *status, cudaStream_t s);
+
+// Two-phase expert FFN over groups.  `offsets` == nullptr means one group of
+// `rows` rows (the shared expert).  Writes the intermediate to `h` and the
+// result to `y`.
+struct FfnArgs {
+  int kind;                 // 0 = fp32 SIMT, 1 = bf16 tensor cores, 2 = q4 (bf16 act)
+  int act;                  // moe_act
+  int E;                    // groups
+  int rows_cap;             // allocated rows of x / h / y
+  int rows;                 // used when offsets == nullptr
+  int d, F;
+  const int32_t *offsets;   // [E+1] device or nullptr
+  const void *x;            // [rows_cap, d]
+  const void *w1, *w2, *w3; // [E,F,d], [E,F,d], [E,d,F] (q4: packed codes)
+  const void *s1, *s2, *s3, *b1, *b2, *b3;  // q4 scale / bias
+  void *h;                  // [rows_cap, F]
+  void *y;                  // [rows_cap, d]
+  int *status;
+  cudaEvent_t mid_event;    // recorded between the two phases when not null
+};
+
+cudaError_t launch_ffn_simt_f32(const FfnArgs &a, cudaStream_t s);
+cudaError_t launch_ffn_tc_bf16(const FfnArgs &a, cudaStream_t s);
+cudaError_t launch_ffn_q4(const FfnArgs &a, cudaStream_t s);
+
+cudaError_t launch_combine(const moe_config &c, const void *y_perm, const int32_t *slot_row,
+                           const float *topk_w, const void *shared_out, void *out,
+                           cudaStream_t s);
+
+}  // namespace moe

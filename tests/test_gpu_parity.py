@@ -1,0 +1,188 @@
+"""CUDA path vs the oracle, through the C ABI, on seeded inputs.
+
+Bars (from the layer's statement of the problem):
+  expert ids, offsets, permutation and drop set bit-exact (ids on tokens
+  whose k-th vs (k+1)-th score margin exceeds 1e-4); routing weights within
+  1e-6 relative; prob_sum within 1e-5 relative; layer output
+  max|err| / max|ref| <= 2e-2 (bf16) or 1e-5 (fp32); aux loss 1e-5 relative.
+"""
+import numpy as np
+import pytest
+import torch
+
+from gpu_harness import (AUX_RTOL, Run, check_aux, check_dispatch, check_output, check_route,
+                         sample_tokens)
+from mixture_experts_layer_41_b200 import api
+from mixture_experts_layer_41_b200.inputs import workload
+from moe_cases import oracle_route
+
+pytestmark = pytest.mark.gpu
+
+# Reduced sizes that the oracle finishes in seconds; each spans several
+# 128-row tiles with a ragged tail, several N tiles and K blocks.
+SMALL = {
+    "tiny_fp32": workload("tiny_fp32"),
+    "mixtral_small": workload("mixtral_prefill", T=700, d=512, F=640),
+    "switch_small": workload("switch_top1", T=1024, d=256, F=512, E=16),
+    "deepseek_small": workload("deepseek_v3", T=512, d=448, F=256, E=32, n_group=8, topk_group=4,
+                               shared_F=256),
+    "decode_small": workload("decode_q4", T=16, d=256, F=128, E=16, k=4),
+    "ragged_nk": workload("mixtral_prefill", T=333, d=200, F=136, E=4, k=2),
+    "relu_ragged_nk": workload("switch_top1", T=257, d=136, F=264, E=8, k=2, capacity_factor=1.25),
+    "fp32_swiglu": workload("tiny_fp32", T=97, d=24, F=40, E=6, k=3, act="swiglu", capacity_factor=0.0),
+}
+
+
+@pytest.fixture(autouse=True)
+def _cuda():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA GPU")
+    yield
+
+
+@pytest.mark.parametrize("name", sorted(SMALL))
+def test_staged_parity(name):
+    w = SMALL[name]
+    run = Run(w, seed=1).staged()
+    assert run.status() == 0
+    r = oracle_route(w, run.inp)
+    info = check_route(run, r)
+    check_dispatch(run)
+    check_output(run, routing="gpu")
+    if info["n_unsafe"] == 0:
+        check_output(run, routing="oracle")
+    assert check_aux(run, r) <= AUX_RTOL
+
+
+@pytest.mark.parametrize("name", sorted(SMALL))
+def test_forward_matches_staged_and_is_deterministic(name):
+    w = SMALL[name]
+    run = Run(w, seed=2).staged()
+    staged = run.out.clone()
+    a = run.forward(torch.empty_like(run.out))
+    b = run.forward(torch.empty_like(run.out))
+    assert run.status() == 0
+    assert torch.equal(a.view(torch.int16) if a.dtype == torch.bfloat16 else a,
+                       b.view(torch.int16) if b.dtype == torch.bfloat16 else b)
+    assert torch.equal(a.float(), staged.float())
+
+
+def test_tiny_fp32_exact_recipe():
+    """The tiny fp32 layer exactly as specified (numpy default_rng(0) inputs)."""
+    w = SMALL["tiny_fp32"]
+    run = Run(w, seed=0)
+    run.forward()
+    assert run.status() == 0
+    r = oracle_route(w, run.inp)
+    check_route(run, r)
+    check_dispatch(run)
+    check_output(run, routing="oracle")
+    assert check_aux(run, r) <= AUX_RTOL
+    assert int(run.stats["dropped"][0]) >= 0
+
+
+EDGE = {
+    "single_token": workload("mixtral_prefill", T=1, d=128, F=256, E=4, k=2),
+    "k_equals_E": workload("mixtral_prefill", T=130, d=64, F=128, E=2, k=2),
+    "capacity_one": workload("switch_top1", T=3, d=64, F=128, E=4, k=1, capacity_factor=1.0,
+                             logit_bias="none"),
+    "fp32_k_equals_E": workload("tiny_fp32", T=33, E=3, k=3),
+    "sigmoid_one_group": workload("deepseek_v3", T=64, d=64, F=128, E=16, n_group=1, topk_group=1, k=4,
+                                  shared_F=0),
+    "sigmoid_all_groups": workload("deepseek_v3", T=64, d=64, F=128, E=16, n_group=4, topk_group=4, k=4,
+                                   shared_F=128),
+    "no_norm_softmax": workload("mixtral_prefill", T=200, d=64, F=128, E=8, k=3, norm_topk_prob=False),
+}
+
+
+@pytest.mark.parametrize("name", sorted(EDGE))
+def test_edge_cases(name):
+    w = EDGE[name]
+    run = Run(w, seed=3).staged()
+    assert run.status() == 0
+    r = oracle_route(w, run.inp)
+    check_route(run, r)
+    check_dispatch(run)
+    check_output(run, routing="gpu")
+
+
+def test_all_tokens_one_expert_and_empty_experts():
+    """A hot expert takes every token (many tiles of one group) while other
+    experts get no rows; with cf = 1 most of its slots are dropped."""
+    w = workload("switch_top1", T=600, d=256, F=256, E=8, k=1, capacity_factor=0.0, logit_bias="none")
+    inp_run = Run(w, seed=4)
+    bias = torch.zeros(8, device="cuda")
+    bias[5] = 100.0
+    inp_run.bias = bias
+    inp_run.inp["logit_bias"] = bias
+    inp_run.staged()
+    assert inp_run.status() == 0
+    assert (inp_run.ids == 5).all()
+    check_dispatch(inp_run)
+    check_output(inp_run, routing="gpu")
+    w2 = w.with_(capacity_factor=1.0)
+    run2 = Run(w2, seed=4)
+    run2.bias = bias
+    run2.inp["logit_bias"] = bias
+    run2.staged()
+    d = check_dispatch(run2)
+    assert d["dropped"] == 600 - 75
+    check_output(run2, routing="gpu")
+    # dropped tokens get exactly zero
+    slot = run2.slot_row.cpu().numpy()
+    out = run2.out.float().cpu().numpy()
+    assert np.all(out[(slot < 0).all(axis=1)] == 0.0)
+
+
+def test_bad_ids_are_reported_not_faulted():
+    w = SMALL["mixtral_small"]
+    run = Run(w, seed=5)
+    c = run.cfg
+    ids = torch.zeros((w.T, w.k), dtype=torch.int32, device="cuda")
+    ids[:, 1] = 1
+    ids[3, 1] = 99          # out of range
+    api.moe_permute(c, run.inp["x"], ids, run.wts, run.offsets, run.perm_token, run.perm_w, run.slot_row,
+                    run.x_perm, run.stats, run.ws)
+    assert run.status() != 0
+    ids[3, 1] = 0           # duplicate of slot 0
+    api.moe_permute(c, run.inp["x"], ids, run.wts, run.offsets, run.perm_token, run.perm_w, run.slot_row,
+                    run.x_perm, run.stats, run.ws)
+    assert run.status() != 0
+    ids[3, 1] = 1
+    api.moe_permute(c, run.inp["x"], ids, run.wts, run.offsets, run.perm_token, run.perm_w, run.slot_row,
+                    run.x_perm, run.stats, run.ws)
+    assert run.status() == 0
+
+
+# ---------------------------------------------------------------- full sizes
+FULL = {
+    "mixtral_prefill": 48,
+    "switch_top1": 64,
+    "decode_q4": None,       # small enough for the whole output
+    "deepseek_v3": 12,
+}
+
+
+@pytest.mark.parametrize("name", list(FULL))
+def test_full_size_parity(name):
+    """Full-size workloads in the launch configuration the bench times
+    (moe_forward): routing and dispatch over the whole batch, the output on
+    a seeded token sample (all tokens for decode)."""
+    w = workload(name)
+    run = Run(w, seed=0)
+    run.forward()
+    assert run.status() == 0
+    r = oracle_route(w, run.inp)
+    check_route(run, r)
+    # moe_forward keeps the permutation in the workspace: recompute it staged
+    api.moe_permute(run.cfg, run.inp["x"], run.ids, run.wts, run.offsets, run.perm_token, run.perm_w,
+                    run.slot_row, run.x_perm, run.stats, run.ws)
+    torch.cuda.synchronize()
+    check_dispatch(run)
+    run.forward()
+    n = FULL[name]
+    toks = None if n is None else sample_tokens(run, n)
+    check_output(run, tokens=toks, routing="gpu")
+    assert check_aux(run, r) <= AUX_RTOL
+    del run
+    torch.cuda.empty_cache()
