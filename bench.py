@@ -300,6 +300,10 @@ def run_ours(args):
     # timed region: K whole-layer steps, phase events recorded on the launching stream
     K = args.steps
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(L.MOE_PHASE_COUNT)] for _ in range(K)]
+    for row in ev:              # torch creates the CUDA event on its first record
+        for e in row:
+            e.record(stream)
+    torch.cuda.synchronize()
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     sampler = ClockSampler(local) if rank == 0 or world == 1 else None
     barrier()

@@ -92,6 +92,9 @@ def moe_set_phase_events(events) -> None:
     if events is None:
         check(L.lib().moe_set_phase_events(None, 0), "moe_set_phase_events")
         return
+    for e in events:
+        if not e.cuda_event:
+            raise ValueError("record each event once before registering it (torch creates it lazily)")
     arr = (C.c_void_p * len(events))(*[e.cuda_event for e in events])
     check(L.lib().moe_set_phase_events(arr, len(events)), "moe_set_phase_events")
 

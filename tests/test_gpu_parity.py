@@ -70,12 +70,13 @@ def test_forward_matches_staged_and_is_deterministic(name):
 def test_tiny_fp32_exact_recipe():
     """The tiny fp32 layer exactly as specified (numpy default_rng(0) inputs)."""
     w = SMALL["tiny_fp32"]
-    run = Run(w, seed=0)
-    run.forward()
+    run = Run(w, seed=0).staged()
     assert run.status() == 0
     r = oracle_route(w, run.inp)
     check_route(run, r)
     check_dispatch(run)
+    run.forward()
+    assert run.status() == 0
     check_output(run, routing="oracle")
     assert check_aux(run, r) <= AUX_RTOL
     assert int(run.stats["dropped"][0]) >= 0
