@@ -207,6 +207,24 @@ moe_status moe_route(const moe_config *cfg, const void *x, const float *w_router
                      const float *router_bias, int32_t *topk_ids, float *topk_w,
                      float *prob_sum, void *ws, size_t ws_bytes, moe_stream_t stream);
 
+/* moe_route without a workspace, for callers that cannot allocate device
+ * memory (no page has a counterpart: this exists for library users only).
+ * Callers hosted by a framework that owns every device allocation, or on a
+ * path where an allocation and the synchronisation it can imply are not
+ * allowed, have no `ws` to pass.  Same arguments and results as moe_route,
+ * minus ws: the router's one scratch buffer (per-block partial probability
+ * sums) is a fixed device array inside the library, 1 MiB on every GPU that
+ * loads it, held until the process exits.
+ * Limit: ceil(T/32) * E <= 131072 (e.g. T = 16384 with E = 256); larger
+ * problems return MOE_ERR_UNSUPPORTED with the reason in moe_last_error().
+ * The first call on each device looks up that device's copy of the array
+ * (with the device current), so make it before any stream capture.  All
+ * calls share the array: calls that overlap on the GPU race, so serialise
+ * them.  Each call writes every entry it reads; nothing carries over. */
+moe_status moe_route_noalloc(const moe_config *cfg, const void *x, const float *w_router,
+                             const float *router_bias, int32_t *topk_ids, float *topk_w,
+                             float *prob_sum, moe_stream_t stream);
+
 /* Dispatch (blog moe_layer capacity loop; route_and_sort / SortedRouting).
  * A slot (t, j) with expert e is kept iff fewer than `capacity` slots of e
  * belong to earlier tokens (in-order dropping); capacity = moe_capacity(...),

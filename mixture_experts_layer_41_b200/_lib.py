@@ -85,6 +85,7 @@ SIGNATURES = {
     "moe_workspace_status": (C.c_int, [_P, _P]),
     "moe_set_phase_events": (C.c_int, [C.POINTER(C.c_void_p), C.c_int32]),
     "moe_route": (C.c_int, [_CFG, _P, _P, _P, _P, _P, _P, _P, C.c_size_t, _P]),
+    "moe_route_noalloc": (C.c_int, [_CFG, _P, _P, _P, _P, _P, _P, _P]),
     "moe_permute": (C.c_int, [_CFG, _P, _P, _P, _P, _P, _P, _P, _P, _S, _P, C.c_size_t, _P]),
     "moe_grouped_ffn": (C.c_int, [_CFG, _P, _P, _W, _P, _P, C.c_size_t, _P]),
     "moe_shared_expert": (C.c_int, [_CFG, _P, _W, _P, _P, C.c_size_t, _P]),

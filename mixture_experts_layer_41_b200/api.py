@@ -123,6 +123,16 @@ def moe_route(cfg, x, w_router, router_bias, topk_ids, topk_w, prob_sum, ws, str
                             _p(prob_sum), _p(ws), _nbytes(ws), _s(stream)), "moe_route")
 
 
+def moe_route_noalloc(cfg, x, w_router, router_bias, topk_ids, topk_w, prob_sum, stream=None):
+    """moe_route for callers that cannot allocate: no workspace argument; the
+    router's scratch is a fixed 1 MiB device array inside the library (see
+    include/moe.h for the size limit and the rule that overlapping calls race)."""
+    st = L.lib().moe_route_noalloc(C.byref(cfg), _p(x), _p(w_router), _p(router_bias), _p(topk_ids),
+                                   _p(topk_w), _p(prob_sum), _s(stream))
+    if st != L.MOE_OK:
+        raise L.MoEError(st, "moe_route_noalloc: " + L.lib().moe_last_error().decode())
+
+
 def moe_permute(cfg, x, topk_ids, topk_w, expert_offsets, perm_token, perm_w, slot_row, x_perm, stats, ws,
                 stream=None):
     st = _stats_struct(stats)

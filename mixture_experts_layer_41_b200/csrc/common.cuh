@@ -165,6 +165,9 @@ cudaError_t launch_ffn_simt_f32(const FfnArgs &a, cudaStream_t s);
 cudaError_t launch_ffn_tc_bf16(const FfnArgs &a, cudaStream_t s);
 cudaError_t launch_ffn_q4(const FfnArgs &a, cudaStream_t s);
 
+// Replaces the text moe_last_error() returns on this thread.
+void set_last_error_text(const char *text);
+
 cudaError_t launch_combine(const moe_config &c, const void *y_perm, const int32_t *slot_row,
                            const float *topk_w, const void *shared_out, void *out,
                            cudaStream_t s);

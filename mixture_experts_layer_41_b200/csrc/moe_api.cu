@@ -146,6 +146,8 @@ moe_status do_shared(const moe_config &c, const void *x, const moe_weights *w, v
 
 }  // namespace
 
+void moe::set_last_error_text(const char *text) { set_error("%s%s", text); }
+
 extern "C" {
 
 int64_t moe_capacity(int32_t num_tokens, int32_t top_k, int32_t num_experts, float capacity_factor) {
