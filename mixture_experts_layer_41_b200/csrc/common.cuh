@@ -37,10 +37,13 @@ __device__ __forceinline__ void record_status(int *status, int code) {
   atomicCAS(status, 0, code);
 }
 
+size_t route_logits_bytes(const moe_config &c);   // defined in router.cu
+
 // ---------------------------------------------------------------- workspace
 struct WsLayout {
   size_t status;       // int32[64]
   size_t route_part;   // double[nb_route][E]
+  size_t route_logits; // double[ks][T][E] (split router pass only)
   size_t blk_counts;   // int32[nb_perm][E]
   size_t blk_base;     // int32[nb_perm][E]
   size_t local_rank;   // int32[T*k]
@@ -90,6 +93,7 @@ inline WsLayout ws_layout(const moe_config &c) {
   const size_t slots = T * K;
   L.status = take(256);
   L.route_part = take(sizeof(double) * route_blocks(c) * E);
+  L.route_logits = take(route_logits_bytes(c));
   L.blk_counts = take(sizeof(int32_t) * perm_blocks(c) * E);
   L.blk_base = take(sizeof(int32_t) * perm_blocks(c) * E);
   L.local_rank = take(sizeof(int32_t) * slots);
@@ -130,9 +134,21 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 }
 
 // ---------------------------------------------------------------- launchers (one per kernel file)
+// Router launch shape.  split: the logits are first computed in `ks` slices
+// of the hidden dimension (float64 partials in the workspace) and summed by a
+// selection pass -- for batches too small to fill the GPU with whole rows.
+struct RoutePlan {
+  bool split;
+  int ks, kchunk;
+  int tpw;          // tokens per warp of the tiled kernel (4 or 8)
+};
+RoutePlan route_plan(const moe_config &c, bool allow_split);
+
+// logits == nullptr forbids the split pass (no workspace for it).
 cudaError_t launch_route(const moe_config &c, const void *x, const float *w_router,
                          const float *router_bias, int32_t *topk_ids, float *topk_w,
-                         double *route_part, float *prob_sum, cudaStream_t s);
+                         double *route_part, float *prob_sum, cudaStream_t s,
+                         double *logits = nullptr);
 
 cudaError_t launch_permute(const moe_config &c, const void *x, const int32_t *topk_ids,
                            const float *topk_w, int64_t capacity, int32_t *expert_offsets,

@@ -87,7 +87,9 @@ cudaError_t run_ffn(const FfnArgs &a, cudaStream_t s) {
 moe_status do_route(const moe_config &c, const void *x, const float *w_router, const float *bias,
                     int32_t *ids, float *wts, float *prob_sum, void *ws, cudaStream_t s) {
   const WsLayout L = ws_layout(c);
-  cudaError_t err = launch_route(c, x, w_router, bias, ids, wts, ws_ptr<double>(ws, L.route_part), prob_sum, s);
+  cudaError_t err = launch_route(c, x, w_router, bias, ids, wts, ws_ptr<double>(ws, L.route_part), prob_sum, s,
+                                 L.route_logits != L.total && route_logits_bytes(c) ? ws_ptr<double>(ws, L.route_logits)
+                                                                                   : nullptr);
   return err == cudaSuccess ? MOE_OK : cuda_fail(err, "moe_route");
 }
 

@@ -6,14 +6,24 @@
 // sigmoid scores, selection = score + bias, groups ranked by the sum of their
 // two best selection scores, routed scaling).
 //
-// One block = 32 tokens x all E experts, 8 warps.  Warp w owns tokens
-// 4w..4w+3; lane l owns experts l, l+32, ... (EPL = ceil(E/32) of them), so
-// after the dot products each warp holds every logit of its tokens in
-// registers and the selection runs on warp shuffles with no shared-memory
-// round trip.  Logits: fp32 products summed over runs of 8 elements, the runs
-// added in float64 (keeps the logit error near 1e-7 at d = 7168 where a
-// straight fp32 sum would reach ~1e-6).  Scores, selection and weights are
-// computed in float64 and rounded to float32 on the store.
+// Logits are fp32 products summed over runs of 8 consecutive elements, the
+// runs added in float64 (keeps the logit error near 1e-7 at d = 7168, where a
+// straight fp32 sum reaches ~1e-6); scores, selection and weights are float64
+// and rounded to float32 on the store.  Three shapes:
+//   route_rows    E <= 16: one warp per 4 tokens, lanes split the hidden
+//                 dimension with 16-byte loads, W_r read through L1; the
+//                 E logits of a token are warp all-reduced, lane e owns e.
+//   route_tiled   E > 16: a block owns 8*TPW tokens x all E experts; x and W_r
+//                 chunks of 32 elements are staged in shared memory (k-major)
+//                 from registers prefetched one chunk ahead; lane l owns
+//                 experts l, l+32, ...  With SPLIT the block covers one slice
+//                 of the hidden dimension and writes float64 partial logits.
+//   route_select  E > 16 after a SPLIT pass: sums the partial logits in a
+//                 fixed order and selects (used when T is too small to fill
+//                 the GPU with whole-row blocks, e.g. decode).
+// Every selecting block covers 32-token groups and writes one float64
+// probability sum per (group, expert); route_finalize adds the groups in
+// order, so prob_sum is deterministic.
 #include "common.cuh"
 
 #include <math.h>
@@ -21,9 +31,9 @@
 namespace moe {
 namespace {
 
-constexpr int KC = 32;      // reduction chunk staged in shared memory
+constexpr int KC = 32;      // hidden-dimension chunk staged in shared memory
 constexpr int RUN = 8;      // fp32 run length before the float64 add
-constexpr int TPW = 4;      // tokens per warp
+constexpr int WARPS = kRouteThreads / 32;
 
 struct RouteParams {
   const void *x;
@@ -35,7 +45,9 @@ struct RouteParams {
   int n_group, topk_group;
   int32_t *ids;
   float *wts;
-  double *part;
+  double *part;      // [ceil(T/32)][E] probability sums per 32-token group
+  double *logits;    // [ks][T][E] partial logits (split path)
+  int ks, kchunk;    // split path: number of hidden slices and their length
 };
 
 __device__ __forceinline__ void argmax_merge(double &v, int &i, double ov, int oi) {
@@ -45,8 +57,8 @@ __device__ __forceinline__ void argmax_merge(double &v, int &i, double ov, int o
 __device__ __forceinline__ void warp_argmax(double &v, int &i) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) {
-    double ov = __shfl_xor_sync(0xffffffffu, v, o);
-    int oi = __shfl_xor_sync(0xffffffffu, i, o);
+    const double ov = __shfl_xor_sync(0xffffffffu, v, o);
+    const int oi = __shfl_xor_sync(0xffffffffu, i, o);
     argmax_merge(v, i, ov, oi);
   }
 }
@@ -63,16 +75,312 @@ __device__ __forceinline__ double warp_max(double v) {
   return v;
 }
 
-template <int EPL, bool BF16>
+// Scores, selection and weights of token t, whose logits (without bias) sit
+// in l[j] for expert lane + 32 j.  Adds the token's probabilities to psum.
+// wscr: this warp's shared scratch row of kMaxExperts doubles.
+template <int EPL>
+__device__ __forceinline__ void select_token(const RouteParams &p, int t, const double (&lg)[EPL],
+                                             double (&psum)[EPL], double *wscr, int lane) {
+  const int E = p.E;
+  double prob[EPL], score[EPL];
+  if (p.router == MOE_ROUTER_SOFTMAX_TOPK) {
+    double l[EPL];
+    double m = -INFINITY;
+#pragma unroll
+    for (int j = 0; j < EPL; ++j) {
+      const int e = lane + 32 * j;
+      l[j] = e < E ? lg[j] + (p.bias ? (double)p.bias[e] : 0.0) : -INFINITY;
+      m = fmax(m, l[j]);
+    }
+    m = warp_max(m);
+    double s = 0.0;
+#pragma unroll
+    for (int j = 0; j < EPL; ++j) {
+      prob[j] = (lane + 32 * j) < E ? exp(l[j] - m) : 0.0;
+      s += prob[j];
+    }
+    s = warp_sum(s);
+#pragma unroll
+    for (int j = 0; j < EPL; ++j) {
+      prob[j] = prob[j] / s;
+      score[j] = (lane + 32 * j) < E ? prob[j] : -INFINITY;
+    }
+  } else {
+#pragma unroll
+    for (int j = 0; j < EPL; ++j) {
+      const int e = lane + 32 * j;
+      if (e < E) {
+        prob[j] = 1.0 / (1.0 + exp(-lg[j]));
+        score[j] = prob[j] + (p.bias ? (double)p.bias[e] : 0.0);
+        wscr[e] = score[j];
+      } else {
+        prob[j] = 0.0;
+        score[j] = -INFINITY;
+      }
+    }
+    __syncwarp();
+    // group score = sum of the two largest selection scores in the group
+    const int G = E / p.n_group;
+    double gs = -INFINITY;
+    if (lane < p.n_group) {
+      double b1 = -INFINITY, b2 = -INFINITY;
+      for (int q = 0; q < G; ++q) {
+        const double v = wscr[lane * G + q];
+        if (v > b1) { b2 = b1; b1 = v; } else if (v > b2) { b2 = v; }
+      }
+      gs = b1 + b2;
+    }
+    __syncwarp();
+    uint32_t keep = 0;
+    for (int r = 0; r < p.topk_group; ++r) {
+      const bool live = lane < p.n_group && !((keep >> lane) & 1u);
+      double v = live ? gs : -INFINITY;
+      int gi = live ? lane : 0x7fffffff;
+      warp_argmax(v, gi);
+      keep |= 1u << (gi & 31);
+    }
+#pragma unroll
+    for (int j = 0; j < EPL; ++j) {
+      const int e = lane + 32 * j;
+      if (e < E && !((keep >> (e / G)) & 1u)) score[j] = -INFINITY;
+    }
+  }
+#pragma unroll
+  for (int j = 0; j < EPL; ++j) psum[j] += prob[j];
+
+  // top-k by score, ties to the lower expert index
+  uint32_t taken = 0;
+  int my_e = -1;
+  double my_w = 0.0;
+  for (int r = 0; r < p.k; ++r) {
+    double bv = -INFINITY;
+    int bi = 0x7fffffff;
+#pragma unroll
+    for (int j = 0; j < EPL; ++j) {
+      const int e = lane + 32 * j;
+      if (e < E && !((taken >> j) & 1u)) argmax_merge(bv, bi, score[j], e);
+    }
+    warp_argmax(bv, bi);
+    double wv = 0.0;
+#pragma unroll
+    for (int j = 0; j < EPL; ++j)
+      if (lane + 32 * j == bi) { wv = prob[j]; taken |= 1u << j; }
+    wv = __shfl_sync(0xffffffffu, wv, bi & 31);
+    if (lane == r) { my_e = bi; my_w = wv; }
+  }
+  const double tot = warp_sum(lane < p.k ? my_w : 0.0);
+  double wout;
+  if (p.router == MOE_ROUTER_SOFTMAX_TOPK) wout = p.norm ? my_w / fmax(tot, 1e-12) : my_w;
+  else wout = (p.norm ? my_w / (tot + 1e-20) : my_w) * p.scaling;
+  if (lane < p.k) {
+    p.ids[(size_t)t * p.k + lane] = my_e;
+    p.wts[(size_t)t * p.k + lane] = (float)wout;
+  }
+}
+
+// Per-warp probability sums -> one row per 32-token group, warps added in
+// order.  tok0_of_warp(w) gives the first token of warp w; every warp's
+// tokens lie inside one group.
+template <int EPL>
+__device__ __forceinline__ void write_prob_partials(const RouteParams &p, double *scratch, const double (&psum)[EPL],
+                                                    int block_tok0, int tokens_per_warp, int lane, int warp) {
+  __syncthreads();
+  const int E = p.E;
+#pragma unroll
+  for (int j = 0; j < EPL; ++j) {
+    const int e = lane + 32 * j;
+    if (e < E) scratch[warp * E + e] = psum[j];
+  }
+  __syncthreads();
+  const int warps_per_group = 32 / tokens_per_warp;
+  const int groups = (WARPS + warps_per_group - 1) / warps_per_group;
+  for (int i = threadIdx.x; i < groups * E; i += kRouteThreads) {
+    const int g = i / E, e = i % E;
+    const int grow = block_tok0 / 32 + g;
+    if (grow * 32 >= p.T) continue;
+    double s = 0.0;
+    for (int w = g * warps_per_group; w < (g + 1) * warps_per_group && w < WARPS; ++w) s += scratch[w * E + e];
+    p.part[(size_t)grow * E + e] = s;
+  }
+}
+
+// ---------------------------------------------------------------- E <= 16
+template <int EP, bool BF16>
 __global__ void __launch_bounds__(kRouteThreads)
-route_kernel(RouteParams p) {
-  extern __shared__ __align__(16) unsigned char smem_raw[];
-  float *xs = reinterpret_cast<float *>(smem_raw);                  // [32][KC+1]
-  float *wsm = xs + kRouteTokens * (KC + 1);                         // [E][KC+1]
-  double *gscr = reinterpret_cast<double *>(smem_raw);               // reused after the dot loop
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int t0 = blockIdx.x * kRouteTokens;
+route_rows(RouteParams p) {
+  __shared__ double scratch[WARPS * 16];       // per-warp probability sums
+  __shared__ double wscr_all[WARPS * 32];      // per-warp selection scores (sigmoid groups)
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int E = p.E, d = p.d;
+  const int t0 = blockIdx.x * kRouteTokens + warp * 4;
+  double acc[4][EP];
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int e = 0; e < EP; ++e) acc[i][e] = 0.0;
+
+  constexpr int V = BF16 ? 8 : 4;   // elements per step and lane
+  const bool vec = (d % V) == 0;
+  if (vec) {
+    for (int k = lane * V; k < d; k += 32 * V) {
+      float xv[4][V];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int t = t0 + i;
+        if (t < p.T) {
+          if (BF16) {
+            const uint4 u = __ldg(reinterpret_cast<const uint4 *>(
+                static_cast<const uint16_t *>(p.x) + (size_t)t * d + k));
+            const uint32_t q[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+              xv[i][2 * c] = __uint_as_float(q[c] << 16);
+              xv[i][2 * c + 1] = __uint_as_float(q[c] & 0xffff0000u);
+            }
+          } else {
+            const float4 f = __ldg(reinterpret_cast<const float4 *>(
+                static_cast<const float *>(p.x) + (size_t)t * d + k));
+            xv[i][0] = f.x; xv[i][1] = f.y; xv[i][2] = f.z; xv[i][3] = f.w;
+          }
+        } else {
+#pragma unroll
+          for (int c = 0; c < V; ++c) xv[i][c] = 0.f;
+        }
+      }
+#pragma unroll
+      for (int e = 0; e < EP; ++e) {
+        if (e < E) {
+          float wv[V];
+          const float4 a = __ldg(reinterpret_cast<const float4 *>(p.w + (size_t)e * d + k));
+          wv[0] = a.x; wv[1] = a.y; wv[2] = a.z; wv[3] = a.w;
+          if constexpr (V == 8) {
+            const float4 b = __ldg(reinterpret_cast<const float4 *>(p.w + (size_t)e * d + k + 4));
+            wv[4] = b.x; wv[5] = b.y; wv[6] = b.z; wv[7] = b.w;
+          }
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            float run = 0.f;
+#pragma unroll
+            for (int c = 0; c < V; ++c) run = fmaf(xv[i][c], wv[c], run);
+            acc[i][e] += (double)run;
+          }
+        }
+      }
+    }
+  } else {
+    // fp32 rows whose length is not a multiple of 4: one element per step
+    for (int k = lane; k < d; k += 32) {
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int t = t0 + i;
+        const float xv = t < p.T ? static_cast<const float *>(p.x)[(size_t)t * d + k] : 0.f;
+#pragma unroll
+        for (int e = 0; e < EP; ++e)
+          if (e < E) acc[i][e] += (double)(xv * __ldg(p.w + (size_t)e * d + k));
+      }
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int e = 0; e < EP; ++e) acc[i][e] = warp_sum(acc[i][e]);
+
+  double psum[1] = {0.0};
+  double *wscr = wscr_all + warp * 32;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int t = t0 + i;
+    if (t < p.T) {
+      double lg[1];
+      lg[0] = 0.0;
+#pragma unroll
+      for (int e = 0; e < EP; ++e)
+        if (e == lane) lg[0] = acc[i][e];
+      select_token<1>(p, t, lg, psum, wscr, lane);
+    }
+  }
+  write_prob_partials<1>(p, scratch, psum, blockIdx.x * kRouteTokens, 4, lane, warp);
+}
+
+// ---------------------------------------------------------------- E > 16
+template <int EPL, int TPW, bool BF16, bool SPLIT>
+__global__ void __launch_bounds__(kRouteThreads)
+route_tiled(RouteParams p) {
+  constexpr int TM = WARPS * TPW;
+  constexpr int XS = TM + 4;                          // xs row stride (floats), keeps 16-byte rows
+  constexpr int XV = BF16 ? 8 : 4;                    // x elements per 16-byte vector
+  constexpr int XN = (TM * KC / XV + kRouteThreads - 1) / kRouteThreads;
+  constexpr int WN = (kMaxExperts * KC / 4) / kRouteThreads;   // float4 per thread at E = 256
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  float *xs = reinterpret_cast<float *>(smem_raw);    // [KC][XS]   x chunk, k-major
+  float *wsm = xs + KC * XS;                          // [KC][E+1]  W_r chunk, k-major
+  double *dscr = reinterpret_cast<double *>(smem_raw);   // reused after the dot loop
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int E = p.E, d = p.d, WSTR = E + 1;
+  const int t0 = blockIdx.x * TM;
+  int kbeg = 0, kend = d;
+  if (SPLIT) {
+    kbeg = blockIdx.y * p.kchunk;
+    kend = min(d, kbeg + p.kchunk);
+  }
+  const int wvec = E * (KC / 4);                      // float4 of W_r per chunk
+
+  uint4 xr[XN];
+  float4 wr[WN];
+  auto gload = [&](int k0) {
+#pragma unroll
+    for (int i = 0; i < XN; ++i) {
+      const int v = tid + i * kRouteThreads;
+      const int tok = v / (KC / XV), q = v % (KC / XV);
+      const int t = t0 + tok, kg = k0 + q * XV;
+      xr[i] = make_uint4(0u, 0u, 0u, 0u);
+      if (tok < TM && t < p.T && kg < kend) {
+        if (BF16) xr[i] = __ldg(reinterpret_cast<const uint4 *>(static_cast<const uint16_t *>(p.x) + (size_t)t * d + kg));
+        else xr[i] = __ldg(reinterpret_cast<const uint4 *>(static_cast<const float *>(p.x) + (size_t)t * d + kg));
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < WN; ++i) {
+      const int v = tid + i * kRouteThreads;
+      const int e = v / (KC / 4), q = v % (KC / 4);
+      const int kg = k0 + q * 4;
+      wr[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (v < wvec && kg < kend) wr[i] = __ldg(reinterpret_cast<const float4 *>(p.w + (size_t)e * d + kg));
+    }
+  };
+  auto sstore = [&]() {
+#pragma unroll
+    for (int i = 0; i < XN; ++i) {
+      const int v = tid + i * kRouteThreads;
+      const int tok = v / (KC / XV), q = v % (KC / XV);
+      if (tok < TM) {
+        if (BF16) {
+          const uint32_t u[4] = {xr[i].x, xr[i].y, xr[i].z, xr[i].w};
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            xs[(q * 8 + 2 * c) * XS + tok] = __uint_as_float(u[c] << 16);
+            xs[(q * 8 + 2 * c + 1) * XS + tok] = __uint_as_float(u[c] & 0xffff0000u);
+          }
+        } else {
+          xs[(q * 4 + 0) * XS + tok] = __uint_as_float(xr[i].x);
+          xs[(q * 4 + 1) * XS + tok] = __uint_as_float(xr[i].y);
+          xs[(q * 4 + 2) * XS + tok] = __uint_as_float(xr[i].z);
+          xs[(q * 4 + 3) * XS + tok] = __uint_as_float(xr[i].w);
+        }
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < WN; ++i) {
+      const int v = tid + i * kRouteThreads;
+      if (v < wvec) {
+        const int e = v / (KC / 4), q = v % (KC / 4);
+        wsm[(q * 4 + 0) * WSTR + e] = wr[i].x;
+        wsm[(q * 4 + 1) * WSTR + e] = wr[i].y;
+        wsm[(q * 4 + 2) * WSTR + e] = wr[i].z;
+        wsm[(q * 4 + 3) * WSTR + e] = wr[i].w;
+      }
+    }
+  };
 
   double acc[TPW][EPL];
 #pragma unroll
@@ -80,22 +388,11 @@ route_kernel(RouteParams p) {
 #pragma unroll
     for (int j = 0; j < EPL; ++j) acc[i][j] = 0.0;
 
-  for (int k0 = 0; k0 < d; k0 += KC) {
-    // stage x[t0:t0+32, k0:k0+KC] and W_r[:, k0:k0+KC] as fp32
-    for (int i = tid; i < kRouteTokens * KC; i += kRouteThreads) {
-      const int tok = i / KC, kk = i % KC, t = t0 + tok, kg = k0 + kk;
-      float v = 0.f;
-      if (t < p.T && kg < d) {
-        if (BF16) v = bf16_to_f32(reinterpret_cast<const uint16_t *>(p.x)[(size_t)t * d + kg]);
-        else v = reinterpret_cast<const float *>(p.x)[(size_t)t * d + kg];
-      }
-      xs[tok * (KC + 1) + kk] = v;
-    }
-    for (int i = tid; i < E * KC; i += kRouteThreads) {
-      const int e = i / KC, kk = i % KC, kg = k0 + kk;
-      wsm[e * (KC + 1) + kk] = kg < d ? __ldg(p.w + (size_t)e * d + kg) : 0.f;
-    }
+  if (kbeg < kend) gload(kbeg);
+  for (int k0 = kbeg; k0 < kend; k0 += KC) {
+    sstore();
     __syncthreads();
+    if (k0 + KC < kend) gload(k0 + KC);      // next chunk in flight during the FMAs
 #pragma unroll
     for (int r0 = 0; r0 < KC; r0 += RUN) {
       float run[TPW][EPL];
@@ -106,12 +403,20 @@ route_kernel(RouteParams p) {
 #pragma unroll
       for (int kk = r0; kk < r0 + RUN; ++kk) {
         float xv[TPW], wv[EPL];
+        if (TPW % 4 == 0) {
 #pragma unroll
-        for (int i = 0; i < TPW; ++i) xv[i] = xs[(warp * TPW + i) * (KC + 1) + kk];
+          for (int m = 0; m < TPW / 4; ++m) {
+            const float4 f = *reinterpret_cast<const float4 *>(xs + kk * XS + warp * TPW + 4 * m);
+            xv[4 * m] = f.x; xv[4 * m + 1] = f.y; xv[4 * m + 2] = f.z; xv[4 * m + 3] = f.w;
+          }
+        } else {
+#pragma unroll
+          for (int i = 0; i < TPW; ++i) xv[i] = xs[kk * XS + warp * TPW + i];
+        }
 #pragma unroll
         for (int j = 0; j < EPL; ++j) {
           const int e = lane + 32 * j;
-          wv[j] = e < E ? wsm[e * (KC + 1) + kk] : 0.f;
+          wv[j] = e < E ? wsm[kk * WSTR + e] : 0.f;
         }
 #pragma unroll
         for (int i = 0; i < TPW; ++i)
@@ -126,130 +431,59 @@ route_kernel(RouteParams p) {
     __syncthreads();
   }
 
-  // ------------------------------------------------------------ selection
+  if (SPLIT) {
+#pragma unroll
+    for (int i = 0; i < TPW; ++i) {
+      const int t = t0 + warp * TPW + i;
+      if (t < p.T) {
+#pragma unroll
+        for (int j = 0; j < EPL; ++j) {
+          const int e = lane + 32 * j;
+          if (e < E) p.logits[((size_t)blockIdx.y * p.T + t) * E + e] = acc[i][j];
+        }
+      }
+    }
+    return;
+  }
+
   double psum[EPL];
 #pragma unroll
   for (int j = 0; j < EPL; ++j) psum[j] = 0.0;
-  double *wscr = gscr + warp * kMaxExperts;   // per-warp scratch row (sigmoid groups)
-
-#pragma unroll 1
+  double *wscr = dscr + warp * kMaxExperts;
+#pragma unroll
   for (int i = 0; i < TPW; ++i) {
     const int t = t0 + warp * TPW + i;
-    if (t >= p.T) break;                       // warp-uniform
-    double prob[EPL], score[EPL];
-    if (p.router == MOE_ROUTER_SOFTMAX_TOPK) {
-      double l[EPL];
-      double m = -INFINITY;
+    if (t < p.T) select_token<EPL>(p, t, acc[i], psum, wscr, lane);
+  }
+  write_prob_partials<EPL>(p, dscr, psum, t0, TPW, lane, warp);
+}
+
+template <int EPL>
+__global__ void __launch_bounds__(kRouteThreads)
+route_select(RouteParams p) {
+  __shared__ double dscr[WARPS * kMaxExperts];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int E = p.E;
+  const int t0 = blockIdx.x * kRouteTokens + warp * 4;
+  double psum[EPL];
 #pragma unroll
-      for (int j = 0; j < EPL; ++j) {
-        const int e = lane + 32 * j;
-        l[j] = e < E ? acc[i][j] + (p.bias ? (double)p.bias[e] : 0.0) : -INFINITY;
-        m = fmax(m, l[j]);
-      }
-      m = warp_max(m);
+  for (int j = 0; j < EPL; ++j) psum[j] = 0.0;
+  double *wscr = dscr + warp * kMaxExperts;
+  for (int i = 0; i < 4; ++i) {
+    const int t = t0 + i;
+    if (t >= p.T) break;
+    double lg[EPL];
+#pragma unroll
+    for (int j = 0; j < EPL; ++j) {
+      const int e = lane + 32 * j;
       double s = 0.0;
-#pragma unroll
-      for (int j = 0; j < EPL; ++j) {
-        prob[j] = (lane + 32 * j) < E ? exp(l[j] - m) : 0.0;
-        s += prob[j];
-      }
-      s = warp_sum(s);
-#pragma unroll
-      for (int j = 0; j < EPL; ++j) {
-        prob[j] = prob[j] / s;
-        score[j] = (lane + 32 * j) < E ? prob[j] : -INFINITY;
-      }
-    } else {
-#pragma unroll
-      for (int j = 0; j < EPL; ++j) {
-        const int e = lane + 32 * j;
-        if (e < E) {
-          prob[j] = 1.0 / (1.0 + exp(-acc[i][j]));
-          score[j] = prob[j] + (p.bias ? (double)p.bias[e] : 0.0);
-          wscr[e] = score[j];
-        } else {
-          prob[j] = 0.0;
-          score[j] = -INFINITY;
-        }
-      }
-      __syncwarp();
-      // group score = sum of the two largest selection scores in the group
-      const int G = E / p.n_group;
-      double gs = -INFINITY;
-      if (lane < p.n_group) {
-        double b1 = -INFINITY, b2 = -INFINITY;
-        for (int q = 0; q < G; ++q) {
-          const double v = wscr[lane * G + q];
-          if (v > b1) { b2 = b1; b1 = v; } else if (v > b2) { b2 = v; }
-        }
-        gs = b1 + b2;
-      }
-      __syncwarp();
-      uint32_t keep = 0;
-      for (int r = 0; r < p.topk_group; ++r) {
-        double v = (keep >> lane) & 1u ? -INFINITY : gs;
-        int gi = lane < p.n_group && !((keep >> lane) & 1u) ? lane : 0x7fffffff;
-        if (lane >= p.n_group) v = -INFINITY;
-        warp_argmax(v, gi);
-        keep |= 1u << gi;
-      }
-#pragma unroll
-      for (int j = 0; j < EPL; ++j) {
-        const int e = lane + 32 * j;
-        if (e < E && !((keep >> (e / G)) & 1u)) score[j] = -INFINITY;
-      }
+      if (e < E)
+        for (int q = 0; q < p.ks; ++q) s += p.logits[((size_t)q * p.T + t) * E + e];
+      lg[j] = s;
     }
-    // psum over all tokens (softmax probability / raw sigmoid)
-#pragma unroll
-    for (int j = 0; j < EPL; ++j) psum[j] += prob[j];
-
-    // top-k by score, ties to the lower expert index
-    uint32_t taken = 0;
-    int my_e = -1;
-    double my_w = 0.0;
-    for (int r = 0; r < p.k; ++r) {
-      double bv = -INFINITY;
-      int bi = 0x7fffffff;
-#pragma unroll
-      for (int j = 0; j < EPL; ++j) {
-        const int e = lane + 32 * j;
-        if (e < E && !((taken >> j) & 1u)) argmax_merge(bv, bi, score[j], e);
-      }
-      warp_argmax(bv, bi);
-      double wv = 0.0;
-#pragma unroll
-      for (int j = 0; j < EPL; ++j)
-        if (lane + 32 * j == bi) { wv = prob[j]; taken |= 1u << j; }
-      wv = __shfl_sync(0xffffffffu, wv, bi & 31);
-      if (lane == r) { my_e = bi; my_w = wv; }
-    }
-    const double tot = warp_sum(lane < p.k ? my_w : 0.0);
-    double wout;
-    if (p.router == MOE_ROUTER_SOFTMAX_TOPK) {
-      wout = p.norm ? my_w / fmax(tot, 1e-12) : my_w;
-    } else {
-      wout = (p.norm ? my_w / (tot + 1e-20) : my_w) * p.scaling;
-    }
-    if (lane < p.k) {
-      p.ids[(size_t)t * p.k + lane] = my_e;
-      p.wts[(size_t)t * p.k + lane] = (float)wout;
-    }
+    select_token<EPL>(p, t, lg, psum, wscr, lane);
   }
-
-  // per-block probability sums in a fixed order
-  __syncthreads();
-  double *part = gscr;  // [8][E]
-#pragma unroll
-  for (int j = 0; j < EPL; ++j) {
-    const int e = lane + 32 * j;
-    if (e < E) part[warp * E + e] = psum[j];
-  }
-  __syncthreads();
-  for (int e = tid; e < E; e += kRouteThreads) {
-    double s = 0.0;
-    for (int w = 0; w < kRouteThreads / 32; ++w) s += part[w * E + e];
-    p.part[(size_t)blockIdx.x * E + e] = s;
-  }
+  write_prob_partials<EPL>(p, dscr, psum, blockIdx.x * kRouteTokens, 4, lane, warp);
 }
 
 __global__ void route_finalize(const double *part, int nb, int E, float *prob_sum) {
@@ -260,32 +494,88 @@ __global__ void route_finalize(const double *part, int nb, int E, float *prob_su
   prob_sum[e] = (float)s;
 }
 
-template <int EPL, bool BF16>
-cudaError_t launch_variant(const RouteParams &p, int nb, cudaStream_t s) {
-  const size_t stage = sizeof(float) * (size_t)(kRouteTokens + p.E) * (KC + 1);
-  const size_t scratch = sizeof(double) * (size_t)(kRouteThreads / 32) * kMaxExperts;
+template <int EPL, int TPW, bool BF16, bool SPLIT>
+cudaError_t launch_tiled(const RouteParams &p, dim3 grid, cudaStream_t s) {
+  constexpr int TM = WARPS * TPW;
+  const size_t stage = sizeof(float) * ((size_t)KC * (TM + 4) + (size_t)KC * (p.E + 1));
+  const size_t scratch = sizeof(double) * (size_t)WARPS * kMaxExperts;
   const size_t smem = stage > scratch ? stage : scratch;
-  auto kern = route_kernel<EPL, BF16>;
+  auto kern = route_tiled<EPL, TPW, BF16, SPLIT>;
   cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (err != cudaSuccess) return err;
-  kern<<<nb, kRouteThreads, smem, s>>>(p);
+  kern<<<grid, kRouteThreads, smem, s>>>(p);
   return cudaGetLastError();
 }
 
+template <int EPL, bool BF16>
+cudaError_t launch_wide(const RouteParams &p, const RoutePlan &plan, cudaStream_t s) {
+  if (plan.split) {
+    const dim3 grid((p.T + kRouteTokens - 1) / kRouteTokens, plan.ks);
+    cudaError_t err = launch_tiled<EPL, 4, BF16, true>(p, grid, s);
+    if (err != cudaSuccess) return err;
+    route_select<EPL><<<(p.T + kRouteTokens - 1) / kRouteTokens, kRouteThreads, 0, s>>>(p);
+    return cudaGetLastError();
+  }
+  if constexpr (EPL <= 4) {
+    if (plan.tpw == 8) return launch_tiled<EPL, 8, BF16, false>(p, dim3((p.T + 63) / 64), s);
+  }
+  return launch_tiled<EPL, 4, BF16, false>(p, dim3((p.T + 31) / 32), s);
+}
+
 template <bool BF16>
-cudaError_t launch_epl(const RouteParams &p, int nb, cudaStream_t s) {
-  const int epl = (p.E + 31) / 32;
-  if (epl <= 1) return launch_variant<1, BF16>(p, nb, s);
-  if (epl <= 2) return launch_variant<2, BF16>(p, nb, s);
-  if (epl <= 4) return launch_variant<4, BF16>(p, nb, s);
-  return launch_variant<8, BF16>(p, nb, s);
+cudaError_t launch_any(const RouteParams &p, const RoutePlan &plan, cudaStream_t s) {
+  const int nb32 = (p.T + kRouteTokens - 1) / kRouteTokens;
+  if (p.E <= 8) {
+    route_rows<8, BF16><<<nb32, kRouteThreads, 0, s>>>(p);
+    return cudaGetLastError();
+  }
+  if (p.E <= 16) {
+    route_rows<16, BF16><<<nb32, kRouteThreads, 0, s>>>(p);
+    return cudaGetLastError();
+  }
+  if (p.E <= 64) return launch_wide<2, BF16>(p, plan, s);
+  if (p.E <= 128) return launch_wide<4, BF16>(p, plan, s);
+  return launch_wide<8, BF16>(p, plan, s);
 }
 
 }  // namespace
 
+RoutePlan route_plan(const moe_config &c, bool allow_split) {
+  RoutePlan plan{};
+  plan.split = false;
+  plan.ks = 1;
+  plan.kchunk = c.hidden;
+  plan.tpw = 4;
+  if (c.num_experts <= 16) return plan;
+  const int nb32 = (c.num_tokens + kRouteTokens - 1) / kRouteTokens;
+  const int target = 2 * 148;
+  const bool vec_ok = c.act_dtype == MOE_BF16 ? (c.hidden % 8 == 0) : (c.hidden % 4 == 0);
+  if (allow_split && vec_ok && nb32 < 148 && c.hidden >= 2 * KC) {
+    int ks = (target + nb32 - 1) / nb32;
+    const int max_ks = c.hidden / KC;
+    ks = ks < max_ks ? ks : max_ks;
+    ks = ks < 64 ? ks : 64;
+    int kchunk = (c.hidden + ks - 1) / ks;
+    kchunk = (kchunk + KC - 1) / KC * KC;
+    ks = (c.hidden + kchunk - 1) / kchunk;
+    plan.split = ks > 1;
+    plan.ks = ks;
+    plan.kchunk = kchunk;
+  }
+  // 8 tokens per warp halves the shared-memory reads per FMA; with 8 experts
+  // per lane its accumulators no longer fit in registers.
+  if (!plan.split && c.num_experts > 64 && c.num_experts <= 128 && (c.num_tokens + 63) / 64 >= 148) plan.tpw = 8;
+  return plan;
+}
+
+size_t route_logits_bytes(const moe_config &c) {
+  const RoutePlan plan = route_plan(c, true);
+  return plan.split ? sizeof(double) * (size_t)plan.ks * c.num_tokens * c.num_experts : 0;
+}
+
 cudaError_t launch_route(const moe_config &c, const void *x, const float *w_router,
                          const float *router_bias, int32_t *topk_ids, float *topk_w,
-                         double *route_part, float *prob_sum, cudaStream_t s) {
+                         double *route_part, float *prob_sum, cudaStream_t s, double *logits) {
   RouteParams p;
   p.x = x;
   p.w = w_router;
@@ -302,9 +592,13 @@ cudaError_t launch_route(const moe_config &c, const void *x, const float *w_rout
   p.ids = topk_ids;
   p.wts = topk_w;
   p.part = route_part;
-  const int nb = route_blocks(c);
-  cudaError_t err = c.act_dtype == MOE_BF16 ? launch_epl<true>(p, nb, s) : launch_epl<false>(p, nb, s);
+  const RoutePlan plan = route_plan(c, logits != nullptr);
+  p.logits = logits;
+  p.ks = plan.ks;
+  p.kchunk = plan.kchunk;
+  cudaError_t err = c.act_dtype == MOE_BF16 ? launch_any<true>(p, plan, s) : launch_any<false>(p, plan, s);
   if (err != cudaSuccess) return err;
+  const int nb = route_blocks(c);
   route_finalize<<<(c.num_experts + 127) / 128, 128, 0, s>>>(route_part, nb, c.num_experts, prob_sum);
   return cudaGetLastError();
 }

@@ -187,3 +187,33 @@ def test_full_size_parity(name):
     assert check_aux(run, r) <= AUX_RTOL
     del run
     torch.cuda.empty_cache()
+
+
+# ---------------------------------------------------------------- router shapes
+ROUTER_SHAPES = {
+    # E <= 16: one warp per 4 tokens, lanes split the hidden dimension
+    "rows_e8_bf16": workload("mixtral_prefill", T=777, d=1032, F=64, E=8, k=2),
+    "rows_e13_sigmoid": workload("deepseek_v3", T=200, d=256, F=64, E=12, n_group=3, topk_group=2, k=3,
+                                 shared_F=0),
+    "rows_f32_odd_d": workload("tiny_fp32", T=50, d=21, F=8, E=5, k=2, act="relu", capacity_factor=0.0),
+    # E > 16, whole rows per block, 4 tokens per warp
+    "tiled_e64": workload("switch_top1", T=5000, d=512, F=64, E=64, k=1),
+    "tiled_e96": workload("mixtral_prefill", T=4800, d=256, F=64, E=96, k=6),
+    "tiled_e256_sigmoid": workload("deepseek_v3", T=4800, d=320, F=64, shared_F=0),
+    # 8 tokens per warp (E in (64, 128], many tokens)
+    "tiled8_e128": workload("mixtral_prefill", T=9500, d=192, F=64, E=128, k=4),
+    # hidden-dimension split + selection pass (few tokens)
+    "split_e128_decode": workload("decode_q4", T=40, d=1024, F=64, k=8, weight_format="dense"),
+    "split_e256_sigmoid": workload("deepseek_v3", T=70, d=2048, F=64, shared_F=0),
+    "split_e40_f32": workload("tiny_fp32", T=90, d=128, F=8, E=40, k=5, act="relu", capacity_factor=0.0),
+}
+
+
+@pytest.mark.parametrize("name", sorted(ROUTER_SHAPES))
+def test_router_shapes(name):
+    w = ROUTER_SHAPES[name]
+    run = Run(w, seed=6)
+    api.moe_route(run.cfg, run.inp["x"], run.inp["w_router"], run.bias, run.ids, run.wts, run.prob_sum, run.ws)
+    torch.cuda.synchronize()
+    assert run.status() == 0
+    check_route(run, oracle_route(w, run.inp))
