@@ -155,6 +155,19 @@ def layer_costs(w, R: int, touched: int) -> dict:
                 ffn2=dict(flops=f2, bytes=w3 + R * w.F * es + R * w.d * es))
 
 
+def kernels_per_step(w) -> int:
+    """Kernels of this library launched by one moe_forward."""
+    if w.E <= 16:
+        route = 2                                   # route_rows + route_finalize
+    else:
+        nb32 = (w.T + 31) // 32
+        route = 3 if (nb32 < 148 and w.d >= 64) else 2   # split pass adds route_select
+    permute = 3                                     # count, scan, scatter
+    ffn = 2                                         # two expert GEMM phases
+    shared = 2 if w.shared_F else 0
+    return route + permute + ffn + shared + 1       # + combine
+
+
 def source_hash(path: str) -> str:
     with open(path, "rb") as fh:
         return hashlib.sha256(fh.read()).hexdigest()[:16]
@@ -303,13 +316,48 @@ def run_ours(args):
     if st != 0:
         raise SystemExit(f"device status {st}: {api.moe_status_string(st)}")
 
-    # timed region: K whole-layer steps, phase events recorded on the launching stream
+    # Eager steps with phase events recorded inside moe_forward on the
+    # launching stream: the per-phase (per-kernel) times for the roofline.
     K = args.steps
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(L.MOE_PHASE_COUNT)] for _ in range(K)]
     for row in ev:              # torch creates the CUDA event on its first record
         for e in row:
             e.record(stream)
     torch.cuda.synchronize()
+    e_start, e_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    e_start.record(stream)
+    for i in range(K):
+        api.moe_set_phase_events(ev[i])
+        layer.forward(x)
+    e_end.record(stream)
+    torch.cuda.synchronize()
+    api.moe_set_phase_events(None)
+    eager_ms = e_start.elapsed_time(e_end) / K
+    phases = {}
+    names = ["route", "permute", "ffn1", "ffn2", "shared", "combine"]
+    for p, nm in enumerate(names, start=1):
+        phases[nm] = statistics.mean(ev[i][p - 1].elapsed_time(ev[i][p]) for i in range(K))
+
+    # Headline: the same step replayed from a CUDA graph (one capture of
+    # moe_forward: every kernel of the layer, launched without host overhead).
+    graph = None
+    try:
+        graph = torch.cuda.CUDAGraph()
+        side = torch.cuda.Stream()
+        side.wait_stream(stream)
+        with torch.cuda.stream(side):
+            layer.forward(x)
+        stream.wait_stream(side)
+        with torch.cuda.graph(graph, capture_error_mode="relaxed"):
+            layer.forward(x)
+        for _ in range(3):
+            graph.replay()
+        torch.cuda.synchronize()
+    except Exception as exc:  # noqa: BLE001
+        graph = None
+        print(f"cuda graph capture failed, timing eager launches: {exc}", file=sys.stderr)
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     sampler = ClockSampler(local) if rank == 0 or world == 1 else None
     barrier()
@@ -318,18 +366,18 @@ def run_ours(args):
         sampler.start()
     start.record(stream)
     for i in range(K):
-        api.moe_set_phase_events(ev[i])
-        layer.forward(x)
+        if graph is not None:
+            graph.replay()
+        else:
+            layer.forward(x)
     end.record(stream)
     torch.cuda.synchronize()
-    api.moe_set_phase_events(None)
     barrier()
     clocks = sampler.stop() if sampler else None
+    st = layer.status()
+    if st != 0:
+        raise SystemExit(f"device status {st}: {api.moe_status_string(st)}")
     ms = start.elapsed_time(end) / K
-    phases = {}
-    names = ["route", "permute", "ffn1", "ffn2", "shared", "combine"]
-    for p, nm in enumerate(names, start=1):
-        phases[nm] = statistics.mean(ev[i][p - 1].elapsed_time(ev[i][p]) for i in range(K))
     ms_t = torch.tensor([ms], device=dev)
     if world > 1:
         dist.all_reduce(ms_t, op=dist.ReduceOp.MAX)
@@ -373,7 +421,10 @@ def run_ours(args):
 
     peaks, peak_src = load_peaks()
     costs = layer_costs(w, R, touched)
-    tensor_peak = peaks["bf16_tflops"] * 1e12          # burst: kernels timed back to back, < 1 s
+    # The expert GEMMs are timed inside back-to-back layer steps that run long
+    # enough to reach the 1 kW power cap, so the tensor roofline is the
+    # sustained cuBLAS figure; the burst fraction is reported beside it.
+    tensor_peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]) * 1e12
     hbm_peak = peaks["hbm_gbs"] * 1e9
     # dominant kernel: the longer expert GEMM phase
     dom = "ffn1" if phases["ffn1"] >= phases["ffn2"] else "ffn2"
@@ -385,15 +436,16 @@ def run_ours(args):
                                ("ffn_simt.cu" if w.dtype == "f32" else "ffn_tc.cu"))
     traffic = recorded_traffic(kernel_file, f"{w.name}:{dom}")
     if t_tensor >= t_hbm and w.weight_format == "dense" and w.dtype == "bf16":
-        roof = {"bound": "tensor", "achieved": dk["flops"] / t_dom / 1e12, "peak": peaks["bf16_tflops"],
-                "unit": "TFLOP/s"}
+        roof = {"bound": "tensor", "achieved": dk["flops"] / t_dom / 1e12,
+                "peak": tensor_peak / 1e12, "unit": "TFLOP/s",
+                "frac_of_burst_peak": dk["flops"] / t_dom / 1e12 / peaks["bf16_tflops"]}
     else:
         roof = {"bound": "hbm", "achieved": dk["bytes"] / t_dom / 1e9, "peak": peaks["hbm_gbs"], "unit": "GB/s"}
     roof["frac"] = roof["achieved"] / roof["peak"]
     roof["traffic"] = traffic
     roof["kernel"] = {"ffn1": "grouped expert GEMM, phase 1 (gate/up or in)",
                       "ffn2": "grouped expert GEMM, phase 2 (down or out)"}[dom]
-    roof["peak_source"] = f"{peak_src} ({'burst' if roof['bound'] == 'tensor' else 'copy'})"
+    roof["peak_source"] = f"{peak_src} ({'bf16 GEMM, sustained' if roof['bound'] == 'tensor' else 'HBM copy'})"
     roof["algorithmic"] = {"flop_per_launch": dk["flops"], "bytes_per_launch": dk["bytes"],
                            "ms_per_launch": phases[dom]}
     t_layer_roof = max(costs["flops"] / tensor_peak, costs["bytes"] / hbm_peak)
@@ -416,7 +468,9 @@ def run_ours(args):
         "routing": {"rows": R, "touched_experts": touched, "dropped": dropped, "aux_raw": aux_raw, "aux": aux},
         "e2e": {"value": world * w.T / (e2e_ms * 1e-3), "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms, "matches_device_out": bool(same)},
-        "gpu_launches": K * (8 + (2 if w.shared_F else 0)),
+        "gpu_launches": K * kernels_per_step(w),
+        "launch": "cuda_graph" if graph is not None else "eager",
+        "eager_ms_per_step": eager_ms,
         "clocks": clocks,
     }
 

@@ -14,8 +14,8 @@
 //                 dimension with 16-byte loads, W_r read through L1; the
 //                 E logits of a token are warp all-reduced, lane e owns e.
 //   route_tiled   E > 16: a block owns 8*TPW tokens x all E experts; x and W_r
-//                 chunks of 32 elements are staged in shared memory (k-major)
-//                 from registers prefetched one chunk ahead; lane l owns
+//                 chunks of 32 elements are copied k-major into shared memory
+//                 with cp.async, double-buffered one chunk ahead; lane l owns
 //                 experts l, l+32, ...  With SPLIT the block covers one slice
 //                 of the hidden dimension and writes float64 partial logits.
 //   route_select  E > 16 after a SPLIT pass: sums the partial logits in a
@@ -303,83 +303,68 @@ route_rows(RouteParams p) {
 }
 
 // ---------------------------------------------------------------- E > 16
+template <int EPL, int TPW, bool BF16>
+struct TiledShape {
+  static constexpr int TM = WARPS * TPW;             // tokens per block
+  static constexpr int XS = TM + 4;                  // x row stride (words), keeps 16-byte rows
+  static constexpr int XW = (BF16 ? KC / 2 : KC) * XS;   // x words per stage (bf16 kept as pairs)
+  __host__ __device__ static int stage_words(int E) { return (XW + KC * (E + 1) + 3) / 4 * 4; }
+};
+
+__device__ __forceinline__ void cp_async4(void *smem, const void *gmem, bool valid) {
+  const uint32_t s = (uint32_t)__cvta_generic_to_shared(smem);
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(s), "l"(gmem), "r"(valid ? 4 : 0) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
 template <int EPL, int TPW, bool BF16, bool SPLIT>
-__global__ void __launch_bounds__(kRouteThreads)
+__global__ void __launch_bounds__(kRouteThreads, 1)
 route_tiled(RouteParams p) {
-  constexpr int TM = WARPS * TPW;
-  constexpr int XS = TM + 4;                          // xs row stride (floats), keeps 16-byte rows
-  constexpr int XV = BF16 ? 8 : 4;                    // x elements per 16-byte vector
-  constexpr int XN = (TM * KC / XV + kRouteThreads - 1) / kRouteThreads;
-  constexpr int WN = (kMaxExperts * KC / 4) / kRouteThreads;   // float4 per thread at E = 256
+  using S = TiledShape<EPL, TPW, BF16>;
+  constexpr int TM = S::TM, XS = S::XS, XW = S::XW;
   extern __shared__ __align__(16) unsigned char smem_raw[];
-  float *xs = reinterpret_cast<float *>(smem_raw);    // [KC][XS]   x chunk, k-major
-  float *wsm = xs + KC * XS;                          // [KC][E+1]  W_r chunk, k-major
+  uint32_t *stage_base = reinterpret_cast<uint32_t *>(smem_raw);
   double *dscr = reinterpret_cast<double *>(smem_raw);   // reused after the dot loop
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int E = p.E, d = p.d, WSTR = E + 1;
+  const int SW = S::stage_words(E);
   const int t0 = blockIdx.x * TM;
   int kbeg = 0, kend = d;
   if (SPLIT) {
     kbeg = blockIdx.y * p.kchunk;
     kend = min(d, kbeg + p.kchunk);
   }
-  const int wvec = E * (KC / 4);                      // float4 of W_r per chunk
 
-  uint4 xr[XN];
-  float4 wr[WN];
-  auto gload = [&](int k0) {
-#pragma unroll
-    for (int i = 0; i < XN; ++i) {
-      const int v = tid + i * kRouteThreads;
-      const int tok = v / (KC / XV), q = v % (KC / XV);
-      const int t = t0 + tok, kg = k0 + q * XV;
-      xr[i] = make_uint4(0u, 0u, 0u, 0u);
-      if (tok < TM && t < p.T && kg < kend) {
-        if (BF16) xr[i] = __ldg(reinterpret_cast<const uint4 *>(static_cast<const uint16_t *>(p.x) + (size_t)t * d + kg));
-        else xr[i] = __ldg(reinterpret_cast<const uint4 *>(static_cast<const float *>(p.x) + (size_t)t * d + kg));
+  // chunk k0 -> stage st: x as bf16 pairs (or fp32) k-major, W_r fp32 k-major;
+  // 4-byte cp.async, zero fill outside the tile
+  auto issue = [&](int k0, int st) {
+    uint32_t *xs = stage_base + st * SW;
+    float *ws = reinterpret_cast<float *>(xs + XW);
+    if (BF16) {
+      const uint32_t *xg = static_cast<const uint32_t *>(p.x);
+      for (int i = tid; i < TM * (KC / 2); i += kRouteThreads) {
+        const int tok = i / (KC / 2), j = i % (KC / 2);
+        const int t = t0 + tok, kg = k0 + 2 * j;
+        const bool ok = t < p.T && kg < kend;
+        cp_async4(xs + j * XS + tok, ok ? xg + ((size_t)t * d + kg) / 2 : xg, ok);
+      }
+    } else {
+      const float *xg = static_cast<const float *>(p.x);
+      for (int i = tid; i < TM * KC; i += kRouteThreads) {
+        const int tok = i / KC, kk = i % KC;
+        const int t = t0 + tok, kg = k0 + kk;
+        const bool ok = t < p.T && kg < kend;
+        cp_async4(xs + kk * XS + tok, ok ? xg + (size_t)t * d + kg : xg, ok);
       }
     }
-#pragma unroll
-    for (int i = 0; i < WN; ++i) {
-      const int v = tid + i * kRouteThreads;
-      const int e = v / (KC / 4), q = v % (KC / 4);
-      const int kg = k0 + q * 4;
-      wr[i] = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (v < wvec && kg < kend) wr[i] = __ldg(reinterpret_cast<const float4 *>(p.w + (size_t)e * d + kg));
+    for (int i = tid; i < E * KC; i += kRouteThreads) {
+      const int e = i / KC, kk = i % KC, kg = k0 + kk;
+      const bool ok = kg < kend;
+      cp_async4(ws + kk * WSTR + e, ok ? p.w + (size_t)e * d + kg : p.w, ok);
     }
-  };
-  auto sstore = [&]() {
-#pragma unroll
-    for (int i = 0; i < XN; ++i) {
-      const int v = tid + i * kRouteThreads;
-      const int tok = v / (KC / XV), q = v % (KC / XV);
-      if (tok < TM) {
-        if (BF16) {
-          const uint32_t u[4] = {xr[i].x, xr[i].y, xr[i].z, xr[i].w};
-#pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            xs[(q * 8 + 2 * c) * XS + tok] = __uint_as_float(u[c] << 16);
-            xs[(q * 8 + 2 * c + 1) * XS + tok] = __uint_as_float(u[c] & 0xffff0000u);
-          }
-        } else {
-          xs[(q * 4 + 0) * XS + tok] = __uint_as_float(xr[i].x);
-          xs[(q * 4 + 1) * XS + tok] = __uint_as_float(xr[i].y);
-          xs[(q * 4 + 2) * XS + tok] = __uint_as_float(xr[i].z);
-          xs[(q * 4 + 3) * XS + tok] = __uint_as_float(xr[i].w);
-        }
-      }
-    }
-#pragma unroll
-    for (int i = 0; i < WN; ++i) {
-      const int v = tid + i * kRouteThreads;
-      if (v < wvec) {
-        const int e = v / (KC / 4), q = v % (KC / 4);
-        wsm[(q * 4 + 0) * WSTR + e] = wr[i].x;
-        wsm[(q * 4 + 1) * WSTR + e] = wr[i].y;
-        wsm[(q * 4 + 2) * WSTR + e] = wr[i].z;
-        wsm[(q * 4 + 3) * WSTR + e] = wr[i].w;
-      }
-    }
+    cp_async_commit();
   };
 
   double acc[TPW][EPL];
@@ -388,11 +373,18 @@ route_tiled(RouteParams p) {
 #pragma unroll
     for (int j = 0; j < EPL; ++j) acc[i][j] = 0.0;
 
-  if (kbeg < kend) gload(kbeg);
-  for (int k0 = kbeg; k0 < kend; k0 += KC) {
-    sstore();
+  int st = 0;
+  if (kbeg < kend) issue(kbeg, 0);
+  for (int k0 = kbeg; k0 < kend; k0 += KC, st ^= 1) {
+    if (k0 + KC < kend) {
+      issue(k0 + KC, st ^ 1);               // next chunk lands while this one is used
+      cp_async_wait<1>();
+    } else {
+      cp_async_wait<0>();
+    }
     __syncthreads();
-    if (k0 + KC < kend) gload(k0 + KC);      // next chunk in flight during the FMAs
+    const uint32_t *xs = stage_base + st * SW;
+    const float *ws = reinterpret_cast<const float *>(xs + XW);
 #pragma unroll
     for (int r0 = 0; r0 < KC; r0 += RUN) {
       float run[TPW][EPL];
@@ -400,28 +392,62 @@ route_tiled(RouteParams p) {
       for (int i = 0; i < TPW; ++i)
 #pragma unroll
         for (int j = 0; j < EPL; ++j) run[i][j] = 0.f;
+      if (BF16) {
 #pragma unroll
-      for (int kk = r0; kk < r0 + RUN; ++kk) {
-        float xv[TPW], wv[EPL];
-        if (TPW % 4 == 0) {
+        for (int kk = r0; kk < r0 + RUN; kk += 2) {
+          uint32_t xp[TPW];
+          if (TPW % 4 == 0) {
 #pragma unroll
-          for (int m = 0; m < TPW / 4; ++m) {
-            const float4 f = *reinterpret_cast<const float4 *>(xs + kk * XS + warp * TPW + 4 * m);
-            xv[4 * m] = f.x; xv[4 * m + 1] = f.y; xv[4 * m + 2] = f.z; xv[4 * m + 3] = f.w;
+            for (int m = 0; m < TPW / 4; ++m) {
+              const uint4 q = *reinterpret_cast<const uint4 *>(xs + (kk / 2) * XS + warp * TPW + 4 * m);
+              xp[4 * m] = q.x; xp[4 * m + 1] = q.y; xp[4 * m + 2] = q.z; xp[4 * m + 3] = q.w;
+            }
+          } else {
+#pragma unroll
+            for (int i = 0; i < TPW; ++i) xp[i] = xs[(kk / 2) * XS + warp * TPW + i];
           }
-        } else {
+          float w0[EPL], w1[EPL];
 #pragma unroll
-          for (int i = 0; i < TPW; ++i) xv[i] = xs[kk * XS + warp * TPW + i];
+          for (int j = 0; j < EPL; ++j) {
+            const int e = lane + 32 * j;
+            w0[j] = e < E ? ws[kk * WSTR + e] : 0.f;
+            w1[j] = e < E ? ws[(kk + 1) * WSTR + e] : 0.f;
+          }
+#pragma unroll
+          for (int i = 0; i < TPW; ++i) {
+            const float x0 = __uint_as_float(xp[i] << 16), x1 = __uint_as_float(xp[i] & 0xffff0000u);
+#pragma unroll
+            for (int j = 0; j < EPL; ++j) {
+              run[i][j] = fmaf(x0, w0[j], run[i][j]);
+              run[i][j] = fmaf(x1, w1[j], run[i][j]);
+            }
+          }
         }
+      } else {
+        const float *xf = reinterpret_cast<const float *>(xs);
 #pragma unroll
-        for (int j = 0; j < EPL; ++j) {
-          const int e = lane + 32 * j;
-          wv[j] = e < E ? wsm[kk * WSTR + e] : 0.f;
+        for (int kk = r0; kk < r0 + RUN; ++kk) {
+          float xv[TPW], wv[EPL];
+          if (TPW % 4 == 0) {
+#pragma unroll
+            for (int m = 0; m < TPW / 4; ++m) {
+              const float4 f = *reinterpret_cast<const float4 *>(xf + kk * XS + warp * TPW + 4 * m);
+              xv[4 * m] = f.x; xv[4 * m + 1] = f.y; xv[4 * m + 2] = f.z; xv[4 * m + 3] = f.w;
+            }
+          } else {
+#pragma unroll
+            for (int i = 0; i < TPW; ++i) xv[i] = xf[kk * XS + warp * TPW + i];
+          }
+#pragma unroll
+          for (int j = 0; j < EPL; ++j) {
+            const int e = lane + 32 * j;
+            wv[j] = e < E ? ws[kk * WSTR + e] : 0.f;
+          }
+#pragma unroll
+          for (int i = 0; i < TPW; ++i)
+#pragma unroll
+            for (int j = 0; j < EPL; ++j) run[i][j] = fmaf(xv[i], wv[j], run[i][j]);
         }
-#pragma unroll
-        for (int i = 0; i < TPW; ++i)
-#pragma unroll
-          for (int j = 0; j < EPL; ++j) run[i][j] = fmaf(xv[i], wv[j], run[i][j]);
       }
 #pragma unroll
       for (int i = 0; i < TPW; ++i)
@@ -496,8 +522,7 @@ __global__ void route_finalize(const double *part, int nb, int E, float *prob_su
 
 template <int EPL, int TPW, bool BF16, bool SPLIT>
 cudaError_t launch_tiled(const RouteParams &p, dim3 grid, cudaStream_t s) {
-  constexpr int TM = WARPS * TPW;
-  const size_t stage = sizeof(float) * ((size_t)KC * (TM + 4) + (size_t)KC * (p.E + 1));
+  const size_t stage = sizeof(uint32_t) * 2 * (size_t)TiledShape<EPL, TPW, BF16>::stage_words(p.E);
   const size_t scratch = sizeof(double) * (size_t)WARPS * kMaxExperts;
   const size_t smem = stage > scratch ? stage : scratch;
   auto kern = route_tiled<EPL, TPW, BF16, SPLIT>;
@@ -516,9 +541,7 @@ cudaError_t launch_wide(const RouteParams &p, const RoutePlan &plan, cudaStream_
     route_select<EPL><<<(p.T + kRouteTokens - 1) / kRouteTokens, kRouteThreads, 0, s>>>(p);
     return cudaGetLastError();
   }
-  if constexpr (EPL <= 4) {
-    if (plan.tpw == 8) return launch_tiled<EPL, 8, BF16, false>(p, dim3((p.T + 63) / 64), s);
-  }
+  if (plan.tpw == 8) return launch_tiled<EPL, 8, BF16, false>(p, dim3((p.T + 63) / 64), s);
   return launch_tiled<EPL, 4, BF16, false>(p, dim3((p.T + 31) / 32), s);
 }
 
@@ -562,9 +585,9 @@ RoutePlan route_plan(const moe_config &c, bool allow_split) {
     plan.ks = ks;
     plan.kchunk = kchunk;
   }
-  // 8 tokens per warp halves the shared-memory reads per FMA; with 8 experts
-  // per lane its accumulators no longer fit in registers.
-  if (!plan.split && c.num_experts > 64 && c.num_experts <= 128 && (c.num_tokens + 63) / 64 >= 148) plan.tpw = 8;
+  // 8 tokens per warp halves the shared-memory reads per FMA once the batch
+  // still fills every SM with 64-token blocks.
+  if (!plan.split && c.num_experts > 64 && (c.num_tokens + 63) / 64 >= 148) plan.tpw = 8;
   return plan;
 }
 
