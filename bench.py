@@ -161,7 +161,7 @@ def kernels_per_step(w) -> int:
         route = 2                                   # route_rows + route_finalize
     else:
         nb32 = (w.T + 31) // 32
-        route = 3 if (nb32 < 148 and w.d >= 64) else 2   # split pass adds route_select
+        route = 3 if nb32 < 148 else 2              # split pass adds route_select
     permute = 3                                     # count, scan, scatter
     ffn = 2                                         # two expert GEMM phases
     shared = 2 if w.shared_F else 0

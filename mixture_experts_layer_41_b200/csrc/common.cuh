@@ -179,7 +179,9 @@ struct FfnArgs {
 
 cudaError_t launch_ffn_simt_f32(const FfnArgs &a, cudaStream_t s);
 cudaError_t launch_ffn_tc_bf16(const FfnArgs &a, cudaStream_t s);
-cudaError_t launch_ffn_q4(const FfnArgs &a, cudaStream_t s);
+cudaError_t launch_ffn_q4(const FfnArgs &a, cudaStream_t s);       // SIMT, any d, F multiple of 64
+bool q4_tc_supported(int d, int F);                                 // the tensor-core 4-bit path's shapes
+cudaError_t launch_ffn_q4_tc(const FfnArgs &a, cudaStream_t s);
 
 // Replaces the text moe_last_error() returns on this thread.
 void set_last_error_text(const char *text);

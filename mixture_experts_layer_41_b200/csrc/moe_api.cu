@@ -80,7 +80,7 @@ cudaError_t run_ffn(const FfnArgs &a, cudaStream_t s) {
   switch (a.kind) {
     case 0: return launch_ffn_simt_f32(a, s);
     case 1: return launch_ffn_tc_bf16(a, s);
-    default: return launch_ffn_q4(a, s);
+    default: return q4_tc_supported(a.d, a.F) ? launch_ffn_q4_tc(a, s) : launch_ffn_q4(a, s);
   }
 }
 

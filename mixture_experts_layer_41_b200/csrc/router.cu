@@ -10,7 +10,7 @@
 // runs added in float64 (keeps the logit error near 1e-7 at d = 7168, where a
 // straight fp32 sum reaches ~1e-6); scores, selection and weights are float64
 // and rounded to float32 on the store.  Three shapes:
-//   route_rows    E <= 16: one warp per 4 tokens, lanes split the hidden
+//   route_rows    E <= 16: one warp per 2 tokens, lanes split the hidden
 //                 dimension with 16-byte loads, W_r read through L1; the
 //                 E logits of a token are warp all-reduced, lane e owns e.
 //   route_tiled   E > 16: a block owns 8*TPW tokens x all E experts; x and W_r
@@ -18,9 +18,11 @@
 //                 with cp.async, double-buffered one chunk ahead; lane l owns
 //                 experts l, l+32, ...  With SPLIT the block covers one slice
 //                 of the hidden dimension and writes float64 partial logits.
-//   route_select  E > 16 after a SPLIT pass: sums the partial logits in a
-//                 fixed order and selects (used when T is too small to fill
-//                 the GPU with whole-row blocks, e.g. decode).
+//   route_select  E > 16 after a SPLIT pass (8-token x 32-expert x hidden-
+//                 slice blocks, used when T is too small to fill the GPU with
+//                 whole-row blocks, e.g. decode): sums the partial logits of
+//                 32 tokens in slice order into shared memory, then selects
+//                 with one warp per token.
 // Every selecting block covers 32-token groups and writes one float64
 // probability sum per (group, expert); route_finalize adds the groups in
 // order, so prob_sum is deterministic.
@@ -181,7 +183,7 @@ __device__ __forceinline__ void select_token(const RouteParams &p, int t, const 
 // Per-warp probability sums -> one row per 32-token group, warps added in
 // order.  tok0_of_warp(w) gives the first token of warp w; every warp's
 // tokens lie inside one group.
-template <int EPL>
+template <int EPL, int NW = WARPS>
 __device__ __forceinline__ void write_prob_partials(const RouteParams &p, double *scratch, const double (&psum)[EPL],
                                                     int block_tok0, int tokens_per_warp, int lane, int warp) {
   __syncthreads();
@@ -193,39 +195,41 @@ __device__ __forceinline__ void write_prob_partials(const RouteParams &p, double
   }
   __syncthreads();
   const int warps_per_group = 32 / tokens_per_warp;
-  const int groups = (WARPS + warps_per_group - 1) / warps_per_group;
-  for (int i = threadIdx.x; i < groups * E; i += kRouteThreads) {
+  const int groups = (NW + warps_per_group - 1) / warps_per_group;
+  for (int i = threadIdx.x; i < groups * E; i += 32 * NW) {
     const int g = i / E, e = i % E;
     const int grow = block_tok0 / 32 + g;
     if (grow * 32 >= p.T) continue;
     double s = 0.0;
-    for (int w = g * warps_per_group; w < (g + 1) * warps_per_group && w < WARPS; ++w) s += scratch[w * E + e];
+    for (int w = g * warps_per_group; w < (g + 1) * warps_per_group && w < NW; ++w) s += scratch[w * E + e];
     p.part[(size_t)grow * E + e] = s;
   }
 }
 
 // ---------------------------------------------------------------- E <= 16
-template <int EP, bool BF16>
-__global__ void __launch_bounds__(kRouteThreads)
+template <int EP, bool BF16, int TPW = 2>
+__global__ void __launch_bounds__(32 * (32 / TPW))
 route_rows(RouteParams p) {
-  __shared__ double scratch[WARPS * 16];       // per-warp probability sums
-  __shared__ double wscr_all[WARPS * 32];      // per-warp selection scores (sigmoid groups)
+  constexpr int NW = 32 / TPW;                 // warps per 32-token block
+  __shared__ double scratch[NW * 16];          // per-warp probability sums
+  __shared__ double wscr_all[NW * 32];         // per-warp selection scores (sigmoid groups)
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int E = p.E, d = p.d;
-  const int t0 = blockIdx.x * kRouteTokens + warp * 4;
-  double acc[4][EP];
+  const int t0 = blockIdx.x * kRouteTokens + warp * TPW;
+  double acc[TPW][EP];
 #pragma unroll
-  for (int i = 0; i < 4; ++i)
+  for (int i = 0; i < TPW; ++i)
 #pragma unroll
     for (int e = 0; e < EP; ++e) acc[i][e] = 0.0;
 
   constexpr int V = BF16 ? 8 : 4;   // elements per step and lane
   const bool vec = (d % V) == 0;
   if (vec) {
+#pragma unroll 2
     for (int k = lane * V; k < d; k += 32 * V) {
-      float xv[4][V];
+      float xv[TPW][V];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
+      for (int i = 0; i < TPW; ++i) {
         const int t = t0 + i;
         if (t < p.T) {
           if (BF16) {
@@ -258,7 +262,7 @@ route_rows(RouteParams p) {
             wv[4] = b.x; wv[5] = b.y; wv[6] = b.z; wv[7] = b.w;
           }
 #pragma unroll
-          for (int i = 0; i < 4; ++i) {
+          for (int i = 0; i < TPW; ++i) {
             float run = 0.f;
 #pragma unroll
             for (int c = 0; c < V; ++c) run = fmaf(xv[i][c], wv[c], run);
@@ -271,7 +275,7 @@ route_rows(RouteParams p) {
     // fp32 rows whose length is not a multiple of 4: one element per step
     for (int k = lane; k < d; k += 32) {
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
+      for (int i = 0; i < TPW; ++i) {
         const int t = t0 + i;
         const float xv = t < p.T ? static_cast<const float *>(p.x)[(size_t)t * d + k] : 0.f;
 #pragma unroll
@@ -281,14 +285,14 @@ route_rows(RouteParams p) {
     }
   }
 #pragma unroll
-  for (int i = 0; i < 4; ++i)
+  for (int i = 0; i < TPW; ++i)
 #pragma unroll
     for (int e = 0; e < EP; ++e) acc[i][e] = warp_sum(acc[i][e]);
 
   double psum[1] = {0.0};
   double *wscr = wscr_all + warp * 32;
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
+  for (int i = 0; i < TPW; ++i) {
     const int t = t0 + i;
     if (t < p.T) {
       double lg[1];
@@ -299,7 +303,7 @@ route_rows(RouteParams p) {
       select_token<1>(p, t, lg, psum, wscr, lane);
     }
   }
-  write_prob_partials<1>(p, scratch, psum, blockIdx.x * kRouteTokens, 4, lane, warp);
+  write_prob_partials<1, NW>(p, scratch, psum, blockIdx.x * kRouteTokens, TPW, lane, warp);
 }
 
 // ---------------------------------------------------------------- E > 16
@@ -328,8 +332,12 @@ route_tiled(RouteParams p) {
   uint32_t *stage_base = reinterpret_cast<uint32_t *>(smem_raw);
   double *dscr = reinterpret_cast<double *>(smem_raw);   // reused after the dot loop
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int E = p.E, d = p.d, WSTR = E + 1;
-  const int SW = S::stage_words(E);
+  const int E = p.E, d = p.d;
+  // experts of this block: all of them, or (SPLIT) a slice of 32*EPL
+  const int e0 = SPLIT ? blockIdx.z * 32 * EPL : 0;
+  const int EB = SPLIT ? min(32 * EPL, E - e0) : E;
+  const int WSTR = EB + 1;
+  const int SW = S::stage_words(EB);
   const int t0 = blockIdx.x * TM;
   int kbeg = 0, kend = d;
   if (SPLIT) {
@@ -359,10 +367,10 @@ route_tiled(RouteParams p) {
         cp_async4(xs + kk * XS + tok, ok ? xg + (size_t)t * d + kg : xg, ok);
       }
     }
-    for (int i = tid; i < E * KC; i += kRouteThreads) {
+    for (int i = tid; i < EB * KC; i += kRouteThreads) {
       const int e = i / KC, kk = i % KC, kg = k0 + kk;
       const bool ok = kg < kend;
-      cp_async4(ws + kk * WSTR + e, ok ? p.w + (size_t)e * d + kg : p.w, ok);
+      cp_async4(ws + kk * WSTR + e, ok ? p.w + (size_t)(e0 + e) * d + kg : p.w, ok);
     }
     cp_async_commit();
   };
@@ -410,8 +418,8 @@ route_tiled(RouteParams p) {
 #pragma unroll
           for (int j = 0; j < EPL; ++j) {
             const int e = lane + 32 * j;
-            w0[j] = e < E ? ws[kk * WSTR + e] : 0.f;
-            w1[j] = e < E ? ws[(kk + 1) * WSTR + e] : 0.f;
+            w0[j] = e < EB ? ws[kk * WSTR + e] : 0.f;
+            w1[j] = e < EB ? ws[(kk + 1) * WSTR + e] : 0.f;
           }
 #pragma unroll
           for (int i = 0; i < TPW; ++i) {
@@ -441,7 +449,7 @@ route_tiled(RouteParams p) {
 #pragma unroll
           for (int j = 0; j < EPL; ++j) {
             const int e = lane + 32 * j;
-            wv[j] = e < E ? ws[kk * WSTR + e] : 0.f;
+            wv[j] = e < EB ? ws[kk * WSTR + e] : 0.f;
           }
 #pragma unroll
           for (int i = 0; i < TPW; ++i)
@@ -465,7 +473,7 @@ route_tiled(RouteParams p) {
 #pragma unroll
         for (int j = 0; j < EPL; ++j) {
           const int e = lane + 32 * j;
-          if (e < E) p.logits[((size_t)blockIdx.y * p.T + t) * E + e] = acc[i][j];
+          if (e < EB) p.logits[((size_t)blockIdx.y * p.T + t) * E + e0 + e] = acc[i][j];
         }
       }
     }
@@ -484,40 +492,73 @@ route_tiled(RouteParams p) {
   write_prob_partials<EPL>(p, dscr, psum, t0, TPW, lane, warp);
 }
 
+constexpr int SEL_WARPS = 32;   // route_select: one warp per token of a 32-token group
+
 template <int EPL>
-__global__ void __launch_bounds__(kRouteThreads)
+__global__ void __launch_bounds__(32 * SEL_WARPS)
 route_select(RouteParams p) {
-  __shared__ double dscr[WARPS * kMaxExperts];
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  double *lgs = reinterpret_cast<double *>(smem_raw);                 // [32][E] summed logits
+  double *dscr = lgs + kRouteTokens * p.E;                           // [SEL_WARPS][kMaxExperts]
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int E = p.E;
-  const int t0 = blockIdx.x * kRouteTokens + warp * 4;
+  const int tb = blockIdx.x * kRouteTokens;
+  constexpr int NT = 32 * SEL_WARPS;
+  // every thread sums the slices of 4 (token, expert) logits at a time, in
+  // slice order, with the loads of a slice in flight together
+  const int n = kRouteTokens * E;
+  for (int o0 = threadIdx.x; o0 < n; o0 += 4 * NT) {
+    double sacc[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) sacc[u] = 0.0;
+    for (int q = 0; q < p.ks; ++q) {
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int o = o0 + u * NT;
+        const int t = tb + o / E;
+        if (o < n && t < p.T) sacc[u] += p.logits[((size_t)q * p.T + t) * E + o % E];
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int o = o0 + u * NT;
+      if (o < n) lgs[o] = sacc[u];
+    }
+  }
+  __syncthreads();
   double psum[EPL];
 #pragma unroll
   for (int j = 0; j < EPL; ++j) psum[j] = 0.0;
   double *wscr = dscr + warp * kMaxExperts;
-  for (int i = 0; i < 4; ++i) {
-    const int t = t0 + i;
-    if (t >= p.T) break;
+  const int t = tb + warp;
+  if (t < p.T) {
     double lg[EPL];
 #pragma unroll
     for (int j = 0; j < EPL; ++j) {
       const int e = lane + 32 * j;
-      double s = 0.0;
-      if (e < E)
-        for (int q = 0; q < p.ks; ++q) s += p.logits[((size_t)q * p.T + t) * E + e];
-      lg[j] = s;
+      lg[j] = e < E ? lgs[warp * E + e] : 0.0;
     }
     select_token<EPL>(p, t, lg, psum, wscr, lane);
   }
-  write_prob_partials<EPL>(p, dscr, psum, blockIdx.x * kRouteTokens, 4, lane, warp);
+  write_prob_partials<EPL, SEL_WARPS>(p, dscr, psum, tb, 1, lane, warp);
 }
 
+// prob_sum[e] = sum over 32-token groups, as eight interleaved running sums
+// (group b feeds sum b % 8, in increasing b) added pairwise at the end: a
+// fixed order, with eight loads in flight per step.
 __global__ void route_finalize(const double *part, int nb, int E, float *prob_sum) {
   const int e = blockIdx.x * blockDim.x + threadIdx.x;
   if (e >= E) return;
-  double s = 0.0;
-  for (int b = 0; b < nb; ++b) s += part[(size_t)b * E + e];
-  prob_sum[e] = (float)s;
+  double s[8];
+#pragma unroll
+  for (int u = 0; u < 8; ++u) s[u] = 0.0;
+  int b = 0;
+  for (; b + 8 <= nb; b += 8) {
+#pragma unroll
+    for (int u = 0; u < 8; ++u) s[u] += part[(size_t)(b + u) * E + e];
+  }
+  for (int u = 0; b + u < nb; ++u) s[u] += part[(size_t)(b + u) * E + e];
+  prob_sum[e] = (float)(((s[0] + s[1]) + (s[2] + s[3])) + ((s[4] + s[5]) + (s[6] + s[7])));
 }
 
 template <int EPL, int TPW, bool BF16, bool SPLIT>
@@ -535,10 +576,15 @@ cudaError_t launch_tiled(const RouteParams &p, dim3 grid, cudaStream_t s) {
 template <int EPL, bool BF16>
 cudaError_t launch_wide(const RouteParams &p, const RoutePlan &plan, cudaStream_t s) {
   if (plan.split) {
-    const dim3 grid((p.T + kRouteTokens - 1) / kRouteTokens, plan.ks);
-    cudaError_t err = launch_tiled<EPL, 4, BF16, true>(p, grid, s);
+    // 8-token tiles x 32-expert slices x hidden-dimension slices
+    const dim3 grid((p.T + 7) / 8, plan.ks, (p.E + 31) / 32);
+    cudaError_t err = launch_tiled<1, 1, BF16, true>(p, grid, s);
     if (err != cudaSuccess) return err;
-    route_select<EPL><<<(p.T + kRouteTokens - 1) / kRouteTokens, kRouteThreads, 0, s>>>(p);
+    const size_t smem = sizeof(double) * ((size_t)kRouteTokens * p.E + (size_t)SEL_WARPS * kMaxExperts);
+    auto sel = route_select<EPL>;
+    err = cudaFuncSetAttribute(sel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (err != cudaSuccess) return err;
+    sel<<<(p.T + kRouteTokens - 1) / kRouteTokens, 32 * SEL_WARPS, smem, s>>>(p);
     return cudaGetLastError();
   }
   if (plan.tpw == 8) return launch_tiled<EPL, 8, BF16, false>(p, dim3((p.T + 63) / 64), s);
@@ -549,11 +595,11 @@ template <bool BF16>
 cudaError_t launch_any(const RouteParams &p, const RoutePlan &plan, cudaStream_t s) {
   const int nb32 = (p.T + kRouteTokens - 1) / kRouteTokens;
   if (p.E <= 8) {
-    route_rows<8, BF16><<<nb32, kRouteThreads, 0, s>>>(p);
+    route_rows<8, BF16, 2><<<nb32, 32 * 16, 0, s>>>(p);
     return cudaGetLastError();
   }
   if (p.E <= 16) {
-    route_rows<16, BF16><<<nb32, kRouteThreads, 0, s>>>(p);
+    route_rows<16, BF16, 4><<<nb32, 32 * 8, 0, s>>>(p);    // 16 experts x 4 tokens of accumulators
     return cudaGetLastError();
   }
   if (p.E <= 64) return launch_wide<2, BF16>(p, plan, s);
@@ -570,24 +616,27 @@ RoutePlan route_plan(const moe_config &c, bool allow_split) {
   plan.kchunk = c.hidden;
   plan.tpw = 4;
   if (c.num_experts <= 16) return plan;
-  const int nb32 = (c.num_tokens + kRouteTokens - 1) / kRouteTokens;
-  const int target = 2 * 148;
+  const int sms = 148;
+  const int whole_row_blocks = (c.num_tokens + kRouteTokens - 1) / kRouteTokens;
   const bool vec_ok = c.act_dtype == MOE_BF16 ? (c.hidden % 8 == 0) : (c.hidden % 4 == 0);
-  if (allow_split && vec_ok && nb32 < 148 && c.hidden >= 2 * KC) {
-    int ks = (target + nb32 - 1) / nb32;
-    const int max_ks = c.hidden / KC;
+  if (allow_split && vec_ok && whole_row_blocks < sms) {
+    // 8-token tiles x 32-expert slices, then as many hidden-dimension slices
+    // (each a multiple of 32 elements, at most 16) as it takes to fill the GPU
+    const int base = ((c.num_tokens + 7) / 8) * ((c.num_experts + 31) / 32);
+    int ks = (sms + base - 1) / base;
+    const int max_ks = c.hidden / KC < 16 ? c.hidden / KC : 16;
     ks = ks < max_ks ? ks : max_ks;
-    ks = ks < 64 ? ks : 64;
+    ks = ks < 1 ? 1 : ks;
     int kchunk = (c.hidden + ks - 1) / ks;
     kchunk = (kchunk + KC - 1) / KC * KC;
-    ks = (c.hidden + kchunk - 1) / kchunk;
-    plan.split = ks > 1;
-    plan.ks = ks;
+    plan.ks = (c.hidden + kchunk - 1) / kchunk;
     plan.kchunk = kchunk;
+    plan.split = true;
+    return plan;
   }
   // 8 tokens per warp halves the shared-memory reads per FMA once the batch
   // still fills every SM with 64-token blocks.
-  if (!plan.split && c.num_experts > 64 && (c.num_tokens + 63) / 64 >= 148) plan.tpw = 8;
+  if (c.num_experts > 64 && (c.num_tokens + 63) / 64 >= sms) plan.tpw = 8;
   return plan;
 }
 

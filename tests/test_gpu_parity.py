@@ -30,6 +30,10 @@ SMALL = {
     "ragged_nk": workload("mixtral_prefill", T=333, d=200, F=136, E=4, k=2),
     "relu_ragged_nk": workload("switch_top1", T=257, d=136, F=264, E=8, k=2, capacity_factor=1.25),
     "fp32_swiglu": workload("tiny_fp32", T=97, d=24, F=40, E=6, k=3, act="swiglu", capacity_factor=0.0),
+    # 4-bit: several 32-token passes per expert on the tensor-core path, and
+    # a shape (d, F not multiples of 128) that takes the CUDA-core path
+    "decode_many_rows": workload("decode_q4", T=200, d=256, F=256, E=8, k=2),
+    "decode_cuda_core_shape": workload("decode_q4", T=24, d=320, F=192, E=16, k=4),
 }
 
 
