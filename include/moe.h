@@ -243,6 +243,28 @@ moe_status moe_permute(const moe_config *cfg, const void *x, const int32_t *topk
                        float *perm_w, int32_t *slot_row, void *x_perm, const moe_stats *stats,
                        void *ws, size_t ws_bytes, moe_stream_t stream);
 
+/* Token-sharded dispatch with the in-order capacity rule of the whole batch
+ * (blog moe_layer: capacity is "per BATCH"; its in-order cut then spans the
+ * token shards held by different GPUs).  A batch split into contiguous token
+ * shards keeps, on the shard of rank r, a slot of expert e iff
+ * shard_base[e] + (its rank among this shard's slots of e) < capacity, where
+ * shard_base[e] is the number of slots of e on the earlier shards -- the one
+ * exchange the sharded layer needs (an all-gather of moe_expert_counts).
+ *
+ * moe_expert_counts: raw per-expert slot counts of this shard's topk_ids
+ *   (the histogram of the dispatch, no capacity, no gather).  Out: raw_counts
+ *   [E] int32 (device).  Uses ws.
+ * moe_permute_shard: moe_permute with capacity = the WHOLE batch's capacity
+ *   (moe_capacity(T_total, ...), -1 for none) and shard_base [E] int32
+ *   (device, NULL = first shard); cfg->num_tokens is this shard's token count.
+ *   Same outputs as moe_permute.  Uses ws. */
+moe_status moe_expert_counts(const moe_config *cfg, const int32_t *topk_ids, int32_t *raw_counts, void *ws,
+                             size_t ws_bytes, moe_stream_t stream);
+moe_status moe_permute_shard(const moe_config *cfg, const void *x, const int32_t *topk_ids, const float *topk_w,
+                             const int32_t *shard_base, int64_t capacity, int32_t *expert_offsets,
+                             int32_t *perm_token, float *perm_w, int32_t *slot_row, void *x_perm,
+                             const moe_stats *stats, void *ws, size_t ws_bytes, moe_stream_t stream);
+
 /* Grouped expert FFN over the ragged groups (design doc: one grouped matmul
  * over the per-expert token groups; blog moe_forward: two GEMMs per expert
  * over contiguous slices).  For every expert e and row r in

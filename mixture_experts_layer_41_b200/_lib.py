@@ -87,6 +87,8 @@ SIGNATURES = {
     "moe_route": (C.c_int, [_CFG, _P, _P, _P, _P, _P, _P, _P, C.c_size_t, _P]),
     "moe_route_noalloc": (C.c_int, [_CFG, _P, _P, _P, _P, _P, _P, _P]),
     "moe_permute": (C.c_int, [_CFG, _P, _P, _P, _P, _P, _P, _P, _P, _S, _P, C.c_size_t, _P]),
+    "moe_expert_counts": (C.c_int, [_CFG, _P, _P, _P, C.c_size_t, _P]),
+    "moe_permute_shard": (C.c_int, [_CFG, _P, _P, _P, _P, C.c_int64, _P, _P, _P, _P, _P, _S, _P, C.c_size_t, _P]),
     "moe_grouped_ffn": (C.c_int, [_CFG, _P, _P, _W, _P, _P, C.c_size_t, _P]),
     "moe_shared_expert": (C.c_int, [_CFG, _P, _W, _P, _P, C.c_size_t, _P]),
     "moe_combine": (C.c_int, [_CFG, _P, _P, _P, _P, _P, _P]),

@@ -142,6 +142,40 @@ def moe_permute(cfg, x, topk_ids, topk_w, expert_offsets, perm_token, perm_w, sl
           "moe_permute")
 
 
+def moe_expert_counts(cfg, topk_ids, raw_counts, ws, stream=None):
+    check(L.lib().moe_expert_counts(C.byref(cfg), _p(topk_ids), _p(raw_counts), _p(ws), _nbytes(ws),
+                                    _s(stream)), "moe_expert_counts")
+
+
+def moe_permute_shard(cfg, x, topk_ids, topk_w, shard_base, capacity, expert_offsets, perm_token, perm_w,
+                      slot_row, x_perm, stats, ws, stream=None):
+    st = _stats_struct(stats)
+    check(L.lib().moe_permute_shard(C.byref(cfg), _p(x), _p(topk_ids), _p(topk_w), _p(shard_base), int(capacity),
+                                    _p(expert_offsets), _p(perm_token), _p(perm_w), _p(slot_row), _p(x_perm),
+                                    C.byref(st) if st is not None else None, _p(ws), _nbytes(ws), _s(stream)),
+          "moe_permute_shard")
+
+
+def shard_base_from_counts(counts_by_rank: torch.Tensor, rank: int) -> torch.Tensor:
+    """Slots of each expert on the shards before ``rank``: the exclusive
+    prefix over ranks of the gathered [world, E] raw counts."""
+    if rank == 0:
+        return torch.zeros_like(counts_by_rank[0])
+    return counts_by_rank[:rank].sum(dim=0).to(counts_by_rank.dtype)
+
+
+def exchange_shard_base(raw_counts: torch.Tensor, group=None) -> torch.Tensor:
+    """The sharded layer's one exchange: all-gather every rank's per-expert
+    raw counts (an E-int32 message per rank) and return this rank's
+    shard_base.  Token shards must be contiguous and in rank order."""
+    import torch.distributed as dist
+    world = dist.get_world_size(group)
+    rank = dist.get_rank(group)
+    gathered = [torch.empty_like(raw_counts) for _ in range(world)]
+    dist.all_gather(gathered, raw_counts.contiguous(), group=group)
+    return shard_base_from_counts(torch.stack(gathered), rank)
+
+
 def moe_grouped_ffn(cfg, x_perm, expert_offsets, weights: dict, y_perm, ws, stream=None):
     w = _weights_struct(weights)
     check(L.lib().moe_grouped_ffn(C.byref(cfg), _p(x_perm), _p(expert_offsets), C.byref(w), _p(y_perm),

@@ -155,7 +155,7 @@ cudaError_t launch_permute(const moe_config &c, const void *x, const int32_t *to
                            int32_t *perm_token, float *perm_w, int32_t *slot_row, void *x_perm,
                            int32_t *raw_counts, int32_t *kept_counts, int32_t *dropped,
                            int32_t *blk_counts, int32_t *blk_base, int32_t *local_rank,
-                           int *status, cudaStream_t s);
+                           int *status, cudaStream_t s, const int32_t *shard_base = nullptr);
 
 // Two-phase expert FFN over groups.  `offsets` == nullptr means one group of
 // `rows` rows (the shared expert).  Writes the intermediate to `h` and the

@@ -341,6 +341,52 @@ moe_status moe_permute(const moe_config *cfg, const void *x, const int32_t *topk
                     stats->raw_counts, stats->kept_counts, stats->dropped, ws, s);
 }
 
+moe_status moe_expert_counts(const moe_config *cfg, const int32_t *topk_ids, int32_t *raw_counts, void *ws,
+                             size_t ws_bytes, moe_stream_t stream) {
+  moe_status st = moe_validate(cfg);
+  if (st != MOE_OK) return st;
+  const moe_config &c = *cfg;
+  if (!aligned16(topk_ids) || !aligned16(raw_counts)) return MOE_ERR_INVALID_ARG;
+  if ((st = check_ws(c, ws, ws_bytes)) != MOE_OK) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if ((st = clear_status(ws, s)) != MOE_OK) return st;
+  const WsLayout L = ws_layout(c);
+  // the dispatch's own histogram and scan, without a capacity and without the gather
+  cudaError_t err = launch_permute(c, nullptr, topk_ids, nullptr, -1, ws_ptr<int32_t>(ws, L.offsets),
+                                   ws_ptr<int32_t>(ws, L.perm_token), ws_ptr<float>(ws, L.perm_w),
+                                   ws_ptr<int32_t>(ws, L.slot_row), nullptr, raw_counts,
+                                   ws_ptr<int32_t>(ws, L.kept_counts), ws_ptr<int32_t>(ws, L.dropped),
+                                   ws_ptr<int32_t>(ws, L.blk_counts), ws_ptr<int32_t>(ws, L.blk_base),
+                                   ws_ptr<int32_t>(ws, L.local_rank), ws_ptr<int>(ws, L.status), s);
+  return err == cudaSuccess ? MOE_OK : cuda_fail(err, "moe_expert_counts");
+}
+
+moe_status moe_permute_shard(const moe_config *cfg, const void *x, const int32_t *topk_ids, const float *topk_w,
+                             const int32_t *shard_base, int64_t capacity, int32_t *expert_offsets,
+                             int32_t *perm_token, float *perm_w, int32_t *slot_row, void *x_perm,
+                             const moe_stats *stats, void *ws, size_t ws_bytes, moe_stream_t stream) {
+  moe_status st = moe_validate(cfg);
+  if (st != MOE_OK) return st;
+  const moe_config &c = *cfg;
+  if (capacity < -1) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(topk_ids) || !aligned16(topk_w) || !aligned16(expert_offsets) || !aligned16(perm_token) ||
+      !aligned16(perm_w) || !aligned16(slot_row) || !aligned16_or_null(x) || !aligned16_or_null(x_perm) ||
+      !aligned16_or_null(shard_base))
+    return MOE_ERR_INVALID_ARG;
+  if ((x == nullptr) != (x_perm == nullptr)) return MOE_ERR_INVALID_ARG;
+  if (!stats || !aligned16(stats->raw_counts) || !aligned16(stats->kept_counts) || !aligned16(stats->dropped))
+    return MOE_ERR_INVALID_ARG;
+  if ((st = check_ws(c, ws, ws_bytes)) != MOE_OK) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if ((st = clear_status(ws, s)) != MOE_OK) return st;
+  const WsLayout L = ws_layout(c);
+  cudaError_t err = launch_permute(c, x, topk_ids, topk_w, capacity, expert_offsets, perm_token, perm_w, slot_row,
+                                   x_perm, stats->raw_counts, stats->kept_counts, stats->dropped,
+                                   ws_ptr<int32_t>(ws, L.blk_counts), ws_ptr<int32_t>(ws, L.blk_base),
+                                   ws_ptr<int32_t>(ws, L.local_rank), ws_ptr<int>(ws, L.status), s, shard_base);
+  return err == cudaSuccess ? MOE_OK : cuda_fail(err, "moe_permute_shard");
+}
+
 moe_status moe_grouped_ffn(const moe_config *cfg, const void *x_perm, const int32_t *expert_offsets,
                            const moe_weights *w, void *y_perm, void *ws, size_t ws_bytes, moe_stream_t stream) {
   moe_status st = moe_validate(cfg);

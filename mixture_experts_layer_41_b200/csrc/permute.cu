@@ -59,7 +59,9 @@ count_kernel(const int32_t *ids, int T, int k, int E, int32_t *blk_counts, int32
 }
 
 // One block of up to 1024 threads, one thread per expert.
-__global__ void scan_kernel(const int32_t *blk_counts, int nb, int E, long long cap,
+// shard_base (nullable): slots of each expert held by earlier token shards of
+// the same batch; the capacity left for this shard is cap - shard_base[e].
+__global__ void scan_kernel(const int32_t *blk_counts, int nb, int E, long long cap, const int32_t *shard_base,
                             int32_t *blk_base, int32_t *raw_counts, int32_t *kept_counts,
                             int32_t *offsets, int32_t *dropped) {
   __shared__ int32_t kept_s[kMaxExperts];
@@ -71,7 +73,9 @@ __global__ void scan_kernel(const int32_t *blk_counts, int nb, int E, long long 
       blk_base[(size_t)b * E + e] = run;
       run += blk_counts[(size_t)b * E + e];
     }
-    const int kept = (cap >= 0 && (long long)run > cap) ? (int)cap : run;
+    long long room = cap;
+    if (cap >= 0 && shard_base) room = cap - shard_base[e] > 0 ? cap - shard_base[e] : 0;
+    const int kept = (room >= 0 && (long long)run > room) ? (int)room : run;
     raw_counts[e] = run;
     kept_counts[e] = kept;
     kept_s[e] = kept;
@@ -94,7 +98,7 @@ template <int VEC_BYTES>
 __global__ void __launch_bounds__(256)
 scatter_kernel(const int32_t *ids, const float *wts, const int32_t *local_rank,
                const int32_t *blk_base, const int32_t *offsets, int T, int k, int E,
-               long long cap, const char *x, size_t row_bytes, int32_t *perm_token,
+               long long cap, const int32_t *shard_base, const char *x, size_t row_bytes, int32_t *perm_token,
                float *perm_w, int32_t *slot_row, char *x_perm) {
   const int warp_global = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
@@ -105,7 +109,8 @@ scatter_kernel(const int32_t *ids, const float *wts, const int32_t *local_rank,
   int row = -1;
   if (e >= 0 && e < E && lr >= 0) {
     const int rank = blk_base[(size_t)(t / kPermTokens) * E + e] + lr;
-    if (cap < 0 || (long long)rank < cap) row = offsets[e] + rank;
+    const long long room = (cap >= 0 && shard_base) ? cap - shard_base[e] : cap;
+    if (cap < 0 || (long long)rank < room) row = offsets[e] + rank;
   }
   if (lane == 0) {
     slot_row[warp_global] = row;
@@ -137,13 +142,13 @@ cudaError_t launch_permute(const moe_config &c, const void *x, const int32_t *to
                            int32_t *perm_token, float *perm_w, int32_t *slot_row, void *x_perm,
                            int32_t *raw_counts, int32_t *kept_counts, int32_t *dropped,
                            int32_t *blk_counts, int32_t *blk_base, int32_t *local_rank,
-                           int *status, cudaStream_t s) {
+                           int *status, cudaStream_t s, const int32_t *shard_base) {
   const int T = c.num_tokens, k = c.top_k, E = c.num_experts;
   const int nb = perm_blocks(c);
   count_kernel<<<nb, kPermTokens, 0, s>>>(topk_ids, T, k, E, blk_counts, local_rank, status);
   cudaError_t err = cudaGetLastError();
   if (err != cudaSuccess) return err;
-  scan_kernel<<<1, kMaxExperts, 0, s>>>(blk_counts, nb, E, (long long)capacity, blk_base,
+  scan_kernel<<<1, kMaxExperts, 0, s>>>(blk_counts, nb, E, (long long)capacity, shard_base, blk_base,
                                         raw_counts, kept_counts, expert_offsets, dropped);
   err = cudaGetLastError();
   if (err != cudaSuccess) return err;
@@ -153,12 +158,12 @@ cudaError_t launch_permute(const moe_config &c, const void *x, const int32_t *to
   const bool vec16 = (row_bytes % 16) == 0;
   if (vec16)
     scatter_kernel<16><<<blocks, 256, 0, s>>>(topk_ids, topk_w, local_rank, blk_base, expert_offsets,
-                                              T, k, E, (long long)capacity,
+                                              T, k, E, (long long)capacity, shard_base,
                                               static_cast<const char *>(x), row_bytes, perm_token,
                                               perm_w, slot_row, static_cast<char *>(x_perm));
   else
     scatter_kernel<4><<<blocks, 256, 0, s>>>(topk_ids, topk_w, local_rank, blk_base, expert_offsets,
-                                             T, k, E, (long long)capacity,
+                                             T, k, E, (long long)capacity, shard_base,
                                              static_cast<const char *>(x), row_bytes, perm_token,
                                              perm_w, slot_row, static_cast<char *>(x_perm));
   return cudaGetLastError();

@@ -221,3 +221,67 @@ def test_router_shapes(name):
     torch.cuda.synchronize()
     assert run.status() == 0
     check_route(run, oracle_route(w, run.inp))
+
+
+def test_token_sharded_capacity_on_one_gpu():
+    """Two token shards of one batch, dispatched one after the other on one
+    GPU with moe_expert_counts -> shard_base -> moe_permute_shard: the kept
+    slots and the layer output equal the oracle's whole-batch in-order
+    dispatch (the sharded layer's single exchange is the count all-gather)."""
+    from mixture_experts_layer_41_b200.inputs import make_inputs, to_host
+    from moe_cases import HostExperts, cfg_of, weights_of
+    from oracle import moe_oracle as O
+    w = workload("switch_top1", T=1000, d=256, F=256, E=16, k=2, capacity_factor=1.0)
+    dev = torch.device("cuda")
+    inp = make_inputs(w, seed=8, device=dev)
+    weights = weights_of(inp)
+    cap = api.moe_capacity(w.T, w.k, w.E, w.capacity_factor)
+    halves = [(0, 440), (440, w.T)]          # unequal shards
+    counts, parts = [], []
+    for lo, hi in halves:
+        ws_ = w.with_(T=hi - lo)
+        cfg = cfg_of(ws_)
+        ws = torch.empty(api.moe_workspace_size(cfg), dtype=torch.uint8, device=dev)
+        x = inp["x"][lo:hi].contiguous()
+        ids = torch.empty((hi - lo, w.k), dtype=torch.int32, device=dev)
+        wts = torch.empty((hi - lo, w.k), dtype=torch.float32, device=dev)
+        ps = torch.empty(w.E, dtype=torch.float32, device=dev)
+        api.moe_route(cfg, x, inp["w_router"], inp["logit_bias"], ids, wts, ps, ws)
+        raw = torch.empty(w.E, dtype=torch.int32, device=dev)
+        api.moe_expert_counts(cfg, ids, raw, ws)
+        counts.append(raw)
+        parts.append((cfg, ws, x, ids, wts))
+    torch.cuda.synchronize()
+    gathered = torch.stack(counts)
+    out = torch.empty((w.T, w.d), dtype=torch.bfloat16, device=dev)
+    slot_all = []
+    for r, ((lo, hi), (cfg, ws, x, ids, wts)) in enumerate(zip(halves, parts)):
+        base = api.shard_base_from_counts(gathered, r).contiguous()
+        n = hi - lo
+        i32 = dict(dtype=torch.int32, device=dev)
+        off = torch.empty(w.E + 1, **i32)
+        perm_token = torch.empty(n * w.k, **i32)
+        perm_w = torch.empty(n * w.k, dtype=torch.float32, device=dev)
+        slot_row = torch.empty((n, w.k), **i32)
+        x_perm = torch.empty((n * w.k, w.d), dtype=torch.bfloat16, device=dev)
+        y_perm = torch.empty_like(x_perm)
+        stats = dict(raw_counts=torch.empty(w.E, **i32), kept_counts=torch.empty(w.E, **i32),
+                     dropped=torch.empty(4, **i32))
+        api.moe_permute_shard(cfg, x, ids, wts, base, cap, off, perm_token, perm_w, slot_row, x_perm, stats, ws)
+        api.moe_grouped_ffn(cfg, x_perm, off, weights, y_perm, ws)
+        api.moe_combine(cfg, y_perm, slot_row, wts, None, out[lo:hi])
+        torch.cuda.synchronize()
+        assert api.moe_workspace_status(ws) == 0
+        slot_all.append(slot_row.cpu().numpy())
+    ids_all = torch.cat([p[3] for p in parts]).cpu().numpy()
+    wts_all = torch.cat([p[4] for p in parts]).cpu().numpy().astype(np.float64)
+    ref = O.dispatch(ids_all, w.E, cap, wts_all)
+    kept_gpu = np.concatenate(slot_all) >= 0
+    assert np.array_equal(kept_gpu, ref["slot_row"] >= 0)
+    assert ref["dropped"] > 0
+    res = O.layer_forward(to_host(inp["x"]), to_host(inp["w_router"]), HostExperts(inp), top_k=w.k, act=w.act,
+                          capacity_factor=w.capacity_factor, logit_bias=to_host(inp["logit_bias"]),
+                          routing=dict(ids=ids_all, weights=wts_all, probs=np.zeros((w.T, w.E))))
+    got = out.float().cpu().numpy().astype(np.float64)
+    err = float(np.abs(got - res["out"]).max() / np.abs(res["out"]).max())
+    assert err <= 2e-2, err
