@@ -15,12 +15,28 @@
 //               128-byte swizzle) into a stage; per tile the tile's scale and
 //               bias rows (contiguous in [E, N, K/64]) by bulk copy.
 //   warp 1      TMEM owner and single-thread tcgen05.mma issuer
-//               (kind::f16, M=128, N=32, K=16), commits free the stages.
-//   warps 2-17  dequantise codes into the K-major 128-byte-swizzled bf16
-//               operand (nibble -> exact bf16 through the 0x4300 magic, one
-//               bf16x2 FMA with the group's scale and bias: a single
-//               rounding of s*q + b), then run the tile epilogue:
-//               SwiGLU (gate, up accumulators) or a plain store of y.
+//               (kind::f16, M=128, N=32, K=16) with the weight operand read
+//               from TMEM and the token operand from shared memory; its
+//               commits hand the operand slots back.
+//   warps 2-17  dequantisers, in groups of 4 x (matrices) warps taking K-blocks
+//               round robin: read a stage's codes and token chunks into
+//               registers and release the stage at once, dequantise (nibble
+//               -> exact bf16 through the 0x4300 magic, one bf16x2 FMA with
+//               the group's scale and bias: a single rounding of s*q + b) and
+//               write the weight operand straight into a TMEM slot
+//               (tcgen05.st; thread = weight row = TMEM lane) and the token
+//               tile into that slot's shared buffer.
+//   warps 18-21 epilogue, one per TMEM lane quarter: SwiGLU of the gate and
+//               up accumulators into h, or a plain store of y.
+// Accumulators are double-buffered, so MMA and dequantisation stream across
+// tile boundaries while the epilogue drains the previous tile.  The operand
+// slots (6 with gate+up, 14 with one matrix) fill the rest of TMEM, so the
+// dequantisers run many K-blocks ahead of the MMA and the per-K-block
+// commit-to-reuse round trip stays hidden.
+// Inside every 8-element chunk both operands use the K order 0,4,1,5,2,6,3,7
+// (what the nibble extraction yields without byte permutes): phase 1
+// reorders its token tile in shared memory, and writes h already in that
+// order for phase 2.  Sums over K do not depend on the order.
 // Every mbarrier wait is bounded (2 s of %globaltimer) as in the bf16
 // grouped GEMM: on expiry the CTA records a status, drains its own TMA/MMA
 // work, frees TMEM and exits.
@@ -36,10 +52,10 @@ constexpr int BM = 128;                 // weight rows (features) per tile
 constexpr int BK = 64;                  // K per block = one quantisation group
 constexpr int NT = 32;                  // tokens per pass (MMA N)
 constexpr int DQ_WARPS = 16;
-constexpr int THREADS = 32 * (2 + DQ_WARPS);
+constexpr int EPI_WARPS = 4;            // one per TMEM lane quarter
+constexpr int THREADS = 32 * (2 + DQ_WARPS + EPI_WARPS);
 constexpr int CODE_BYTES = BM * BK / 2; // 4 KiB of codes per matrix per K-block
 constexpr int B_BYTES = NT * BK * 2;    // 4 KiB token tile per K-block
-constexpr int A_BYTES = BM * BK * 2;    // 16 KiB dequantised operand per matrix
 constexpr uint64_t TIMEOUT_NS = 2000000000ull;
 constexpr uint64_t DRAIN_NS = 200000000ull;
 
@@ -50,9 +66,13 @@ constexpr uint32_t IDESC = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(NT >
 template <bool PAIR>
 struct Q4Shape {
   static constexpr int MATS = PAIR ? 2 : 1;
-  static constexpr int STAGES = PAIR ? 6 : 8;
+  static constexpr int STAGES = PAIR ? 8 : 12;
   static constexpr int STAGE_BYTES = MATS * CODE_BYTES + B_BYTES;   // multiple of 1024
-  static constexpr int TMEM_COLS = PAIR ? 64 : 32;
+  static constexpr int ACC_COLS = MATS * NT;                        // fp32 accumulators of one tile
+  static constexpr int A_COLS = MATS * BK / 2;                      // one K-block of bf16 pairs per matrix
+  static constexpr int SLOTS = (512 - 2 * ACC_COLS) / A_COLS;       // operand slots in TMEM
+  static constexpr int WARPS_PER_KB = 4 * MATS;                     // one warp per (matrix, lane quarter)
+  static constexpr int GROUPS = DQ_WARPS / WARPS_PER_KB;            // K-blocks in flight in dequant
 };
 
 struct Q4Params {
@@ -69,10 +89,10 @@ struct Q4Params {
 };
 
 struct Q4Shared {
-  uint64_t full[8], empty[8];
-  uint64_t a_full[2], a_empty[2];
+  uint64_t full[12], empty[12];
+  uint64_t a_full[16], a_empty[16];
   uint64_t sc_full[2], sc_empty[2];
-  uint64_t acc_full;
+  uint64_t acc_full[2], acc_empty[2];
   uint64_t drain;
   uint32_t tmem_base;
   int abort_flag;
@@ -188,6 +208,27 @@ __device__ __forceinline__ void tmem_ld8(uint32_t taddr, uint32_t (&v)[8]) {
                : "r"(taddr));
 }
 
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&v)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+      "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, "
+      "%17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};" ::"r"(taddr),
+      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]),
+      "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15]), "r"(v[16]),
+      "r"(v[17]), "r"(v[18]), "r"(v[19]), "r"(v[20]), "r"(v[21]), "r"(v[22]), "r"(v[23]), "r"(v[24]),
+      "r"(v[25]), "r"(v[26]), "r"(v[27]), "r"(v[28]), "r"(v[29]), "r"(v[30]), "r"(v[31])
+      : "memory");
+}
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+// D (TMEM) += A (TMEM, M x 16, rows in lanes) * B (shared memory descriptor)
+__device__ __forceinline__ void tc_mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t accum) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %3, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %4, p;\n\t}\n" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(bdesc), "r"(accum), "r"(IDESC));
+}
+
 // bf16x2 arithmetic (one rounding per lane)
 __device__ __forceinline__ uint32_t bf2_sub(uint32_t a, uint32_t b) {
   uint32_t d;
@@ -205,9 +246,12 @@ __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
   return d;
 }
 
-// Eight 4-bit codes (element j at bits 4j) -> eight bf16 s*q + b, in order.
+// Eight 4-bit codes (element j at bits 4j) -> eight bf16 s*q + b.
 // (w >> 4i) & 0x000F000F | 0x43004300 is the bf16 pair (128 + q_i, 128 + q_{i+4});
 // subtracting 128 is exact, so each element is rounded once, in the FMA.
+// The chunk keeps that pairing: its 16 bytes hold elements in the order
+// 0,4,1,5,2,6,3,7 (the operand K order used throughout this kernel; the
+// token operand is stored in the same order, see permute_chunk).
 __device__ __forceinline__ uint4 dequant8(uint32_t w, uint32_t s2, uint32_t b2) {
   const uint32_t magic = 0x43004300u;   // bf16 128.0 in both halves
   uint32_t p[4];
@@ -216,13 +260,17 @@ __device__ __forceinline__ uint4 dequant8(uint32_t w, uint32_t s2, uint32_t b2) 
     const uint32_t v = ((w >> (4 * i)) & 0x000F000Fu) | magic;
     p[i] = bf2_fma(bf2_sub(v, magic), s2, b2);      // (q_i, q_{i+4})
   }
-  uint4 o;
-  o.x = prmt(p[0], p[1], 0x5410);   // (q0, q1)
-  o.y = prmt(p[2], p[3], 0x5410);   // (q2, q3)
-  o.z = prmt(p[0], p[1], 0x7632);   // (q4, q5)
-  o.w = prmt(p[2], p[3], 0x7632);   // (q6, q7)
-  return o;
+  return make_uint4(p[0], p[1], p[2], p[3]);
 }
+
+// Eight consecutive bf16 (e0..e7) -> the order e0,e4,e1,e5,e2,e6,e3,e7.
+__device__ __forceinline__ uint4 permute_chunk(uint4 c) {
+  return make_uint4(prmt(c.x, c.z, 0x5410), prmt(c.x, c.z, 0x7632), prmt(c.y, c.w, 0x5410),
+                    prmt(c.y, c.w, 0x7632));
+}
+
+// Position of logical element L (0..7) of an 8-element chunk in that order.
+__device__ __forceinline__ int chunk_pos(int L) { return L < 4 ? 2 * L : 2 * L - 7; }
 
 struct Tile {
   int e, row0, rows, m;
@@ -249,13 +297,14 @@ __global__ void __launch_bounds__(THREADS, 1)
 q4_tc_gemm(const __grid_constant__ CUtensorMap mapC0, const __grid_constant__ CUtensorMap mapC1,
            const __grid_constant__ CUtensorMap mapB, const Q4Params p) {
   using S = Q4Shape<PAIR>;
-  constexpr int MATS = S::MATS, STAGES = S::STAGES;
+  constexpr int MATS = S::MATS, STAGES = S::STAGES, SLOTS = S::SLOTS, GROUPS = S::GROUPS;
+  constexpr int WPK = S::WARPS_PER_KB;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   const uint32_t pad = (1024u - (smem_u32(smem_raw) & 1023u)) & 1023u;
   uint8_t *base = smem_raw + pad;
-  uint8_t *stages = base;                                            // STAGES x [codes(MATS) | B]
-  uint8_t *abuf = stages + (size_t)STAGES * S::STAGE_BYTES;         // 2 x MATS x A_BYTES
-  uint16_t *sbuf = reinterpret_cast<uint16_t *>(abuf + 2 * MATS * A_BYTES);   // 2 x MATS x {scale, bias}
+  uint8_t *stages = base;                                            // STAGES x [codes(MATS) | tokens]
+  uint8_t *bslots = stages + (size_t)STAGES * S::STAGE_BYTES;       // SLOTS x token tile (operand K order)
+  uint16_t *sbuf = reinterpret_cast<uint16_t *>(bslots + (size_t)SLOTS * B_BYTES);   // 2 x MATS x {scale, bias}
   const int sc_elems = BM * p.kgroups;                               // per matrix per kind
   Q4Shared *st = reinterpret_cast<Q4Shared *>(sbuf + 2 * MATS * 2 * sc_elems + 64);   // +128 bytes
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -266,15 +315,20 @@ q4_tc_gemm(const __grid_constant__ CUtensorMap mapC0, const __grid_constant__ CU
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(&st->full[s], 1);
-      mbar_init(&st->empty[s], DQ_WARPS + 1);   // dequant warps read codes, MMA reads B
+      mbar_init(&st->empty[s], WPK);         // the warps that dequantise that K-block
+    }
+    for (int j = 0; j < SLOTS; ++j) {
+      mbar_init(&st->a_full[j], WPK);
+      mbar_init(&st->a_empty[j], 1);
     }
     for (int b = 0; b < 2; ++b) {
-      mbar_init(&st->a_full[b], DQ_WARPS);
-      mbar_init(&st->a_empty[b], 1);
       mbar_init(&st->sc_full[b], 1);
       mbar_init(&st->sc_empty[b], DQ_WARPS);
     }
-    mbar_init(&st->acc_full, 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&st->acc_full[b], 1);
+      mbar_init(&st->acc_empty[b], EPI_WARPS);   // the epilogue warps done reading the accumulators
+    }
     mbar_init(&st->drain, 1);
     st->abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -282,7 +336,7 @@ q4_tc_gemm(const __grid_constant__ CUtensorMap mapC0, const __grid_constant__ CU
   }
   if (warp == 1) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&st->tmem_base)),
-                 "r"((uint32_t)S::TMEM_COLS)
+                 "r"(512u)
                  : "memory");
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
   }
@@ -365,49 +419,56 @@ q4_tc_gemm(const __grid_constant__ CUtensorMap mapC0, const __grid_constant__ CU
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      uint32_t it = 0, ab = 0;
+      uint32_t it = 0, tcount = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
-        for (int kb = 0; kb < kb_n; ++kb, ++it, ++ab) {
-          const int s = it % STAGES;
-          const uint32_t ph = (it / STAGES) & 1u;
-          const uint32_t b = ab & 1u;
-          if (!wait_bounded(&st->full[s], ph, abort_flag, p.status, kDevTimeoutMma) ||
-              !wait_bounded(&st->a_full[b], (ab >> 1) & 1u, abort_flag, p.status, kDevTimeoutMma)) {
+      for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x, ++tcount) {
+        // accumulator buffer tcount % 2: the epilogue of two tiles ago must be done with it
+        const uint32_t abuf = tcount & 1u;
+        if (!wait_bounded(&st->acc_empty[abuf], ((tcount >> 1) & 1u) ^ 1u, abort_flag, p.status, kDevTimeoutMma)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t dcol = tmem_base + abuf * S::ACC_COLS;
+        for (int kb = 0; kb < kb_n; ++kb, ++it) {
+          const uint32_t j = it % SLOTS, use = it / SLOTS;
+          if (!wait_bounded(&st->a_full[j], use & 1u, abort_flag, p.status, kDevTimeoutMma)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint32_t bsm = smem_u32(stages + (size_t)s * S::STAGE_BYTES + MATS * CODE_BYTES);
-          const uint64_t db = sw128_desc(bsm);
+          const uint64_t db = sw128_desc(smem_u32(bslots + (size_t)j * B_BYTES));
+          const uint32_t acol = tmem_base + 2 * S::ACC_COLS + j * S::A_COLS;
 #pragma unroll
           for (int m = 0; m < MATS; ++m) {
-            const uint64_t da = sw128_desc(smem_u32(abuf + ((size_t)b * MATS + m) * A_BYTES));
 #pragma unroll
             for (int kk = 0; kk < BK / 16; ++kk)
-              tc_mma(tmem_base + m * NT, da + (uint64_t)(kk * 2), db + (uint64_t)(kk * 2), (kb | kk) != 0 ? 1u : 0u);
+              tc_mma_ts(dcol + m * NT, acol + m * (BK / 2) + kk * 8, db + (uint64_t)(kk * 2),
+                        (kb | kk) != 0 ? 1u : 0u);
           }
-          tc_commit(&st->a_empty[b]);
-          tc_commit(&st->empty[s]);
+          tc_commit(&st->a_empty[j]);
         }
         if (!ok) break;
-        tc_commit(&st->acc_full);
+        tc_commit(&st->acc_full[abuf]);
       }
       tc_commit(&st->drain);
       if (!wait_drain(&st->drain, 0u)) record_status(p.status, kDevTimeoutDrain);
     }
     __syncwarp();
-  } else {
-    // ------------------------------------------------------------ dequant + epilogue
-    const int dt = threadIdx.x - 64;                    // 0 .. 32*DQ_WARPS-1
-    constexpr int PER_MAT = 32 * DQ_WARPS / MATS;       // threads per matrix
-    constexpr int PARTS = PER_MAT / BM;                  // threads per weight row
-    constexpr int WORDS = 8 / PARTS;                     // 32-bit code words per thread per K-block
-    const int mat = dt / PER_MAT;
-    const int row = (dt % PER_MAT) / PARTS;
-    const int part = dt % PARTS;
-    const uint32_t stages_sa = smem_u32(stages), abuf_sa = smem_u32(abuf);
-    uint32_t it = 0, ab = 0, tc = 0;
+  } else if (warp < 2 + DQ_WARPS) {
+    // ------------------------------------------------------------ dequant
+    // GROUPS groups of WPK warps take K-blocks round robin.  Inside a group a
+    // warp owns one matrix and one TMEM lane quarter: thread = weight row
+    // (= TMEM lane), 64 codes per K-block, stored as 32 columns of bf16 pairs.
+    const int dw = warp - 2;
+    const int grp = dw / WPK;
+    const int gt = (dw % WPK) * 32 + lane;              // thread within the group
+    const int mat = (dw % WPK) / 4;
+    const int q = warp & 3;                             // TMEM lane quarter this warp may access
+    const int row = q * 32 + lane;
+    constexpr int BCH = (B_BYTES / 16) / (32 * WPK);    // token-tile chunks per thread
+    const uint32_t stages_sa = smem_u32(stages), bslots_sa = smem_u32(bslots);
+    uint32_t tc = 0;
     bool ok = true;
     for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x, ++tc) {
       const Tile ti = decode_tile(st, nE, m_tiles, tile);
@@ -418,90 +479,112 @@ q4_tc_gemm(const __grid_constant__ CUtensorMap mapC0, const __grid_constant__ CU
       }
       const uint32_t scl = smem_u32(sbuf + ((size_t)sb * MATS + mat) * 2 * sc_elems + (size_t)row * p.kgroups);
       const uint32_t bis = scl + 2u * (uint32_t)sc_elems;
-      for (int kb = 0; kb < kb_n; ++kb, ++it, ++ab) {
-        const int s = it % STAGES;
+      const uint32_t it0 = tc * (uint32_t)kb_n;
+      const int kb_first = (int)((grp - (int)(it0 % GROUPS) + GROUPS) % GROUPS);
+      for (int kb = kb_first; kb < kb_n; kb += GROUPS) {
+        const uint32_t it = it0 + kb;                    // it % GROUPS == grp
+        const int s = (int)(it % STAGES);
         const uint32_t ph = (it / STAGES) & 1u;
-        const uint32_t b = ab & 1u;
+        const uint32_t j = it % SLOTS, use = it / SLOTS;
         if (!wait_bounded(&st->full[s], ph, abort_flag, p.status, kDevTimeoutEpilogue)) {
           ok = false;
           break;
         }
-        const uint32_t cp = stages_sa + (uint32_t)(s * S::STAGE_BYTES + mat * CODE_BYTES + row * (BK / 2) +
-                                                   part * (WORDS * 4));
-        uint32_t wv[WORDS];
+        const uint32_t stage_sa = stages_sa + (uint32_t)(s * S::STAGE_BYTES);
+        const uint32_t cp = stage_sa + (uint32_t)(mat * CODE_BYTES + row * (BK / 2));
+        const uint4 c0 = lds128(cp), c1 = lds128(cp + 16);
+        const uint32_t wv[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+        // token tile chunks (phase 1 reorders them into the operand K order;
+        // phase 2's token tile, h, already is in it)
+        uint4 bch[BCH];
 #pragma unroll
-        for (int q = 0; q < (WORDS + 3) / 4; ++q) {
-          if constexpr (WORDS >= 4) {
-            const uint4 u = lds128(cp + 16 * q);
-            wv[4 * q] = u.x; wv[4 * q + 1] = u.y; wv[4 * q + 2] = u.z; wv[4 * q + 3] = u.w;
-          } else {
-            uint32_t a0, a1;
-            asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(a0), "=r"(a1) : "r"(cp));
-            wv[0] = a0;
-            wv[WORDS - 1] = a1;
-          }
+        for (int i = 0; i < BCH; ++i) {
+          bch[i] = lds128(stage_sa + (uint32_t)(MATS * CODE_BYTES) + (uint32_t)(gt + i * 32 * WPK) * 16u);
+          if (PAIR) bch[i] = permute_chunk(bch[i]);
         }
+        // the stage's bytes are all in registers: hand it back to the producer
         __syncwarp();
         if (lane == 0) mbar_arrive(&st->empty[s]);
         const uint32_t s1 = lds16(scl + 2u * kb), b1 = lds16(bis + 2u * kb);
         const uint32_t s2 = s1 | (s1 << 16), b2 = b1 | (b1 << 16);
-        if (!wait_bounded(&st->a_empty[b], ((ab >> 1) & 1u) ^ 1u, abort_flag, p.status, kDevTimeoutEpilogue)) {
+        uint32_t av[32];
+#pragma unroll
+        for (int w = 0; w < 8; ++w) {
+          const uint4 d = dequant8(wv[w], s2, b2);
+          av[4 * w] = d.x; av[4 * w + 1] = d.y; av[4 * w + 2] = d.z; av[4 * w + 3] = d.w;
+        }
+        if (!wait_bounded(&st->a_empty[j], (use & 1u) ^ 1u, abort_flag, p.status, kDevTimeoutEpilogue)) {
           ok = false;
           break;
         }
-        const uint32_t arow = abuf_sa + (uint32_t)((b * MATS + mat) * A_BYTES + row * 128);
+        tc_fence_after();
+        tmem_st32(tmem_base + ((uint32_t)(q * 32) << 16) + 2 * S::ACC_COLS + j * S::A_COLS + mat * (BK / 2), av);
 #pragma unroll
-        for (int w = 0; w < WORDS; ++w) {
-          const int chunk = part * WORDS + w;   // 16-byte chunk = 8 elements of the 64
-          sts128(arow + ((chunk ^ (row & 7)) << 4), dequant8(wv[w], s2, b2));
-        }
+        for (int i = 0; i < BCH; ++i)
+          sts128(bslots_sa + j * (uint32_t)B_BYTES + (uint32_t)(gt + i * 32 * WPK) * 16u, bch[i]);
+        tmem_wait_st();
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&st->a_full[b]);
+        if (lane == 0) mbar_arrive(&st->a_full[j]);
       }
       if (!ok) break;
       // scale rows of this tile no longer needed
       __syncwarp();
       if (lane == 0) mbar_arrive(&st->sc_empty[sb]);
-      // epilogue: warp quarter q reads TMEM lanes 32q..32q+31, group g the tokens 8g..8g+7
-      if (!wait_bounded(&st->acc_full, tc & 1u, abort_flag, p.status, kDevTimeoutEpilogue)) {
-        ok = false;
-        break;
-      }
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    // warp quarter q reads TMEM lanes 32q..32q+31 (weight rows), 32 token columns
+    const int q = warp & 3;
+    const int row = q * 32 + lane;
+    uint32_t tc = 0;
+    for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++tc) {
+      const Tile ti = decode_tile(st, nE, m_tiles, tile);
+      const uint32_t abuf = tc & 1u;
+      if (!wait_bounded(&st->acc_full[abuf], (tc >> 1) & 1u, abort_flag, p.status, kDevTimeoutEpilogue)) break;
       tc_fence_after();
-      const int q = warp & 3;
-      const int g = (warp - 2) >> 2;
-      const uint32_t ta = tmem_base + ((uint32_t)(q * 32) << 16) + g * 8;
-      const int f = ti.m * BM + q * 32 + lane;
+      const uint32_t ta = tmem_base + ((uint32_t)(q * 32) << 16) + abuf * S::ACC_COLS;
+      const int f = ti.m * BM + row;
       if (PAIR) {
-        uint32_t gv8[8], uv8[8];
-        tmem_ld8(ta, gv8);
-        tmem_ld8(ta + NT, uv8);
-        tmem_wait_ld();
+        uint32_t gv[16], uv[16];
 #pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          const int tok = g * 8 + c;
-          if (tok < ti.rows) {
-            const float gv = __uint_as_float(gv8[c]);
-            const float hv = gv / (1.f + __expf(-gv)) * __uint_as_float(uv8[c]);
-            const __nv_bfloat16 hb = __float2bfloat16_rn(hv);
-            p.out[(size_t)(ti.row0 + tok) * p.N + f] = *reinterpret_cast<const uint16_t *>(&hb);
+        for (int half = 0; half < 2; ++half) {
+          tmem_ld16(ta + half * 16, gv);
+          tmem_ld16(ta + NT + half * 16, uv);
+          tmem_wait_ld();
+#pragma unroll
+          for (int c = 0; c < 16; ++c) {
+            const int tok = half * 16 + c;
+            if (tok < ti.rows) {
+              const float g = __uint_as_float(gv[c]);
+              const float hv = g / (1.f + __expf(-g)) * __uint_as_float(uv[c]);
+              const __nv_bfloat16 hb = __float2bfloat16_rn(hv);
+              // h is the next phase's token operand: stored in its K order
+              p.out[(size_t)(ti.row0 + tok) * p.N + ((f & ~7) | chunk_pos(f & 7))] =
+                  *reinterpret_cast<const uint16_t *>(&hb);
+            }
           }
         }
       } else {
-        uint32_t y[8];
-        tmem_ld8(ta, y);
-        tmem_wait_ld();
+        uint32_t y[16];
 #pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          const int tok = g * 8 + c;
-          if (tok < ti.rows) {
-            const __nv_bfloat16 yb = __float2bfloat16_rn(__uint_as_float(y[c]));
-            p.out[(size_t)(ti.row0 + tok) * p.N + f] = *reinterpret_cast<const uint16_t *>(&yb);
+        for (int half = 0; half < 2; ++half) {
+          tmem_ld16(ta + half * 16, y);
+          tmem_wait_ld();
+#pragma unroll
+          for (int c = 0; c < 16; ++c) {
+            const int tok = half * 16 + c;
+            if (tok < ti.rows) {
+              const __nv_bfloat16 yb = __float2bfloat16_rn(__uint_as_float(y[c]));
+              p.out[(size_t)(ti.row0 + tok) * p.N + f] = *reinterpret_cast<const uint16_t *>(&yb);
+            }
           }
         }
       }
       tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&st->acc_empty[abuf]);
     }
   }
 
@@ -509,9 +592,7 @@ q4_tc_gemm(const __grid_constant__ CUtensorMap mapC0, const __grid_constant__ CU
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
-                 "r"((uint32_t)S::TMEM_COLS)
-                 : "memory");
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(512u) : "memory");
   }
 }
 
@@ -565,7 +646,7 @@ int sm_count() {
 template <bool PAIR>
 size_t smem_bytes(int kgroups) {
   using S = Q4Shape<PAIR>;
-  return 1024 + (size_t)S::STAGES * S::STAGE_BYTES + 2 * S::MATS * A_BYTES +
+  return 1024 + (size_t)S::STAGES * S::STAGE_BYTES + (size_t)S::SLOTS * B_BYTES +
          2 * S::MATS * 2 * (size_t)BM * kgroups * 2 + 128 + sizeof(Q4Shared);
 }
 
