@@ -69,6 +69,13 @@ typedef enum moe_dtype {
   MOE_Q4_AFFINE_G64 = 2   /* weights only: Edge0 QuantSpec(bits=4, group_size=64, mode=affine) */
 } moe_dtype;
 
+/* How the gate and up projections are stored ("MoE Spec and Routing",
+ * WeightLayout and "Bundle layout and the up-first order"). */
+typedef enum moe_weight_layout {
+  MOE_LAYOUT_SEPARATE = 0,        /* w1 = gate [E,F,d], w2 = up [E,F,d] */
+  MOE_LAYOUT_FUSED_GATE_UP = 1    /* w1 = gate_up [E,2F,d]: per expert, F gate rows then F up rows; w2 = NULL */
+} moe_weight_layout;
+
 /*
  * Layer configuration (the blog's MoEConfig and Edge0's MoESpec, flattened
  * into plain fields).  Enum-valued fields are int32 so the layout is fixed.
@@ -90,6 +97,7 @@ typedef struct moe_config {
   int32_t weight_dtype;         /* MOE_F32 (with F32 act), MOE_BF16 or MOE_Q4_AFFINE_G64 (with BF16 act) */
   int32_t shared_intermediate;  /* 0: no shared expert; else the shared SwiGLU expert's width */
   float aux_alpha;              /* balancing-loss coefficient >= 0 (blog default 0.01) */
+  int32_t weight_layout;        /* moe_weight_layout; FUSED_GATE_UP needs SwiGLU */
 } moe_config;
 
 /*
@@ -102,6 +110,13 @@ typedef struct moe_config {
  * 4*(j%8) of word j/8), and scale_i / bias_i are bf16 [E, N, K/64]: the
  * weight is scale*q + bias, one scale/bias pair per 64 consecutive elements
  * of the reduction axis K (d for w1/w2, F for w3).
+ * With weight_layout = MOE_LAYOUT_FUSED_GATE_UP the gate and up matrices
+ * come as ONE tensor in w1, [E, 2F, d] (Q4: codes [E, 2F, d/8], scale1 /
+ * bias1 [E, 2F, d/64]): expert e's F gate rows are followed by its F up rows,
+ * so splitting one expert's projection into two halves along the output axis
+ * gives (gate, up), and the experts' blocks are interleaved, not two stacked
+ * tensors.  w2, scale2 and bias2 must then be NULL.  The shared expert always
+ * uses the separate layout.
  *   shared1/2/3: the always-active shared expert (MoE competition docs:
  *   "Shared expert"; Edge0 MoESpec.shared_experts), SwiGLU,
  *   [Fs, d], [Fs, d], [d, Fs] in act_dtype; NULL when shared_intermediate = 0.
@@ -224,6 +239,43 @@ moe_status moe_route(const moe_config *cfg, const void *x, const float *w_router
 moe_status moe_route_noalloc(const moe_config *cfg, const void *x, const float *w_router,
                              const float *router_bias, int32_t *topk_ids, float *topk_w,
                              float *prob_sum, moe_stream_t stream);
+
+/* Router replay ("Mixture-of-Experts" design doc, Router replay (R3)): the
+ * expert choice is forced to recorded ids while the weights still come from
+ * this router's own gate.  Logits, scores and prob_sum are those of
+ * moe_route; then token t's slots j = 0..k-1 take expert forced_ids[t, j] in
+ * that order, weighted as moe_route weights its own choices:
+ *   softmax_topk:  w_j = p[t, id_j], or p[t, id_j] / max(sum_j p[t, id_j], 1e-12)
+ *                  when norm_topk_prob;
+ *   sigmoid_group: w_j = s[t, id_j] [/ (sum_j s[t, id_j] + 1e-20)] * routed_scaling
+ *                  (the selection bias and the group limit take no part).
+ * In:  forced_ids [T,k] int32 device, k distinct ids in [0, E) per token.
+ * Out: topk_ids [T,k] (a copy of forced_ids), topk_w [T,k], prob_sum [E].
+ * A recorded id outside [0, E) (a missing-route sentinel) or one repeated in
+ * its row is not replayed silently: its slot gets weight 0 and is left out of
+ * the normalising sum, and the call records a device status, which
+ * moe_workspace_status(ws) reports as MOE_ERR_DEVICE (moe_permute rejects
+ * the same ids).  Uses ws. */
+moe_status moe_route_forced(const moe_config *cfg, const void *x, const float *w_router,
+                            const float *router_bias, const int32_t *forced_ids, int32_t *topk_ids,
+                            float *topk_w, float *prob_sum, void *ws, size_t ws_bytes,
+                            moe_stream_t stream);
+
+/* Aux-loss-free balancing bias update ("Mixture-of-Experts" design doc,
+ * Aux-loss-free load balancing): each expert's routing bias takes one step of
+ * size coeff toward balanced use, up for an under-used expert and down for an
+ * over-used one:
+ *   mean = sum_e counts[e] / E;
+ *   expert_bias[e] += coeff if counts[e] < mean; -= coeff if counts[e] > mean;
+ *   unchanged if counts[e] == mean (compared exactly, as E*counts[e] vs the sum).
+ * counts [E] int32 device: the step's assignments per expert, normally
+ * moe_stats.raw_counts (before the capacity cut).  expert_bias [E] f32
+ * device, updated in place by one fp32 add.  coeff: the step size
+ * (load_balance_coeff), >= 0 and finite, else MOE_ERR_INVALID_ARG; 0 leaves
+ * the bias as it is (the scheme off).  Only num_experts of cfg is used
+ * beyond validation.  Stream-ordered, no workspace, one launch. */
+moe_status moe_update_bias(const moe_config *cfg, const int32_t *counts, float *expert_bias, float coeff,
+                           moe_stream_t stream);
 
 /* Dispatch (blog moe_layer capacity loop; route_and_sort / SortedRouting).
  * A slot (t, j) with expert e is kept iff fewer than `capacity` slots of e

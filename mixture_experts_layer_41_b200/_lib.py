@@ -33,6 +33,9 @@ MOE_ACT_SWIGLU = 1
 MOE_F32 = 0
 MOE_BF16 = 1
 MOE_Q4_AFFINE_G64 = 2
+# moe_weight_layout
+MOE_LAYOUT_SEPARATE = 0
+MOE_LAYOUT_FUSED_GATE_UP = 1
 
 
 class moe_config(C.Structure):
@@ -53,6 +56,7 @@ class moe_config(C.Structure):
         ("weight_dtype", C.c_int32),
         ("shared_intermediate", C.c_int32),
         ("aux_alpha", C.c_float),
+        ("weight_layout", C.c_int32),
     ]
 
 
@@ -86,6 +90,8 @@ SIGNATURES = {
     "moe_set_phase_events": (C.c_int, [C.POINTER(C.c_void_p), C.c_int32]),
     "moe_route": (C.c_int, [_CFG, _P, _P, _P, _P, _P, _P, _P, C.c_size_t, _P]),
     "moe_route_noalloc": (C.c_int, [_CFG, _P, _P, _P, _P, _P, _P, _P]),
+    "moe_route_forced": (C.c_int, [_CFG, _P, _P, _P, _P, _P, _P, _P, _P, C.c_size_t, _P]),
+    "moe_update_bias": (C.c_int, [_CFG, _P, _P, C.c_float, _P]),
     "moe_permute": (C.c_int, [_CFG, _P, _P, _P, _P, _P, _P, _P, _P, _S, _P, C.c_size_t, _P]),
     "moe_expert_counts": (C.c_int, [_CFG, _P, _P, _P, C.c_size_t, _P]),
     "moe_permute_shard": (C.c_int, [_CFG, _P, _P, _P, _P, C.c_int64, _P, _P, _P, _P, _P, _S, _P, C.c_size_t, _P]),

@@ -20,17 +20,19 @@ _ROUTERS = {"softmax_topk": L.MOE_ROUTER_SOFTMAX_TOPK, "sigmoid_group": L.MOE_RO
 _ACTS = {"relu": L.MOE_ACT_RELU, "swiglu": L.MOE_ACT_SWIGLU}
 _DTYPES = {"f32": L.MOE_F32, "bf16": L.MOE_BF16, "q4_affine_g64": L.MOE_Q4_AFFINE_G64}
 _TORCH_DT = {L.MOE_F32: torch.float32, L.MOE_BF16: torch.bfloat16}
+_LAYOUTS = {"separate": L.MOE_LAYOUT_SEPARATE, "fused_gate_up": L.MOE_LAYOUT_FUSED_GATE_UP}
 
 
 def make_config(*, num_tokens: int, hidden: int, intermediate: int, num_experts: int, top_k: int,
                 router: str = "softmax_topk", norm_topk_prob: bool = True, routed_scaling: float = 1.0,
                 n_group: int = 1, topk_group: int = 1, capacity_factor: float = 0.0,
                 act: str = "swiglu", act_dtype: str = "bf16", weight_dtype: str = "bf16",
-                shared_intermediate: int = 0, aux_alpha: float = 0.01) -> moe_config:
+                shared_intermediate: int = 0, aux_alpha: float = 0.01,
+                weight_layout: str = "separate") -> moe_config:
     return moe_config(num_tokens, hidden, intermediate, num_experts, top_k, _ROUTERS[router],
                       1 if norm_topk_prob else 0, routed_scaling, n_group, topk_group,
                       capacity_factor, _ACTS[act], _DTYPES[act_dtype], _DTYPES[weight_dtype],
-                      shared_intermediate, aux_alpha)
+                      shared_intermediate, aux_alpha, _LAYOUTS[weight_layout])
 
 
 def _p(t: Optional[torch.Tensor]):
@@ -121,6 +123,17 @@ def _stats_struct(stats: Optional[dict]) -> Optional[moe_stats]:
 def moe_route(cfg, x, w_router, router_bias, topk_ids, topk_w, prob_sum, ws, stream=None):
     check(L.lib().moe_route(C.byref(cfg), _p(x), _p(w_router), _p(router_bias), _p(topk_ids), _p(topk_w),
                             _p(prob_sum), _p(ws), _nbytes(ws), _s(stream)), "moe_route")
+
+
+def moe_route_forced(cfg, x, w_router, router_bias, forced_ids, topk_ids, topk_w, prob_sum, ws, stream=None):
+    check(L.lib().moe_route_forced(C.byref(cfg), _p(x), _p(w_router), _p(router_bias), _p(forced_ids),
+                                   _p(topk_ids), _p(topk_w), _p(prob_sum), _p(ws), _nbytes(ws), _s(stream)),
+          "moe_route_forced")
+
+
+def moe_update_bias(cfg, counts, expert_bias, coeff: float, stream=None):
+    check(L.lib().moe_update_bias(C.byref(cfg), _p(counts), _p(expert_bias), coeff, _s(stream)),
+          "moe_update_bias")
 
 
 def moe_route_noalloc(cfg, x, w_router, router_bias, topk_ids, topk_w, prob_sum, stream=None):
@@ -250,11 +263,45 @@ class MoELayer:
         o = self.o
         return dict(raw_counts=o.raw_counts, kept_counts=o.kept_counts, prob_sum=o.prob_sum, dropped=o.dropped)
 
-    def forward(self, x: torch.Tensor, stream=None) -> Outputs:
+    def forward(self, x: torch.Tensor, stream=None, forced_ids: Optional[torch.Tensor] = None) -> Outputs:
+        """One layer forward.  ``forced_ids`` [T, k] int32 replays recorded
+        expert choices (router replay): the stages then run one by one, with
+        moe_route_forced in place of the router.  Bad recorded ids surface, as
+        in moe_forward, through ``status()`` (the dispatch flags them too)."""
         o = self.o
-        moe_forward(self.cfg, x, self.w_router, self.router_bias, self.weights, o.out, o.topk_ids, o.topk_w,
-                    self.stats(), self.ws, stream)
+        if forced_ids is None:
+            moe_forward(self.cfg, x, self.w_router, self.router_bias, self.weights, o.out, o.topk_ids,
+                        o.topk_w, self.stats(), self.ws, stream)
+            return o
+        cfg = self.cfg
+        T, k, d = cfg.num_tokens, cfg.top_k, cfg.hidden
+        if not hasattr(self, "_stage"):
+            i32 = dict(dtype=torch.int32, device=self.device)
+            dt = _TORCH_DT[cfg.act_dtype]
+            self._stage = dict(off=torch.empty(cfg.num_experts + 1, **i32), perm_token=torch.empty(T * k, **i32),
+                               perm_w=torch.empty(T * k, dtype=torch.float32, device=self.device),
+                               slot_row=torch.empty((T, k), **i32),
+                               x_perm=torch.empty((T * k, d), dtype=dt, device=self.device),
+                               y_perm=torch.empty((T * k, d), dtype=dt, device=self.device),
+                               shared=torch.empty((T, d), dtype=dt, device=self.device)
+                               if cfg.shared_intermediate > 0 else None)
+        st = self._stage
+        moe_route_forced(cfg, x, self.w_router, self.router_bias, forced_ids, o.topk_ids, o.topk_w, o.prob_sum,
+                         self.ws, stream)
+        moe_permute(cfg, x, o.topk_ids, o.topk_w, st["off"], st["perm_token"], st["perm_w"], st["slot_row"],
+                    st["x_perm"], self.stats(), self.ws, stream)
+        moe_grouped_ffn(cfg, st["x_perm"], st["off"], self.weights, st["y_perm"], self.ws, stream)
+        if st["shared"] is not None:
+            moe_shared_expert(cfg, x, self.weights, st["shared"], self.ws, stream)
+        moe_combine(cfg, st["y_perm"], st["slot_row"], o.topk_w, st["shared"], o.out, stream)
         return o
+
+    def update_bias(self, coeff: float, stream=None) -> None:
+        """Aux-loss-free balancing step on ``router_bias`` from the last
+        forward's raw per-expert counts (moe_update_bias)."""
+        if self.router_bias is None:
+            raise ValueError("update_bias needs a router_bias tensor")
+        moe_update_bias(self.cfg, self.o.raw_counts, self.router_bias, coeff, stream)
 
     def status(self, stream=None) -> int:
         return moe_workspace_status(self.ws, stream)

@@ -148,7 +148,10 @@ RoutePlan route_plan(const moe_config &c, bool allow_split);
 cudaError_t launch_route(const moe_config &c, const void *x, const float *w_router,
                          const float *router_bias, int32_t *topk_ids, float *topk_w,
                          double *route_part, float *prob_sum, cudaStream_t s,
-                         double *logits = nullptr);
+                         double *logits = nullptr, const int32_t *forced_ids = nullptr,
+                         int *status = nullptr);
+// Aux-loss-free balancing: expert_bias[e] += coeff * sign(sum(counts) - E * counts[e]).
+cudaError_t launch_bias_update(int E, const int32_t *counts, float *expert_bias, float coeff, cudaStream_t s);
 
 cudaError_t launch_permute(const moe_config &c, const void *x, const int32_t *topk_ids,
                            const float *topk_w, int64_t capacity, int32_t *expert_offsets,
@@ -171,6 +174,8 @@ struct FfnArgs {
   const void *x;            // [rows_cap, d]
   const void *w1, *w2, *w3; // [E,F,d], [E,F,d], [E,d,F] (q4: packed codes)
   const void *s1, *s2, *s3, *b1, *b2, *b3;  // q4 scale / bias
+  int w_stride;             // rows from one expert's w1 (w2) block to the next: F, or 2F when
+                            // gate and up rows are stacked per expert (w2 = w1 + F rows)
   void *h;                  // [rows_cap, F]
   void *y;                  // [rows_cap, d]
   int *status;

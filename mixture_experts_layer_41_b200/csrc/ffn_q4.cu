@@ -26,6 +26,7 @@ constexpr int SMEM_ROW_LIMIT = 96 * 1024;
 struct Q4Args {
   const int32_t *offsets;
   int E, K, N, rows_cap;
+  int w_stride;                    // weight rows from one expert to the next (N, or 2N for stacked gate/up)
   const uint16_t *a;               // activations [rows_cap, K] bf16
   const uint32_t *q0, *q1;         // codes [E, N, K/8] (q1 only for the SwiGLU pair)
   const uint16_t *s0, *s1, *b0, *b1;   // [E, N, K/64] bf16
@@ -98,7 +99,7 @@ q4_gemm(Q4Args a) {
     for (int fi = warp; fi < FEAT; fi += WARPS) {
       const int f = f0 + fi;
       if (f >= a.N) break;
-      const size_t row = (size_t)e * a.N + f;
+      const size_t row = (size_t)e * a.w_stride + f;
       float acc0[MAXR], acc1[MAXR];
 #pragma unroll
       for (int r = 0; r < MAXR; ++r) { acc0[r] = 0.f; acc1[r] = 0.f; }
@@ -159,6 +160,7 @@ cudaError_t launch_ffn_q4(const FfnArgs &f, cudaStream_t s) {
   a.b1 = static_cast<const uint16_t *>(f.b2);
   a.out = static_cast<uint16_t *>(f.h);
   a.swiglu = 1;
+  a.w_stride = f.w_stride;
   cudaError_t err = run_q4(a, f.F, f.d, s);
   if (err != cudaSuccess) return err;
   if (f.mid_event && (err = cudaEventRecord(f.mid_event, s)) != cudaSuccess) return err;
@@ -171,6 +173,7 @@ cudaError_t launch_ffn_q4(const FfnArgs &f, cudaStream_t s) {
   a.s1 = a.b1 = nullptr;
   a.out = static_cast<uint16_t *>(f.y);
   a.swiglu = 0;
+  a.w_stride = f.d;
   return run_q4(a, f.d, f.F, s);
 }
 

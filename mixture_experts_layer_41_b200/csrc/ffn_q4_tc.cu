@@ -80,6 +80,7 @@ struct Q4Params {
   int E;
   int rows_cap;
   int N;                    // weight rows per expert (output features)
+  int w_stride;             // rows from one expert's block to the next (N, or 2N for stacked gate/up)
   int K;                    // reduction length
   int kgroups;              // K / 64
   const uint16_t *sc[2];    // [E, N, K/64] bf16 scales (gate / up, or down)
@@ -374,7 +375,7 @@ q4_tc_gemm(const __grid_constant__ CUtensorMap mapC0, const __grid_constant__ CU
       bool ok = true;
       for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x, ++tc) {
         const Tile ti = decode_tile(st, nE, m_tiles, tile);
-        const int wrow = ti.e * p.N + ti.m * BM;           // first weight row of the tile
+        const int wrow = ti.e * p.w_stride + ti.m * BM;           // first weight row of the tile
         // scale / bias rows of the tile: contiguous BM * kgroups bf16 per tensor
         const uint32_t sb = tc & 1u;
         if (!wait_bounded(&st->sc_empty[sb], ((tc >> 1) & 1u) ^ 1u, abort_flag, p.status, kDevTimeoutProducer)) {
@@ -651,10 +652,11 @@ size_t smem_bytes(int kgroups) {
 }
 
 template <bool PAIR>
-cudaError_t run(const FfnArgs &a, const void *tokens, int K, int N, const void *c0, const void *c1, const void *s0,
-                const void *s1, const void *b0, const void *b1, void *out, cudaStream_t s) {
+cudaError_t run(const FfnArgs &a, const void *tokens, int K, int N, int w_stride, const void *c0, const void *c1,
+                const void *s0, const void *s1, const void *b0, const void *b1, void *out, cudaStream_t s) {
   CUtensorMap mc0, mc1, mb;
-  const uint64_t wrows = (uint64_t)a.E * N;
+  // rows a map may address: the last expert's block ends N rows past its start
+  const uint64_t wrows = (uint64_t)(a.E - 1) * w_stride + N;
   cudaError_t err = map_codes(&mc0, c0, (uint64_t)K / 2, wrows);
   if (err == cudaSuccess) err = map_codes(&mc1, PAIR ? c1 : c0, (uint64_t)K / 2, wrows);
   if (err == cudaSuccess) err = map_tokens(&mb, tokens, (uint64_t)K, (uint64_t)a.rows_cap);
@@ -664,6 +666,7 @@ cudaError_t run(const FfnArgs &a, const void *tokens, int K, int N, const void *
   p.E = a.E;
   p.rows_cap = a.rows_cap;
   p.N = N;
+  p.w_stride = w_stride;
   p.K = K;
   p.kgroups = K / BK;
   p.sc[0] = static_cast<const uint16_t *>(s0);
@@ -694,10 +697,10 @@ bool q4_tc_supported(int d, int F) {
 }
 
 cudaError_t launch_ffn_q4_tc(const FfnArgs &a, cudaStream_t s) {
-  cudaError_t err = run<true>(a, a.x, a.d, a.F, a.w1, a.w2, a.s1, a.s2, a.b1, a.b2, a.h, s);
+  cudaError_t err = run<true>(a, a.x, a.d, a.F, a.w_stride, a.w1, a.w2, a.s1, a.s2, a.b1, a.b2, a.h, s);
   if (err != cudaSuccess) return err;
   if (a.mid_event && (err = cudaEventRecord(a.mid_event, s)) != cudaSuccess) return err;
-  return run<false>(a, a.h, a.F, a.d, a.w3, nullptr, a.s3, nullptr, a.b3, nullptr, a.y, s);
+  return run<false>(a, a.h, a.F, a.d, a.d, a.w3, nullptr, a.s3, nullptr, a.b3, nullptr, a.y, s);
 }
 
 }  // namespace moe

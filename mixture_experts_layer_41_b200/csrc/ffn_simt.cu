@@ -23,6 +23,7 @@ __device__ __forceinline__ int group_of(const int32_t *off, int E, int r) {
 struct SimtArgs {
   const int32_t *offsets;
   int E, rows, d, F, act;
+  int w_stride;   // rows between experts in w1 / w2
   const float *x, *w1, *w2, *w3;
   float *h, *y;
 };
@@ -38,14 +39,14 @@ __global__ void simt_phase1(SimtArgs a) {
   if (c >= a.F || r >= off[nE]) return;
   const int e = group_of(off, nE, r);
   const float *xr = a.x + (size_t)r * a.d;
-  const float *g = a.w1 + ((size_t)e * a.F + c) * a.d;
+  const float *g = a.w1 + ((size_t)e * a.w_stride + c) * a.d;
   float acc = 0.f;
   for (int k = 0; k < a.d; ++k) acc = fmaf(xr[k], g[k], acc);
   float hv;
   if (a.act == MOE_ACT_RELU) {
     hv = acc > 0.f ? acc : 0.f;
   } else {
-    const float *u = a.w2 + ((size_t)e * a.F + c) * a.d;
+    const float *u = a.w2 + ((size_t)e * a.w_stride + c) * a.d;
     float up = 0.f;
     for (int k = 0; k < a.d; ++k) up = fmaf(xr[k], u[k], up);
     hv = acc / (1.f + expf(-acc)) * up;
@@ -80,6 +81,7 @@ cudaError_t launch_ffn_simt_f32(const FfnArgs &f, cudaStream_t s) {
   a.d = f.d;
   a.F = f.F;
   a.act = f.act;
+  a.w_stride = f.w_stride;
   a.x = static_cast<const float *>(f.x);
   a.w1 = static_cast<const float *>(f.w1);
   a.w2 = static_cast<const float *>(f.w2);

@@ -61,6 +61,7 @@ struct TcParams {
   int rows;
   int rows_cap;             // rows of A and out
   int N;                    // output columns
+  int b_stride;             // B rows from one expert to the next (N, or 2N for stacked gate/up)
   int K;
   int mode;
   int n_tiles;              // output tiles per group along N
@@ -289,10 +290,10 @@ tc_grouped_gemm(const __grid_constant__ CUtensorMap mapA, const __grid_constant_
         const TileInfo ti = decode_tile(st, nE, p.n_tiles, tile);
         int b0, b1;
         if (p.mode == MODE_SWIGLU) {
-          b0 = ti.e * p.N + ti.n * 128;
+          b0 = ti.e * p.b_stride + ti.n * 128;
           b1 = b0;
         } else {
-          b0 = ti.e * p.N + ti.n * BN;
+          b0 = ti.e * p.b_stride + ti.n * BN;
           b1 = b0 + 128;
         }
         for (int kb = 0; kb < kb_n; ++kb, ++it) {
@@ -477,10 +478,13 @@ int sm_count() {
   return n > 0 ? n : 148;
 }
 
-cudaError_t run_gemm(const void *A, int rows_cap, int K, const void *B0, const void *B1, int b_rows, int N,
+// B0 / B1: expert e's rows start at e * b_stride; a map covers the rows up to
+// the end of the last expert's N.
+cudaError_t run_gemm(const void *A, int rows_cap, int K, const void *B0, const void *B1, int b_stride, int N,
                      int mode, const int32_t *offsets, int E, int rows, void *out, int *status,
                      cudaStream_t s) {
   CUtensorMap ma, mb0, mb1;
+  const int b_rows = ((offsets ? E : 1) - 1) * b_stride + N;
   cudaError_t err = make_map(&ma, A, (uint64_t)K, (uint64_t)rows_cap, BM);
   if (err == cudaSuccess) err = make_map(&mb0, B0, (uint64_t)K, (uint64_t)b_rows, 128);
   if (err == cudaSuccess) err = make_map(&mb1, B1, (uint64_t)K, (uint64_t)b_rows, 128);
@@ -491,6 +495,7 @@ cudaError_t run_gemm(const void *A, int rows_cap, int K, const void *B0, const v
   p.rows = rows;
   p.rows_cap = rows_cap;
   p.N = N;
+  p.b_stride = b_stride;
   p.K = K;
   p.mode = mode;
   p.n_tiles = mode == MODE_SWIGLU ? (N + 127) / 128 : (N + BN - 1) / BN;
@@ -509,17 +514,16 @@ cudaError_t run_gemm(const void *A, int rows_cap, int K, const void *B0, const v
 }  // namespace
 
 cudaError_t launch_ffn_tc_bf16(const FfnArgs &a, cudaStream_t s) {
-  const int nE = a.offsets ? a.E : 1;
   cudaError_t err;
   if (a.act == MOE_ACT_SWIGLU)
-    err = run_gemm(a.x, a.rows_cap, a.d, a.w1, a.w2, nE * a.F, a.F, MODE_SWIGLU, a.offsets, a.E, a.rows, a.h,
+    err = run_gemm(a.x, a.rows_cap, a.d, a.w1, a.w2, a.w_stride, a.F, MODE_SWIGLU, a.offsets, a.E, a.rows, a.h,
                    a.status, s);
   else
-    err = run_gemm(a.x, a.rows_cap, a.d, a.w1, a.w1, nE * a.F, a.F, MODE_RELU, a.offsets, a.E, a.rows, a.h,
+    err = run_gemm(a.x, a.rows_cap, a.d, a.w1, a.w1, a.w_stride, a.F, MODE_RELU, a.offsets, a.E, a.rows, a.h,
                    a.status, s);
   if (err != cudaSuccess) return err;
   if (a.mid_event && (err = cudaEventRecord(a.mid_event, s)) != cudaSuccess) return err;
-  return run_gemm(a.h, a.rows_cap, a.F, a.w3, a.w3, nE * a.d, a.d, MODE_PLAIN, a.offsets, a.E, a.rows, a.y,
+  return run_gemm(a.h, a.rows_cap, a.F, a.w3, a.w3, a.d, a.d, MODE_PLAIN, a.offsets, a.E, a.rows, a.y,
                   a.status, s);
 }
 

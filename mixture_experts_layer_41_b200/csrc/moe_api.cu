@@ -35,15 +35,20 @@ int64_t capacity_of(const moe_config &c) {
   return moe_capacity(c.num_tokens, c.top_k, c.num_experts, c.capacity_factor);
 }
 
-// Dense weights need both SwiGLU projections; ReLU uses w1 / w3 only.
+bool fused_gate_up(const moe_config &c) { return c.weight_layout == MOE_LAYOUT_FUSED_GATE_UP; }
+
+// Dense weights need both SwiGLU projections; ReLU uses w1 / w3 only.  The
+// fused gate/up layout carries both in w1 and leaves the w2 slots empty.
 moe_status check_weights(const moe_config &c, const moe_weights *w) {
   if (!w) return MOE_ERR_INVALID_ARG;
   if (!aligned16(w->w1) || !aligned16(w->w3)) return MOE_ERR_INVALID_ARG;
-  if (c.act == MOE_ACT_SWIGLU && !aligned16(w->w2)) return MOE_ERR_INVALID_ARG;
+  const bool fused = fused_gate_up(c);
+  if (fused && (w->w2 || w->scale2 || w->bias2)) return MOE_ERR_INVALID_ARG;
+  if (c.act == MOE_ACT_SWIGLU && !fused && !aligned16(w->w2)) return MOE_ERR_INVALID_ARG;
   if (c.weight_dtype == MOE_Q4_AFFINE_G64) {
-    if (!aligned16(w->scale1) || !aligned16(w->scale2) || !aligned16(w->scale3) || !aligned16(w->bias1) ||
-        !aligned16(w->bias2) || !aligned16(w->bias3))
+    if (!aligned16(w->scale1) || !aligned16(w->scale3) || !aligned16(w->bias1) || !aligned16(w->bias3))
       return MOE_ERR_INVALID_ARG;
+    if (!fused && (!aligned16(w->scale2) || !aligned16(w->bias2))) return MOE_ERR_INVALID_ARG;
   }
   if (c.shared_intermediate > 0) {
     if (!aligned16(w->shared1) || !aligned16(w->shared2) || !aligned16(w->shared3)) return MOE_ERR_INVALID_ARG;
@@ -85,12 +90,14 @@ cudaError_t run_ffn(const FfnArgs &a, cudaStream_t s) {
 }
 
 moe_status do_route(const moe_config &c, const void *x, const float *w_router, const float *bias,
-                    int32_t *ids, float *wts, float *prob_sum, void *ws, cudaStream_t s) {
+                    int32_t *ids, float *wts, float *prob_sum, void *ws, cudaStream_t s,
+                    const int32_t *forced = nullptr) {
   const WsLayout L = ws_layout(c);
   cudaError_t err = launch_route(c, x, w_router, bias, ids, wts, ws_ptr<double>(ws, L.route_part), prob_sum, s,
                                  L.route_logits != L.total && route_logits_bytes(c) ? ws_ptr<double>(ws, L.route_logits)
-                                                                                   : nullptr);
-  return err == cudaSuccess ? MOE_OK : cuda_fail(err, "moe_route");
+                                                                                   : nullptr,
+                                 forced, ws_ptr<int>(ws, L.status));
+  return err == cudaSuccess ? MOE_OK : cuda_fail(err, forced ? "moe_route_forced" : "moe_route");
 }
 
 moe_status do_permute(const moe_config &c, const void *x, const int32_t *ids, const float *wts, int32_t *off,
@@ -120,6 +127,20 @@ moe_status do_ffn(const moe_config &c, const void *x_perm, const int32_t *off, c
   a.b1 = w->bias1;
   a.b2 = w->bias2;
   a.b3 = w->bias3;
+  a.w_stride = c.intermediate;
+  if (fused_gate_up(c)) {
+    // expert e's up rows follow its F gate rows: the up view starts F rows in
+    // and both views step 2F rows per expert
+    const size_t F = (size_t)c.intermediate, d = (size_t)c.hidden;
+    a.w_stride = 2 * c.intermediate;
+    if (c.weight_dtype == MOE_Q4_AFFINE_G64) {
+      a.w2 = static_cast<const char *>(w->w1) + F * (d / 2);
+      a.s2 = static_cast<const char *>(w->scale1) + F * (d / 64) * 2;
+      a.b2 = static_cast<const char *>(w->bias1) + F * (d / 64) * 2;
+    } else {
+      a.w2 = static_cast<const char *>(w->w1) + F * d * (c.weight_dtype == MOE_F32 ? 4 : 2);
+    }
+  }
   a.y = y;
   cudaError_t err = run_ffn(a, s);
   return err == cudaSuccess ? MOE_OK : cuda_fail(err, "moe_grouped_ffn");
@@ -140,6 +161,7 @@ moe_status do_shared(const moe_config &c, const void *x, const moe_weights *w, v
   a.w1 = w->shared1;
   a.w2 = w->shared2;
   a.w3 = w->shared3;
+  a.w_stride = c.shared_intermediate;
   a.h = ws_ptr<char>(ws, L.shared_h);
   a.y = out;
   cudaError_t err = run_ffn(a, s);
@@ -171,6 +193,9 @@ moe_status moe_validate(const moe_config *cfg) {
   if (!(c.aux_alpha >= 0.0f)) return MOE_ERR_INVALID_ARG;
   if (c.num_tokens < 1 || c.hidden < 1 || c.intermediate < 1) return MOE_ERR_INVALID_ARG;
   if (c.act != MOE_ACT_RELU && c.act != MOE_ACT_SWIGLU) return MOE_ERR_INVALID_ARG;
+  if (c.weight_layout != MOE_LAYOUT_SEPARATE && c.weight_layout != MOE_LAYOUT_FUSED_GATE_UP)
+    return MOE_ERR_INVALID_ARG;
+  if (c.weight_layout == MOE_LAYOUT_FUSED_GATE_UP && c.act != MOE_ACT_SWIGLU) return MOE_ERR_INVALID_ARG;
   if (c.act_dtype != MOE_F32 && c.act_dtype != MOE_BF16) return MOE_ERR_INVALID_ARG;
   if (c.weight_dtype != MOE_F32 && c.weight_dtype != MOE_BF16 && c.weight_dtype != MOE_Q4_AFFINE_G64)
     return MOE_ERR_INVALID_ARG;
@@ -320,6 +345,32 @@ moe_status moe_route(const moe_config *cfg, const void *x, const float *w_router
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if ((st = clear_status(ws, s)) != MOE_OK) return st;
   return do_route(c, x, w_router, router_bias, topk_ids, topk_w, prob_sum, ws, s);
+}
+
+moe_status moe_route_forced(const moe_config *cfg, const void *x, const float *w_router, const float *router_bias,
+                            const int32_t *forced_ids, int32_t *topk_ids, float *topk_w, float *prob_sum, void *ws,
+                            size_t ws_bytes, moe_stream_t stream) {
+  moe_status st = moe_validate(cfg);
+  if (st != MOE_OK) return st;
+  const moe_config &c = *cfg;
+  if (!aligned16(x) || !aligned16(w_router) || !aligned16_or_null(router_bias) || !aligned16(forced_ids) ||
+      !aligned16(topk_ids) || !aligned16(topk_w) || !aligned16(prob_sum))
+    return MOE_ERR_INVALID_ARG;
+  if ((st = check_ws(c, ws, ws_bytes)) != MOE_OK) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if ((st = clear_status(ws, s)) != MOE_OK) return st;
+  return do_route(c, x, w_router, router_bias, topk_ids, topk_w, prob_sum, ws, s, forced_ids);
+}
+
+moe_status moe_update_bias(const moe_config *cfg, const int32_t *counts, float *expert_bias, float coeff,
+                           moe_stream_t stream) {
+  moe_status st = moe_validate(cfg);
+  if (st != MOE_OK) return st;
+  if (!aligned16(counts) || !aligned16(expert_bias)) return MOE_ERR_INVALID_ARG;
+  if (!(coeff >= 0.0f) || isinf(coeff)) return MOE_ERR_INVALID_ARG;
+  cudaError_t err = launch_bias_update(cfg->num_experts, counts, expert_bias, coeff,
+                                       reinterpret_cast<cudaStream_t>(stream));
+  return err == cudaSuccess ? MOE_OK : cuda_fail(err, "moe_update_bias");
 }
 
 moe_status moe_permute(const moe_config *cfg, const void *x, const int32_t *topk_ids, const float *topk_w,

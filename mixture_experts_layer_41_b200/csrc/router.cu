@@ -50,6 +50,8 @@ struct RouteParams {
   double *part;      // [ceil(T/32)][E] probability sums per 32-token group
   double *logits;    // [ks][T][E] partial logits (split path)
   int ks, kchunk;    // split path: number of hidden slices and their length
+  const int32_t *forced;   // [T][k] replayed expert ids, or null to select
+  int *status;             // device status word (bad / repeated forced ids)
 };
 
 __device__ __forceinline__ void argmax_merge(double &v, int &i, double ov, int oi) {
@@ -150,23 +152,39 @@ __device__ __forceinline__ void select_token(const RouteParams &p, int t, const 
 #pragma unroll
   for (int j = 0; j < EPL; ++j) psum[j] += prob[j];
 
-  // top-k by score, ties to the lower expert index
+  // top-k by score, ties to the lower expert index; or, when replaying, the
+  // recorded ids in their recorded order (an id outside [0, E) or one already
+  // taken gets weight 0 and flags the status word)
   uint32_t taken = 0;
   int my_e = -1;
   double my_w = 0.0;
   for (int r = 0; r < p.k; ++r) {
-    double bv = -INFINITY;
     int bi = 0x7fffffff;
+    if (p.forced) {
+      bi = p.forced[(size_t)t * p.k + r];
+    } else {
+      double bv = -INFINITY;
 #pragma unroll
-    for (int j = 0; j < EPL; ++j) {
-      const int e = lane + 32 * j;
-      if (e < E && !((taken >> j) & 1u)) argmax_merge(bv, bi, score[j], e);
+      for (int j = 0; j < EPL; ++j) {
+        const int e = lane + 32 * j;
+        if (e < E && !((taken >> j) & 1u)) argmax_merge(bv, bi, score[j], e);
+      }
+      warp_argmax(bv, bi);
     }
-    warp_argmax(bv, bi);
     double wv = 0.0;
+    bool again = false;
 #pragma unroll
     for (int j = 0; j < EPL; ++j)
-      if (lane + 32 * j == bi) { wv = prob[j]; taken |= 1u << j; }
+      if (lane + 32 * j == bi && bi < E) {
+        again = (taken >> j) & 1u;
+        wv = again ? 0.0 : prob[j];
+        taken |= 1u << j;
+      }
+    if (p.forced) {
+      again = __any_sync(0xffffffffu, again);
+      if (lane == 0 && (bi < 0 || bi >= E)) record_status(p.status, kDevBadExpertId);
+      else if (lane == 0 && again) record_status(p.status, kDevDuplicateId);
+    }
     wv = __shfl_sync(0xffffffffu, wv, bi & 31);
     if (lane == r) { my_e = bi; my_w = wv; }
   }
@@ -647,8 +665,11 @@ size_t route_logits_bytes(const moe_config &c) {
 
 cudaError_t launch_route(const moe_config &c, const void *x, const float *w_router,
                          const float *router_bias, int32_t *topk_ids, float *topk_w,
-                         double *route_part, float *prob_sum, cudaStream_t s, double *logits) {
+                         double *route_part, float *prob_sum, cudaStream_t s, double *logits,
+                         const int32_t *forced_ids, int *status) {
   RouteParams p;
+  p.forced = forced_ids;
+  p.status = status;
   p.x = x;
   p.w = w_router;
   p.bias = router_bias;

@@ -262,8 +262,34 @@ def expert_mlp(x_rows: np.ndarray, w1: np.ndarray, w3: np.ndarray, act: str,
     return h @ w3.T
 
 
+def fuse_gate_up(gate, up) -> np.ndarray:
+    """[Edge0] WeightLayout.FUSED_GATE_UP: ONE stacked tensor in which expert
+    e's block is its gate rows followed by its up rows, built expert by expert
+    ("interleaved expert by expert"), not by putting one whole stack after
+    the other.  gate, up [E, F, ...] -> [E, 2F, ...]."""
+    gate, up = np.asarray(gate), np.asarray(up)
+    assert gate.shape == up.shape
+    return np.stack([np.concatenate([gate[e], up[e]], axis=0) for e in range(gate.shape[0])])
+
+
+def split_gate_up(block: np.ndarray):
+    """One expert's fused block [2F, ...] -> (gate, up): the two halves along
+    the output axis, gate first ([Edge0] one split(x_gu, 2) gives (gate, up))."""
+    block = np.asarray(block)
+    half = block.shape[0] // 2
+    assert 2 * half == block.shape[0]
+    return block[:half], block[half:]
+
+
 def expert_weights_f64(raw: Mapping, act: str):
-    """Widen (or dequantise) one expert's stored weights to float64."""
+    """Widen (or dequantise) one expert's stored weights to float64.  A fused
+    gate/up block (key w13, or q13/s13/b13 when 4-bit) is split first."""
+    if "w13" in raw or "q13" in raw:
+        raw = dict(raw)
+        for fused, (a, b) in (("w13", ("w1", "w2")), ("q13", ("q1", "q2")), ("s13", ("s1", "s2")),
+                              ("b13", ("b1", "b2"))):
+            if fused in raw:
+                raw[a], raw[b] = split_gate_up(raw.pop(fused))
     if "q1" in raw:
         w1 = dequant_q4(raw["q1"], raw["s1"], raw["b1"])
         w2 = dequant_q4(raw["q2"], raw["s2"], raw["b2"]) if act == "swiglu" else None
@@ -348,6 +374,66 @@ def route(x, w_router, *, top_k: int, router: str = "softmax_topk", norm: bool =
         raise ValueError(router)
     return dict(ids=ids, weights=w, probs=p, margin=margin, logits=logits,
                 prob_sum=p.sum(axis=0))
+
+
+def route_forced(x, w_router, forced_ids, *, top_k: int, router: str = "softmax_topk",
+                 norm: bool = True, routed_scaling: float = 1.0, logit_bias=None) -> dict:
+    """Router replay ([dockyard] Router replay (R3)): the expert ids are the
+    recorded ones, the weights come from this router's own gate.
+
+    The scores are those of ``route`` (softmax probabilities, or raw sigmoid
+    scores); slot j of token t takes expert forced_ids[t, j] with the score
+    of that expert, then the same renormalisation (and routed scaling) as the
+    free router.  The selection bias and the group limit take no part: they
+    only choose experts.  A recorded id outside [0, E), or one repeated in its
+    row, is a bad route: the slot's weight is 0 and it is left out of the
+    normalising sum; ``bad`` [T, k] marks such slots (the caller must reject
+    them, never replay them silently).  Margins are +inf: nothing is chosen.
+    """
+    logits = router_logits(x, w_router, logit_bias)
+    ids = np.asarray(forced_ids, dtype=np.int64)
+    n_tok, n_exp = logits.shape
+    assert ids.shape == (n_tok, top_k)
+    scores = softmax(logits) if router == "softmax_topk" else sigmoid(logits)
+    weights = np.zeros((n_tok, top_k), dtype=np.float64)
+    bad = np.zeros((n_tok, top_k), dtype=bool)
+    for t in range(n_tok):
+        seen = set()
+        for j in range(top_k):
+            e = int(ids[t, j])
+            if e < 0 or e >= n_exp or e in seen:
+                bad[t, j] = True
+                continue
+            seen.add(e)
+            weights[t, j] = scores[t, e]
+    total = weights.sum(axis=-1, keepdims=True)
+    if router == "softmax_topk":
+        if norm:
+            weights = weights / np.maximum(total, 1e-12)
+    else:
+        if norm:
+            weights = weights / (total + 1e-20)
+        weights = weights * routed_scaling
+    return dict(ids=ids.astype(np.int32), weights=weights, probs=scores, bad=bad,
+                margin=np.full(n_tok, np.inf), logits=logits, prob_sum=scores.sum(axis=0))
+
+
+def update_bias(bias, counts, coeff: float) -> np.ndarray:
+    """One step of the aux-loss-free balancing bias ([dockyard] Aux-loss-free
+    load balancing): an expert that took fewer assignments than the mean
+    count goes up by ``coeff``, one that took more goes down by ``coeff``, one
+    exactly at the mean stays.  The mean is compared as an exact fraction.
+    The bias is a float32 parameter: the new value is the float64 result
+    rounded to float32 (a single rounding for the sizes used here)."""
+    from fractions import Fraction
+    counts = [int(c) for c in np.asarray(counts).ravel()]
+    mean = Fraction(sum(counts), len(counts))
+    b = np.asarray(bias, dtype=np.float32).astype(np.float64)
+    out = np.empty(len(counts), dtype=np.float32)
+    for e, c in enumerate(counts):
+        step = 1.0 if c < mean else (-1.0 if c > mean else 0.0)
+        out[e] = np.float32(b[e] + step * float(np.float32(coeff)))
+    return out
 
 
 def layer_forward(x, w_router, experts: Callable[[int], Mapping], *, top_k: int, act: str,

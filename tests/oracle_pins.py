@@ -465,4 +465,80 @@ def pin_q4_roundtrip(O):
     assert np.array_equal((W - bias.astype(np.float64)[:, g]) / scale.astype(np.float64)[:, g], q)
 
 
+# ---------------------------------------------------------------- weight layout
+
+def pin_fused_gate_up_split(O):
+    """The fused layout's projection splits into (gate, up) per expert: checked
+    by brute force with torch's linear on the separate stacks."""
+    import torch
+    rng = _rng(21)
+    E, F, d = 3, 4, 5
+    gate = rng.standard_normal((E, F, d))
+    up = rng.standard_normal((E, F, d))
+    fused = O.fuse_gate_up(gate, up)
+    assert fused.shape == (E, 2 * F, d)
+    x = rng.standard_normal((7, d))
+    for e in range(E):
+        xg = torch.nn.functional.linear(torch.from_numpy(x), torch.from_numpy(gate[e])).numpy()
+        xu = torch.nn.functional.linear(torch.from_numpy(x), torch.from_numpy(up[e])).numpy()
+        xgu = x @ fused[e].T
+        assert np.allclose(xgu[:, :F], xg, rtol=0, atol=1e-12) and np.allclose(xgu[:, F:], xu, rtol=0, atol=1e-12)
+        g2, u2 = O.split_gate_up(fused[e])
+        assert np.array_equal(g2, gate[e]) and np.array_equal(u2, up[e])
+        w3 = rng.standard_normal((d, F))
+        a = O.expert_weights_f64(dict(w13=fused[e], w3=w3), "swiglu")
+        b = O.expert_weights_f64(dict(w1=gate[e], w2=up[e], w3=w3), "swiglu")
+        assert all(np.array_equal(p, q) for p, q in zip(a, b))
+
+
+# ---------------------------------------------------------------- router replay
+
+def pin_route_forced_replays_free_route(O):
+    """Replaying the free router's own choices gives its weights back (the free
+    router is pinned by brute force above); a permuted replay permutes them."""
+    rng = _rng(22)
+    x = rng.standard_normal((30, 6))
+    wr = rng.standard_normal((8, 6))
+    bias = rng.uniform(-0.3, 0.3, 8)
+    for kw in (dict(router="softmax_topk", norm=True), dict(router="softmax_topk", norm=False),
+               dict(router="sigmoid_group", norm=True, routed_scaling=2.5, n_group=4, topk_group=2,
+                    expert_bias=bias)):
+        free = O.route(x, wr, top_k=3, **kw)
+        fkw = {k_: v for k_, v in kw.items() if k_ not in ("n_group", "topk_group", "expert_bias")}
+        rep = O.route_forced(x, wr, free["ids"], top_k=3, **fkw)
+        assert np.array_equal(rep["ids"], free["ids"]) and not rep["bad"].any()
+        assert np.allclose(rep["weights"], free["weights"], rtol=1e-13, atol=0), kw
+        assert np.allclose(rep["prob_sum"], free["prob_sum"], rtol=1e-13, atol=0)
+        perm = free["ids"][:, ::-1].copy()
+        rep2 = O.route_forced(x, wr, perm, top_k=3, **fkw)
+        assert np.allclose(rep2["weights"], free["weights"][:, ::-1], rtol=1e-13, atol=0)
+
+
+def pin_route_forced_bad_ids(O):
+    """A sentinel or repeated recorded id is flagged, weighted 0 and left out of
+    the renormalisation (closed form: the remaining weights sum to 1)."""
+    rng = _rng(23)
+    x = rng.standard_normal((3, 5))
+    wr = rng.standard_normal((6, 5))
+    ids = np.array([[0, 1, 2], [-1, 3, 4], [5, 5, 2]], dtype=np.int32)
+    rep = O.route_forced(x, wr, ids, top_k=3, router="softmax_topk", norm=True)
+    assert rep["bad"].tolist() == [[False] * 3, [True, False, False], [False, True, False]]
+    assert rep["weights"][1, 0] == 0.0 and rep["weights"][2, 1] == 0.0
+    assert np.allclose(rep["weights"].sum(axis=1), 1.0, rtol=0, atol=1e-15)
+    p = np.exp(x @ wr.T - (x @ wr.T).max(axis=1, keepdims=True))
+    p /= p.sum(axis=1, keepdims=True)
+    assert abs(rep["weights"][1, 1] - p[1, 3] / (p[1, 3] + p[1, 4])) < 1e-15
+
+
+# ---------------------------------------------------------------- balancing bias
+
+def pin_hand_bias_update(O):
+    g = _load("hand_bias_update.json")
+    for case in g["cases"]:
+        bias = _arr(case["bias"]).astype(np.float32)
+        out = O.update_bias(bias, np.array(case["counts"]), _num(case["coeff"]))
+        assert out.dtype == np.float32
+        assert np.array_equal(out.astype(np.float64), _arr(case["expected"])), (case, out)
+
+
 PINS = [v for k_, v in sorted(globals().items()) if k_.startswith("pin_")]

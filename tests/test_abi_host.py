@@ -106,6 +106,9 @@ def _cfg(**kw):
     (dict(weight_dtype="q4_affine_g64", hidden=96), L.MOE_ERR_UNSUPPORTED),
     (dict(shared_intermediate=64), L.MOE_OK),
     (dict(weight_dtype="q4_affine_g64", shared_intermediate=64), L.MOE_ERR_UNSUPPORTED),
+    (dict(weight_layout="fused_gate_up"), L.MOE_OK),
+    (dict(weight_layout="fused_gate_up", weight_dtype="q4_affine_g64"), L.MOE_OK),
+    (dict(weight_layout="fused_gate_up", act="relu"), L.MOE_ERR_INVALID_ARG),
 ])
 def test_validate(kw, status):
     cfg = _cfg(**kw)
@@ -170,3 +173,20 @@ def test_device_calls_reject_bad_arguments_before_any_launch():
     st = lib.moe_combine(C.byref(cfg_cap), fake, fake, fake, None, fake, None)
     assert st == L.MOE_ERR_CAPACITY_TOO_TIGHT
     assert "capacity" in api.moe_status_string(L.MOE_ERR_CAPACITY_TOO_TIGHT)
+    # router replay needs the recorded ids; the bias update a finite step >= 0
+    st = lib.moe_route_forced(C.byref(cfg), fake, fake, None, None, fake, fake, fake, fake, ws_need, None)
+    assert st == L.MOE_ERR_INVALID_ARG
+    st = lib.moe_route_forced(C.byref(cfg), fake, fake, None, fake, fake, fake, fake, fake, ws_need - 16, None)
+    assert st == L.MOE_ERR_WORKSPACE
+    assert lib.moe_update_bias(C.byref(cfg), fake, fake, -1e-3, None) == L.MOE_ERR_INVALID_ARG
+    assert lib.moe_update_bias(C.byref(cfg), fake, fake, float("inf"), None) == L.MOE_ERR_INVALID_ARG
+    assert lib.moe_update_bias(C.byref(cfg), None, fake, 1e-3, None) == L.MOE_ERR_INVALID_ARG
+    assert lib.moe_update_bias(C.byref(bad), fake, fake, 1e-3, None) == L.MOE_ERR_INVALID_TOPK
+    # the fused layout leaves the separate up slots empty
+    fused = _cfg(weight_layout="fused_gate_up")
+    w = L.moe_weights(w1=fake, w2=fake, w3=fake)
+    st = lib.moe_grouped_ffn(C.byref(fused), fake, fake, C.byref(w), fake, fake, ws_need, None)
+    assert st == L.MOE_ERR_INVALID_ARG
+    bad_layout = _cfg()
+    bad_layout.weight_layout = 2
+    assert api.moe_validate(bad_layout) == L.MOE_ERR_INVALID_ARG

@@ -146,6 +146,52 @@ def m_bf16_widen_wrong(O):
                          else np.asarray(a).astype(np.float64) / 65536.0)
 
 
+def m_fused_wholesale(O):
+    # both stacks one after the other, then cut into experts: rows misalign
+    O.fuse_gate_up = lambda g, u: np.concatenate([np.asarray(g), np.asarray(u)], axis=0).reshape(
+        (np.asarray(g).shape[0], 2 * np.asarray(g).shape[1]) + np.asarray(g).shape[2:])
+
+
+def m_split_up_first(O):
+    orig = O.split_gate_up
+    O.split_gate_up = lambda b: orig(b)[::-1]
+
+
+def m_forced_no_renorm(O):
+    orig = O.route_forced
+    O.route_forced = lambda *a, **kw: orig(*a, **{**kw, "norm": False})
+
+
+def m_forced_keeps_repeats(O):
+    orig = O.route_forced
+
+    def forced(x, w, ids, **kw):
+        ids = np.asarray(ids)
+        r = orig(x, w, ids, **kw)
+        # treat a repeated id as a good route: copy the first occurrence's score in
+        for t in range(ids.shape[0]):
+            for j in range(ids.shape[1]):
+                if r["bad"][t, j] and 0 <= ids[t, j] < r["probs"].shape[1]:
+                    r["bad"][t, j] = False
+                    r["weights"][t, j] = r["probs"][t, ids[t, j]]
+        return r
+    O.route_forced = forced
+
+
+def m_bias_sign_flipped(O):
+    orig = O.update_bias
+    O.update_bias = lambda b, c, coeff: orig(b, c, -coeff)
+
+
+def m_bias_integer_mean(O):
+    def upd(bias, counts, coeff):
+        counts = np.asarray(counts)
+        mean = counts.sum() // len(counts)
+        step = np.where(counts < mean, 1.0, np.where(counts > mean, -1.0, 0.0))
+        return (np.asarray(bias, dtype=np.float64) + step * coeff).astype(np.float32)
+    O.update_bias = upd
+
+
 MUTANTS = [v for k_, v in sorted(globals().items()) if k_.startswith("m_")]
 
 
