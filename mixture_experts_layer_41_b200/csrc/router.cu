@@ -483,7 +483,7 @@ route_tiled(RouteParams p) {
     __syncthreads();
   }
 
-  if (SPLIT) {
+  if constexpr (SPLIT) {
 #pragma unroll
     for (int i = 0; i < TPW; ++i) {
       const int t = t0 + warp * TPW + i;
@@ -495,19 +495,18 @@ route_tiled(RouteParams p) {
         }
       }
     }
-    return;
-  }
-
-  double psum[EPL];
+  } else {
+    double psum[EPL];
 #pragma unroll
-  for (int j = 0; j < EPL; ++j) psum[j] = 0.0;
-  double *wscr = dscr + warp * kMaxExperts;
+    for (int j = 0; j < EPL; ++j) psum[j] = 0.0;
+    double *wscr = dscr + warp * kMaxExperts;
 #pragma unroll
-  for (int i = 0; i < TPW; ++i) {
-    const int t = t0 + warp * TPW + i;
-    if (t < p.T) select_token<EPL>(p, t, acc[i], psum, wscr, lane);
+    for (int i = 0; i < TPW; ++i) {
+      const int t = t0 + warp * TPW + i;
+      if (t < p.T) select_token<EPL>(p, t, acc[i], psum, wscr, lane);
+    }
+    write_prob_partials<EPL>(p, dscr, psum, t0, TPW, lane, warp);
   }
-  write_prob_partials<EPL>(p, dscr, psum, t0, TPW, lane, warp);
 }
 
 constexpr int SEL_WARPS = 32;   // route_select: one warp per token of a 32-token group
