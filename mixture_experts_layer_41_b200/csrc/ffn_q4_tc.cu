@@ -10,12 +10,10 @@
 // "swapped": D[feature, token] = sum_k W[feature, k] x[token, k] with the
 // weights as the M = 128 operand and up to 32 tokens as N.  Per CTA
 // (persistent over (expert, 32-token pass, 128-feature tile) tiles):
-//   warp 0      TMA producer: per stage of 4 K-blocks the raw code tiles
-//               (128 rows x 128 bytes, one per matrix, so every weight row is
-//               read as a whole 128-byte line) and the 4 token tiles (32 rows
-//               x 64 bf16 each); 128-byte swizzle for both; per tile the
-//               tile's scale and bias rows (contiguous in [E, N, K/64]) by
-//               bulk copy.
+//   warp 0      TMA producer: per K-block the raw code tiles (128 rows x 32
+//               bytes, one per matrix) and the token tile (32 rows x 64 bf16,
+//               128-byte swizzle) into a stage; per tile the tile's scale and
+//               bias rows (contiguous in [E, N, K/64]) by bulk copy.
 //   warp 1      TMEM owner and single-thread tcgen05.mma issuer
 //               (kind::f16, M=128, N=32, K=16) with the weight operand read
 //               from TMEM and the token operand from shared memory; its
@@ -32,12 +30,9 @@
 //               up accumulators into h, or a plain store of y.
 // Accumulators are double-buffered, so MMA and dequantisation stream across
 // tile boundaries while the epilogue drains the previous tile.  The operand
-// slots (6 with gate+up, 12 with one matrix) fill the rest of TMEM, so the
-// dequantisers run many K-blocks ahead of the MMA.  With N = 32 an MMA costs
-// the tensor pipe's per-instruction minimum, and a commit waits for the
-// MMAs before it to finish, so slots are handed back in groups (2 or 4
-// K-blocks per commit) and the issuer takes its next operand wait before
-// committing: the pipe then idles only for the commit's drain.
+// slots (6 with gate+up, 14 with one matrix) fill the rest of TMEM, so the
+// dequantisers run many K-blocks ahead of the MMA and the per-K-block
+// commit-to-reuse round trip stays hidden.
 // Inside every 8-element chunk both operands use the K order 0,4,1,5,2,6,3,7
 // (what the nibble extraction yields without byte permutes): phase 1
 // reorders its token tile in shared memory, and writes h already in that
@@ -60,8 +55,6 @@ constexpr int DQ_WARPS = 16;
 constexpr int EPI_WARPS = 4;            // one per TMEM lane quarter
 constexpr int THREADS = 32 * (2 + DQ_WARPS + EPI_WARPS);
 constexpr int CODE_BYTES = BM * BK / 2; // 4 KiB of codes per matrix per K-block
-constexpr int KPS = 4;                  // K-blocks per stage: each weight row moves as one 128-byte segment
-constexpr int CODE_STAGE = KPS * CODE_BYTES;   // 16 KiB per matrix per stage (128 rows x 128 B, 128-byte swizzle)
 constexpr int B_BYTES = NT * BK * 2;    // 4 KiB token tile per K-block
 constexpr uint64_t TIMEOUT_NS = 2000000000ull;
 constexpr uint64_t DRAIN_NS = 200000000ull;
@@ -73,14 +66,11 @@ constexpr uint32_t IDESC = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(NT >
 template <bool PAIR>
 struct Q4Shape {
   static constexpr int MATS = PAIR ? 2 : 1;
-  static constexpr int STAGES = PAIR ? 2 : 4;
-  static constexpr int STAGE_BYTES = MATS * CODE_STAGE + KPS * B_BYTES;   // multiple of 1024
+  static constexpr int STAGES = PAIR ? 8 : 12;
+  static constexpr int STAGE_BYTES = MATS * CODE_BYTES + B_BYTES;   // multiple of 1024
   static constexpr int ACC_COLS = MATS * NT;                        // fp32 accumulators of one tile
   static constexpr int A_COLS = MATS * BK / 2;                      // one K-block of bf16 pairs per matrix
-  // operand slots released together by one commit: a commit waits for the
-  // MMAs before it to finish (a pipeline drain), so it is paid once per group
-  static constexpr int CG = PAIR ? 2 : 4;
-  static constexpr int SLOTS = (512 - 2 * ACC_COLS) / A_COLS / CG * CG;   // operand slots in TMEM
+  static constexpr int SLOTS = (512 - 2 * ACC_COLS) / A_COLS;       // operand slots in TMEM
   static constexpr int WARPS_PER_KB = 4 * MATS;                     // one warp per (matrix, lane quarter)
   static constexpr int GROUPS = DQ_WARPS / WARPS_PER_KB;            // K-blocks in flight in dequant
 };
@@ -300,7 +290,7 @@ q4_tc_gemm(const __grid_constant__ CUtensorMap mapC0, const __grid_constant__ CU
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   const uint32_t pad = (1024u - (smem_u32(smem_raw) & 1023u)) & 1023u;
   uint8_t *base = smem_raw + pad;
-  uint8_t *stages = base;                                            // STAGES x [codes(MATS) | KPS token tiles]
+  uint8_t *stages = base;                                            // STAGES x [codes(MATS) | tokens]
   uint8_t *bslots = stages + (size_t)STAGES * S::STAGE_BYTES;       // SLOTS x token tile (operand K order)
   uint16_t *sbuf = reinterpret_cast<uint16_t *>(bslots + (size_t)SLOTS * B_BYTES);   // 2 x MATS x {scale, bias}
   const int sc_elems = BM * p.kgroups;                               // per matrix per kind
@@ -309,15 +299,16 @@ q4_tc_gemm(const __grid_constant__ CUtensorMap mapC0, const __grid_constant__ CU
   const int nE = p.E;
   const int m_tiles = p.N / BM;
   const int kb_n = p.kgroups;
-  const int n_st = (kb_n + KPS - 1) / KPS;                          // stages per tile
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(&st->full[s], 1);
-      mbar_init(&st->empty[s], DQ_WARPS);    // every dequantising warp, once per use of the stage
+      mbar_init(&st->empty[s], WPK);         // the warps that dequantise that K-block
     }
-    for (int j = 0; j < SLOTS; ++j) mbar_init(&st->a_full[j], WPK);
-    for (int g = 0; g < SLOTS / S::CG; ++g) mbar_init(&st->a_empty[g], 1);
+    for (int j = 0; j < SLOTS; ++j) {
+      mbar_init(&st->a_full[j], WPK);
+      mbar_init(&st->a_empty[j], 1);
+    }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&st->sc_full[b], 1);
       mbar_init(&st->sc_empty[b], DQ_WARPS);
@@ -387,7 +378,7 @@ q4_tc_gemm(const __grid_constant__ CUtensorMap mapC0, const __grid_constant__ CU
                     smem_u32(&st->sc_full[sb]));
         }
         sc_issued = tc + 1;
-        for (int ks = 0; ks < n_st; ++ks, ++it) {
+        for (int kb = 0; kb < kb_n; ++kb, ++it) {
           const int s = it % STAGES;
           const uint32_t ph = (it / STAGES) & 1u;
           if (!wait_bounded(&st->empty[s], ph ^ 1u, abort_flag, p.status, kDevTimeoutProducer)) {
@@ -396,14 +387,10 @@ q4_tc_gemm(const __grid_constant__ CUtensorMap mapC0, const __grid_constant__ CU
           }
           uint8_t *sp = stages + (size_t)s * S::STAGE_BYTES;
           const uint32_t fb = smem_u32(&st->full[s]);
-          // a stage past the end of K holds fewer K-blocks: only theirs are
-          // loaded (the code segment's tail is zero-filled by the copy)
-          const int nkb = min(KPS, kb_n - ks * KPS);
-          mbar_expect_tx(&st->full[s], (uint32_t)(MATS * CODE_STAGE + nkb * B_BYTES));
-          tma_load_2d(smem_u32(sp), &mapC0, fb, ks * (KPS * BK / 2), wrow);
-          if (PAIR) tma_load_2d(smem_u32(sp + CODE_STAGE), &mapC1, fb, ks * (KPS * BK / 2), wrow);
-          for (int i = 0; i < nkb; ++i)
-            tma_load_2d(smem_u32(sp + MATS * CODE_STAGE + i * B_BYTES), &mapB, fb, (ks * KPS + i) * BK, ti.row0);
+          mbar_expect_tx(&st->full[s], S::STAGE_BYTES);
+          tma_load_2d(smem_u32(sp), &mapC0, fb, kb * (BK / 2), wrow);
+          if (PAIR) tma_load_2d(smem_u32(sp + CODE_BYTES), &mapC1, fb, kb * (BK / 2), wrow);
+          tma_load_2d(smem_u32(sp + MATS * CODE_BYTES), &mapB, fb, kb * BK, ti.row0);
         }
       }
       if (!ok) {
@@ -421,7 +408,7 @@ q4_tc_gemm(const __grid_constant__ CUtensorMap mapC0, const __grid_constant__ CU
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       uint32_t it = 0, tcount = 0;
-      bool ok = true, ready = false;   // ready: a_full of K-block `it` already waited for
+      bool ok = true;
       for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x, ++tcount) {
         // accumulator buffer tcount % 2: the epilogue of two tiles ago must be done with it
         const uint32_t abuf = tcount & 1u;
@@ -432,12 +419,11 @@ q4_tc_gemm(const __grid_constant__ CUtensorMap mapC0, const __grid_constant__ CU
         tc_fence_after();
         const uint32_t dcol = tmem_base + abuf * S::ACC_COLS;
         for (int kb = 0; kb < kb_n; ++kb, ++it) {
-          const uint32_t j = it % SLOTS;
-          if (!ready && !wait_bounded(&st->a_full[j], (it / SLOTS) & 1u, abort_flag, p.status, kDevTimeoutMma)) {
+          const uint32_t j = it % SLOTS, use = it / SLOTS;
+          if (!wait_bounded(&st->a_full[j], use & 1u, abort_flag, p.status, kDevTimeoutMma)) {
             ok = false;
             break;
           }
-          ready = false;
           tc_fence_after();
           const uint64_t db = sw128_desc(smem_u32(bslots + (size_t)j * B_BYTES));
           const uint32_t acol = tmem_base + 2 * S::ACC_COLS + j * S::A_COLS;
@@ -448,19 +434,7 @@ q4_tc_gemm(const __grid_constant__ CUtensorMap mapC0, const __grid_constant__ CU
               tc_mma_ts(dcol + m * NT, acol + m * (BK / 2) + kk * 8, db + (uint64_t)(kk * 2),
                         (kb | kk) != 0 ? 1u : 0u);
           }
-          if (it % S::CG == S::CG - 1) {
-            // take the next K-block's wait while these MMAs run, so the
-            // commit's drain is the only gap in the tensor pipe
-            if (kb + 1 < kb_n) {
-              const uint32_t n = it + 1;
-              if (!wait_bounded(&st->a_full[n % SLOTS], (n / SLOTS) & 1u, abort_flag, p.status, kDevTimeoutMma)) {
-                ok = false;
-                break;
-              }
-              ready = true;
-            }
-            tc_commit(&st->a_empty[j / S::CG]);
-          }
+          tc_commit(&st->a_empty[j]);
         }
         if (!ok) break;
         tc_commit(&st->acc_full[abuf]);
@@ -481,10 +455,8 @@ q4_tc_gemm(const __grid_constant__ CUtensorMap mapC0, const __grid_constant__ CU
     const int q = warp & 3;                             // TMEM lane quarter this warp may access
     const int row = q * 32 + lane;
     constexpr int BCH = (B_BYTES / 16) / (32 * WPK);    // token-tile chunks per thread
-    constexpr int PER = KPS / GROUPS;                   // K-blocks per stage for one group
-    static_assert(KPS % GROUPS == 0, "every group takes the same number of K-blocks of a stage");
     const uint32_t stages_sa = smem_u32(stages), bslots_sa = smem_u32(bslots);
-    uint32_t tc = 0, sit = 0;                           // tiles done, stage uses done
+    uint32_t tc = 0;
     bool ok = true;
     for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x, ++tc) {
       const Tile ti = decode_tile(st, nE, m_tiles, tile);
@@ -495,70 +467,54 @@ q4_tc_gemm(const __grid_constant__ CUtensorMap mapC0, const __grid_constant__ CU
       }
       const uint32_t scl = smem_u32(sbuf + ((size_t)sb * MATS + mat) * 2 * sc_elems + (size_t)row * p.kgroups);
       const uint32_t bis = scl + 2u * (uint32_t)sc_elems;
-      const uint32_t it0 = tc * (uint32_t)kb_n;            // global index of the tile's first K-block
-      for (int ks = 0; ks < n_st && ok; ++ks, ++sit) {
-        const int s = (int)(sit % STAGES);
-        if (!wait_bounded(&st->full[s], (sit / STAGES) & 1u, abort_flag, p.status, kDevTimeoutEpilogue)) {
+      const uint32_t it0 = tc * (uint32_t)kb_n;
+      const int kb_first = (int)((grp - (int)(it0 % GROUPS) + GROUPS) % GROUPS);
+      for (int kb = kb_first; kb < kb_n; kb += GROUPS) {
+        const uint32_t it = it0 + kb;                    // it % GROUPS == grp
+        const int s = (int)(it % STAGES);
+        const uint32_t ph = (it / STAGES) & 1u;
+        const uint32_t j = it % SLOTS, use = it / SLOTS;
+        if (!wait_bounded(&st->full[s], ph, abort_flag, p.status, kDevTimeoutEpilogue)) {
           ok = false;
           break;
         }
-        // this group's K-blocks of the stage (kk = grp, grp + GROUPS, ...) into
-        // registers; a code row is one 128-byte line whose 16-byte chunks are
-        // swizzled by (row & 7), so K-block kk sits in chunks 2kk, 2kk+1 ^ (row & 7)
         const uint32_t stage_sa = stages_sa + (uint32_t)(s * S::STAGE_BYTES);
-        const uint32_t rb = stage_sa + (uint32_t)(mat * CODE_STAGE + row * 128);
-        uint32_t wv[PER][8];
-        uint4 bch[PER][BCH];
+        const uint32_t cp = stage_sa + (uint32_t)(mat * CODE_BYTES + row * (BK / 2));
+        const uint4 c0 = lds128(cp), c1 = lds128(cp + 16);
+        const uint32_t wv[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+        // token tile chunks (phase 1 reorders them into the operand K order;
+        // phase 2's token tile, h, already is in it)
+        uint4 bch[BCH];
 #pragma unroll
-        for (int u = 0; u < PER; ++u) {
-          const int kk = grp + u * GROUPS;
-          if (ks * KPS + kk < kb_n) {
-            const uint4 c0 = lds128(rb + ((uint32_t)((2 * kk) ^ (row & 7)) << 4));
-            const uint4 c1 = lds128(rb + ((uint32_t)((2 * kk + 1) ^ (row & 7)) << 4));
-            wv[u][0] = c0.x; wv[u][1] = c0.y; wv[u][2] = c0.z; wv[u][3] = c0.w;
-            wv[u][4] = c1.x; wv[u][5] = c1.y; wv[u][6] = c1.z; wv[u][7] = c1.w;
-            // token tile chunks (phase 1 reorders them into the operand K
-            // order; phase 2's token tile, h, already is in it)
-#pragma unroll
-            for (int i = 0; i < BCH; ++i) {
-              bch[u][i] = lds128(stage_sa + (uint32_t)(MATS * CODE_STAGE + kk * B_BYTES) +
-                                 (uint32_t)(gt + i * 32 * WPK) * 16u);
-              if (PAIR) bch[u][i] = permute_chunk(bch[u][i]);
-            }
-          }
+        for (int i = 0; i < BCH; ++i) {
+          bch[i] = lds128(stage_sa + (uint32_t)(MATS * CODE_BYTES) + (uint32_t)(gt + i * 32 * WPK) * 16u);
+          if (PAIR) bch[i] = permute_chunk(bch[i]);
         }
-        // the stage's bytes this warp needs are in registers: hand it back
+        // the stage's bytes are all in registers: hand it back to the producer
         __syncwarp();
         if (lane == 0) mbar_arrive(&st->empty[s]);
+        const uint32_t s1 = lds16(scl + 2u * kb), b1 = lds16(bis + 2u * kb);
+        const uint32_t s2 = s1 | (s1 << 16), b2 = b1 | (b1 << 16);
+        uint32_t av[32];
 #pragma unroll
-        for (int u = 0; u < PER; ++u) {
-          const int kb = ks * KPS + grp + u * GROUPS;
-          if (kb >= kb_n || !ok) continue;
-          const uint32_t it = it0 + kb;
-          const uint32_t j = it % SLOTS, use = it / SLOTS;
-          const uint32_t s1 = lds16(scl + 2u * kb), b1 = lds16(bis + 2u * kb);
-          const uint32_t s2 = s1 | (s1 << 16), b2 = b1 | (b1 << 16);
-          uint32_t av[32];
-#pragma unroll
-          for (int w = 0; w < 8; ++w) {
-            const uint4 d = dequant8(wv[u][w], s2, b2);
-            av[4 * w] = d.x; av[4 * w + 1] = d.y; av[4 * w + 2] = d.z; av[4 * w + 3] = d.w;
-          }
-          if (!wait_bounded(&st->a_empty[j / S::CG], (use & 1u) ^ 1u, abort_flag, p.status, kDevTimeoutEpilogue)) {
-            ok = false;
-            continue;
-          }
-          tc_fence_after();
-          tmem_st32(tmem_base + ((uint32_t)(q * 32) << 16) + 2 * S::ACC_COLS + j * S::A_COLS + mat * (BK / 2), av);
-#pragma unroll
-          for (int i = 0; i < BCH; ++i)
-            sts128(bslots_sa + j * (uint32_t)B_BYTES + (uint32_t)(gt + i * 32 * WPK) * 16u, bch[u][i]);
-          tmem_wait_st();
-          asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&st->a_full[j]);
+        for (int w = 0; w < 8; ++w) {
+          const uint4 d = dequant8(wv[w], s2, b2);
+          av[4 * w] = d.x; av[4 * w + 1] = d.y; av[4 * w + 2] = d.z; av[4 * w + 3] = d.w;
         }
+        if (!wait_bounded(&st->a_empty[j], (use & 1u) ^ 1u, abort_flag, p.status, kDevTimeoutEpilogue)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        tmem_st32(tmem_base + ((uint32_t)(q * 32) << 16) + 2 * S::ACC_COLS + j * S::A_COLS + mat * (BK / 2), av);
+#pragma unroll
+        for (int i = 0; i < BCH; ++i)
+          sts128(bslots_sa + j * (uint32_t)B_BYTES + (uint32_t)(gt + i * 32 * WPK) * 16u, bch[i]);
+        tmem_wait_st();
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&st->a_full[j]);
       }
       if (!ok) break;
       // scale rows of this tile no longer needed
@@ -641,18 +597,16 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-// Codes as bytes: [rows, K/2] uint8, box 128 bytes (KPS K-blocks) x 128 rows,
-// 128-byte swizzle (the dequantisers read one row per lane without bank
-// conflicts).  Whole 128-byte row segments keep the HBM reads in full lines.
+// Codes as bytes: [rows, K/2] uint8, box 32 bytes x 128 rows, no swizzle.
 cudaError_t map_codes(CUtensorMap *m, const void *ptr, uint64_t kbytes, uint64_t rows) {
   auto fn = encode_fn();
   if (!fn) return cudaErrorNotSupported;
   cuuint64_t dims[2] = {kbytes, rows};
   cuuint64_t strides[1] = {kbytes};
-  cuuint32_t box[2] = {(cuuint32_t)(KPS * BK / 2), (cuuint32_t)BM};
+  cuuint32_t box[2] = {(cuuint32_t)(BK / 2), (cuuint32_t)BM};
   cuuint32_t es[2] = {1, 1};
   CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(ptr), dims, strides, box, es,
-                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
