@@ -157,7 +157,9 @@ def layer_costs(w, R: int, touched: int) -> dict:
 
 def kernels_per_step(w) -> int:
     """Kernels of this library launched by one moe_forward."""
-    if w.E <= 16:
+    if w.dtype == "bf16" and w.T >= 512 and (w.router == "sigmoid_group" or w.norm_topk_prob):
+        route = 4                                   # weight split, tensor-core logits, selection, finalize
+    elif w.E <= 16:
         route = 2                                   # route_rows + route_finalize
     else:
         nb32 = (w.T + 31) // 32

@@ -139,10 +139,21 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 // selection pass -- for batches too small to fill the GPU with whole rows.
 struct RoutePlan {
   bool split;
+  bool tc;          // bf16 tokens: logits on the tensor cores (router_tc.cu), then the selection pass
   int ks, kchunk;
   int tpw;          // tokens per warp of the tiled kernel (4 or 8)
 };
 RoutePlan route_plan(const moe_config &c, bool allow_split);
+
+// Tensor-core logits: expert tile width, padded expert count, hidden slices.
+struct TcRoutePlan {
+  int nte, e_pad, ks, kb_per_slice;
+  size_t wsplit_bytes;   // the three bf16 slices of the router weight, [3][e_pad][d]
+};
+TcRoutePlan tc_route_plan(const moe_config &c);
+// Splits w_router into wsplit and writes float64 logits partials [ks][T][E].
+cudaError_t launch_route_tc_logits(const moe_config &c, const void *x, const float *w_router,
+                                   __nv_bfloat16 *wsplit, double *logits, int *status, cudaStream_t s);
 
 // logits == nullptr forbids the split pass (no workspace for it).
 cudaError_t launch_route(const moe_config &c, const void *x, const float *w_router,

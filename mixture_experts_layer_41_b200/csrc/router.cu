@@ -52,6 +52,7 @@ struct RouteParams {
   int ks, kchunk;    // split path: number of hidden slices and their length
   const int32_t *forced;   // [T][k] replayed expert ids, or null to select
   int *status;             // device status word (bad / repeated forced ids)
+  int refine;              // logits are selection-grade only: weight from exact chosen logits
 };
 
 __device__ __forceinline__ void argmax_merge(double &v, int &i, double ov, int oi) {
@@ -79,9 +80,32 @@ __device__ __forceinline__ double warp_max(double v) {
   return v;
 }
 
+// Exact logit of bf16 token t and expert e: every product is exact in
+// float64 (8-bit by 24-bit significands), summed per lane in index order and
+// then across the warp.  d % 8 == 0 (bf16 rows are 16-byte vectors).
+__device__ __forceinline__ double exact_logit(const RouteParams &p, int t, int e, int lane) {
+  const uint4 *xr = reinterpret_cast<const uint4 *>(static_cast<const __nv_bfloat16 *>(p.x) + (size_t)t * p.d);
+  const float4 *wr = reinterpret_cast<const float4 *>(p.w + (size_t)e * p.d);
+  double s = 0.0;
+  for (int i = lane; i < p.d / 8; i += 32) {
+    const uint4 xv = __ldg(xr + i);
+    const float4 w0 = __ldg(wr + 2 * i), w1 = __ldg(wr + 2 * i + 1);
+    const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
+    const float wf[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      s = fma((double)__uint_as_float(xw[u] << 16), (double)wf[2 * u], s);
+      s = fma((double)__uint_as_float(xw[u] & 0xFFFF0000u), (double)wf[2 * u + 1], s);
+    }
+  }
+  return warp_sum(s);
+}
+
 // Scores, selection and weights of token t, whose logits (without bias) sit
 // in l[j] for expert lane + 32 j.  Adds the token's probabilities to psum.
-// wscr: this warp's shared scratch row of kMaxExperts doubles.
+// wscr: this warp's shared scratch row of kMaxExperts doubles.  With
+// p.refine the logits only choose the experts (and give the probability
+// sums); the chosen experts' logits are recomputed exactly for the weights.
 template <int EPL>
 __device__ __forceinline__ void select_token(const RouteParams &p, int t, const double (&lg)[EPL],
                                              double (&psum)[EPL], double *wscr, int lane) {
@@ -157,7 +181,8 @@ __device__ __forceinline__ void select_token(const RouteParams &p, int t, const 
   // taken gets weight 0 and flags the status word)
   uint32_t taken = 0;
   int my_e = -1;
-  double my_w = 0.0;
+  double my_w = 0.0, my_key = 0.0;
+  bool my_ok = false;
   for (int r = 0; r < p.k; ++r) {
     int bi = 0x7fffffff;
     if (p.forced) {
@@ -186,15 +211,48 @@ __device__ __forceinline__ void select_token(const RouteParams &p, int t, const 
       else if (lane == 0 && again) record_status(p.status, kDevDuplicateId);
     }
     wv = __shfl_sync(0xffffffffu, wv, bi & 31);
-    if (lane == r) { my_e = bi; my_w = wv; }
+    double key = 0.0;
+    if (p.refine && bi >= 0 && bi < E && !again) {
+      // softmax keeps the exact logit (with the logit bias) for the
+      // renormalisation below; sigmoid scores it at once (its bias only
+      // selects).  key: the exact selection score, for the slot order
+      const double l = exact_logit(p, t, bi, lane);
+      const double b = p.bias ? (double)p.bias[bi] : 0.0;
+      if (p.router == MOE_ROUTER_SOFTMAX_TOPK) {
+        wv = l + b;
+        key = wv;
+      } else {
+        wv = 1.0 / (1.0 + exp(-l));
+        key = wv + b;
+      }
+    }
+    if (lane == r) { my_e = bi; my_w = wv; my_key = key; my_ok = bi >= 0 && bi < E && !again; }
+  }
+  if (p.refine && p.router == MOE_ROUTER_SOFTMAX_TOPK) {
+    // renormalised softmax over the chosen experts from their exact logits:
+    // p_j / sum_sel p = exp(l_j - m) / sum_sel exp(l_i - m)
+    const double m = warp_max(lane < p.k && my_ok ? my_w : -INFINITY);
+    my_w = lane < p.k && my_ok ? exp(my_w - m) : 0.0;
   }
   const double tot = warp_sum(lane < p.k ? my_w : 0.0);
   double wout;
   if (p.router == MOE_ROUTER_SOFTMAX_TOPK) wout = p.norm ? my_w / fmax(tot, 1e-12) : my_w;
   else wout = (p.norm ? my_w / (tot + 1e-20) : my_w) * p.scaling;
+  // slot order: the approximate logits chose the set; with refinement the
+  // chosen experts are ranked again by their exact scores (descending, ties
+  // to the lower index), as a selection on exact logits would order them
+  int slot = lane;
+  if (p.refine && !p.forced) {
+    slot = 0;
+    for (int j = 0; j < p.k; ++j) {
+      const double kj = __shfl_sync(0xffffffffu, my_key, j);
+      const int ej = __shfl_sync(0xffffffffu, my_e, j);
+      if (kj > my_key || (kj == my_key && ej < my_e)) ++slot;
+    }
+  }
   if (lane < p.k) {
-    p.ids[(size_t)t * p.k + lane] = my_e;
-    p.wts[(size_t)t * p.k + lane] = (float)wout;
+    p.ids[(size_t)t * p.k + slot] = my_e;
+    p.wts[(size_t)t * p.k + slot] = (float)wout;
   }
 }
 
@@ -560,22 +618,28 @@ route_select(RouteParams p) {
   write_prob_partials<EPL, SEL_WARPS>(p, dscr, psum, tb, 1, lane, warp);
 }
 
-// prob_sum[e] = sum over 32-token groups, as eight interleaved running sums
-// (group b feeds sum b % 8, in increasing b) added pairwise at the end: a
-// fixed order, with eight loads in flight per step.
-__global__ void route_finalize(const double *part, int nb, int E, float *prob_sum) {
-  const int e = blockIdx.x * blockDim.x + threadIdx.x;
-  if (e >= E) return;
-  double s[8];
-#pragma unroll
-  for (int u = 0; u < 8; ++u) s[u] = 0.0;
-  int b = 0;
-  for (; b + 8 <= nb; b += 8) {
-#pragma unroll
-    for (int u = 0; u < 8; ++u) s[u] += part[(size_t)(b + u) * E + e];
+// prob_sum[e] = sum over 32-token groups in a fixed order: a block per 32
+// experts; warp w adds groups w, w + 8, w + 16, ... (four running sums per
+// lane, loads in flight together), then the eight warp sums are added in warp
+// order.  Deterministic for a given T and E.
+constexpr int FIN_WARPS = 8;
+__global__ void __launch_bounds__(32 * FIN_WARPS) route_finalize(const double *part, int nb, int E, float *prob_sum) {
+  __shared__ double ws[FIN_WARPS][32];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int e = blockIdx.x * 32 + lane;
+  double s[4] = {0.0, 0.0, 0.0, 0.0};
+  if (e < E) {
+    int b = warp, u = 0;
+    for (; b < nb; b += FIN_WARPS, u = (u + 1) & 3) s[u] += part[(size_t)b * E + e];
   }
-  for (int u = 0; b + u < nb; ++u) s[u] += part[(size_t)(b + u) * E + e];
-  prob_sum[e] = (float)(((s[0] + s[1]) + (s[2] + s[3])) + ((s[4] + s[5]) + (s[6] + s[7])));
+  ws[warp][lane] = (s[0] + s[1]) + (s[2] + s[3]);
+  __syncthreads();
+  if (warp == 0 && e < E) {
+    double t = 0.0;
+#pragma unroll
+    for (int w = 0; w < FIN_WARPS; ++w) t += ws[w][lane];
+    prob_sum[e] = (float)t;
+  }
 }
 
 template <int EPL, int TPW, bool BF16, bool SPLIT>
@@ -608,6 +672,24 @@ cudaError_t launch_wide(const RouteParams &p, const RoutePlan &plan, cudaStream_
   return launch_tiled<EPL, 4, BF16, false>(p, dim3((p.T + 31) / 32), s);
 }
 
+// The selection pass over float64 logits partials [ks][T][E].
+template <int EPL>
+cudaError_t launch_select_epl(const RouteParams &p, cudaStream_t s) {
+  const size_t smem = sizeof(double) * ((size_t)kRouteTokens * p.E + (size_t)SEL_WARPS * kMaxExperts);
+  auto sel = route_select<EPL>;
+  cudaError_t err = cudaFuncSetAttribute(sel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (err != cudaSuccess) return err;
+  sel<<<(p.T + kRouteTokens - 1) / kRouteTokens, 32 * SEL_WARPS, smem, s>>>(p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_select(const RouteParams &p, cudaStream_t s) {
+  if (p.E <= 32) return launch_select_epl<1>(p, s);
+  if (p.E <= 64) return launch_select_epl<2>(p, s);
+  if (p.E <= 128) return launch_select_epl<4>(p, s);
+  return launch_select_epl<8>(p, s);
+}
+
 template <bool BF16>
 cudaError_t launch_any(const RouteParams &p, const RoutePlan &plan, cudaStream_t s) {
   const int nb32 = (p.T + kRouteTokens - 1) / kRouteTokens;
@@ -629,9 +711,20 @@ cudaError_t launch_any(const RouteParams &p, const RoutePlan &plan, cudaStream_t
 RoutePlan route_plan(const moe_config &c, bool allow_split) {
   RoutePlan plan{};
   plan.split = false;
+  plan.tc = false;
   plan.ks = 1;
   plan.kchunk = c.hidden;
   plan.tpw = 4;
+  // the weights then depend on the chosen experts' logits alone (renormalised
+  // softmax, or sigmoid scores), which the selection pass recomputes exactly
+  const bool chosen_only = c.router == MOE_ROUTER_SIGMOID_GROUP || c.norm_topk_prob;
+  // (a decode-sized batch is served faster by the split CUDA-core pass)
+  if (allow_split && c.act_dtype == MOE_BF16 && chosen_only && c.num_tokens >= 512) {
+    const TcRoutePlan t = tc_route_plan(c);
+    plan.tc = true;
+    plan.ks = t.ks;
+    return plan;
+  }
   if (c.num_experts <= 16) return plan;
   const int sms = 148;
   const int whole_row_blocks = (c.num_tokens + kRouteTokens - 1) / kRouteTokens;
@@ -657,8 +750,14 @@ RoutePlan route_plan(const moe_config &c, bool allow_split) {
   return plan;
 }
 
+// logits partials, then (tensor-core plan) the split router weight
+static size_t tc_logits_part(const moe_config &c, int ks) {
+  return align_up(sizeof(double) * (size_t)ks * c.num_tokens * c.num_experts, 256);
+}
+
 size_t route_logits_bytes(const moe_config &c) {
   const RoutePlan plan = route_plan(c, true);
+  if (plan.tc) return tc_logits_part(c, plan.ks) + tc_route_plan(c).wsplit_bytes;
   return plan.split ? sizeof(double) * (size_t)plan.ks * c.num_tokens * c.num_experts : 0;
 }
 
@@ -685,13 +784,22 @@ cudaError_t launch_route(const moe_config &c, const void *x, const float *w_rout
   p.wts = topk_w;
   p.part = route_part;
   const RoutePlan plan = route_plan(c, logits != nullptr);
+  p.refine = plan.tc ? 1 : 0;
   p.logits = logits;
   p.ks = plan.ks;
   p.kchunk = plan.kchunk;
-  cudaError_t err = c.act_dtype == MOE_BF16 ? launch_any<true>(p, plan, s) : launch_any<false>(p, plan, s);
+  cudaError_t err;
+  if (plan.tc) {
+    __nv_bfloat16 *wsplit =
+        reinterpret_cast<__nv_bfloat16 *>(reinterpret_cast<char *>(logits) + tc_logits_part(c, plan.ks));
+    err = launch_route_tc_logits(c, x, w_router, wsplit, logits, status, s);
+    if (err == cudaSuccess) err = launch_select(p, s);
+  } else {
+    err = c.act_dtype == MOE_BF16 ? launch_any<true>(p, plan, s) : launch_any<false>(p, plan, s);
+  }
   if (err != cudaSuccess) return err;
   const int nb = route_blocks(c);
-  route_finalize<<<(c.num_experts + 127) / 128, 128, 0, s>>>(route_part, nb, c.num_experts, prob_sum);
+  route_finalize<<<(c.num_experts + 31) / 32, 32 * FIN_WARPS, 0, s>>>(route_part, nb, c.num_experts, prob_sum);
   return cudaGetLastError();
 }
 
