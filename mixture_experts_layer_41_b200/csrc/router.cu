@@ -6,11 +6,16 @@
 // sigmoid scores, selection = score + bias, groups ranked by the sum of their
 // two best selection scores, routed scaling).
 //
-// Logits are fp32 products summed over runs of 8 consecutive elements, the
-// runs added in float64 (keeps the logit error near 1e-7 at d = 7168, where a
-// straight fp32 sum reaches ~1e-6); scores, selection and weights are float64
-// and rounded to float32 on the store.  Three shapes:
-//   route_rows    E <= 16: one warp per 2 tokens, lanes split the hidden
+// Two ways to the logits.  bf16 batches of 512 tokens or more whose weights
+// depend on the chosen experts alone (renormalised softmax, sigmoid) take
+// the tensor-core GEMMs of router_tc.cu (float64 partials per hidden slice);
+// route_select then chooses from those logits and recomputes the k chosen
+// logits exactly (exact_logit) for the weights and the slot order.  All other
+// cases stay on the CUDA cores: fp32 products summed over runs of 8 elements,
+// the runs added in float64 (a straight fp32 sum over d = 7168 misses the
+// 1e-6 weight bound); scores, selection and weights are float64 and rounded
+// to float32 on the store.  CUDA-core shapes:
+//   route_rows    E <= 16: one warp per 2-4 tokens, lanes split the hidden
 //                 dimension with 16-byte loads, W_r read through L1; the
 //                 E logits of a token are warp all-reduced, lane e owns e.
 //   route_tiled   E > 16: a block owns 8*TPW tokens x all E experts; x and W_r
@@ -18,11 +23,11 @@
 //                 with cp.async, double-buffered one chunk ahead; lane l owns
 //                 experts l, l+32, ...  With SPLIT the block covers one slice
 //                 of the hidden dimension and writes float64 partial logits.
-//   route_select  E > 16 after a SPLIT pass (8-token x 32-expert x hidden-
-//                 slice blocks, used when T is too small to fill the GPU with
-//                 whole-row blocks, e.g. decode): sums the partial logits of
-//                 32 tokens in slice order into shared memory, then selects
-//                 with one warp per token.
+//   route_select  after a SPLIT pass (8-token x 32-expert x hidden-slice
+//                 blocks, used when T is too small to fill the GPU with
+//                 whole-row blocks, e.g. decode) or the tensor-core pass: sums
+//                 the partial logits of 32 tokens in slice order into shared
+//                 memory, then selects with one warp per token.
 // Every selecting block covers 32-token groups and writes one float64
 // probability sum per (group, expert); route_finalize adds the groups in
 // order, so prob_sum is deterministic.
