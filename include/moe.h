@@ -98,6 +98,12 @@ typedef struct moe_config {
   int32_t shared_intermediate;  /* 0: no shared expert; else the shared SwiGLU expert's width */
   float aux_alpha;              /* balancing-loss coefficient >= 0 (blog default 0.01) */
   int32_t weight_layout;        /* moe_weight_layout; FUSED_GATE_UP needs SwiGLU */
+  int32_t fused_gather;         /* 1: with bf16 experts, moe_forward gathers each expert's token rows
+                                   inside the grouped GEMM (TMA gather of x rows) instead of copying them
+                                   into an expert-sorted buffer; no such buffer is then part of the
+                                   workspace.  Same results; on B200 the copy is faster for the bench
+                                   shapes (the GEMM re-fetches its token tile for every output tile).
+                                   0 (default): copy.  No effect with other weight types. */
 } moe_config;
 
 /*

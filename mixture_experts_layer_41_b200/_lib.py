@@ -57,6 +57,7 @@ class moe_config(C.Structure):
         ("shared_intermediate", C.c_int32),
         ("aux_alpha", C.c_float),
         ("weight_layout", C.c_int32),
+        ("fused_gather", C.c_int32),
     ]
 
 

@@ -28,11 +28,11 @@ def make_config(*, num_tokens: int, hidden: int, intermediate: int, num_experts:
                 n_group: int = 1, topk_group: int = 1, capacity_factor: float = 0.0,
                 act: str = "swiglu", act_dtype: str = "bf16", weight_dtype: str = "bf16",
                 shared_intermediate: int = 0, aux_alpha: float = 0.01,
-                weight_layout: str = "separate") -> moe_config:
+                weight_layout: str = "separate", fused_gather: bool = False) -> moe_config:
     return moe_config(num_tokens, hidden, intermediate, num_experts, top_k, _ROUTERS[router],
                       1 if norm_topk_prob else 0, routed_scaling, n_group, topk_group,
                       capacity_factor, _ACTS[act], _DTYPES[act_dtype], _DTYPES[weight_dtype],
-                      shared_intermediate, aux_alpha, _LAYOUTS[weight_layout])
+                      shared_intermediate, aux_alpha, _LAYOUTS[weight_layout], 1 if fused_gather else 0)
 
 
 def _p(t: Optional[torch.Tensor]):

@@ -107,7 +107,8 @@ inline WsLayout ws_layout(const moe_config &c) {
   L.kept_counts = take(sizeof(int32_t) * E);
   L.prob_sum = take(sizeof(float) * E);
   L.dropped = take(sizeof(int32_t));
-  L.x_perm = take(es * slots * d);
+  // bf16 experts with the fused gather read their rows from x directly: no copy buffer
+  L.x_perm = take(c.weight_dtype == MOE_BF16 && c.fused_gather ? 0 : es * slots * d);
   L.h = take(es * slots * F);
   L.y_perm = take(es * slots * d);
   L.shared_h = take(es * T * Fs);
@@ -187,6 +188,8 @@ struct FfnArgs {
   const void *s1, *s2, *s3, *b1, *b2, *b3;  // q4 scale / bias
   int w_stride;             // rows from one expert's w1 (w2) block to the next: F, or 2F when
                             // gate and up rows are stacked per expert (w2 = w1 + F rows)
+  const int32_t *gather;    // bf16 tensor-core path only: phase 1 reads row gather[r] of x ([x_rows, d])
+  int x_rows;               // instead of row r of an expert-sorted copy (the fused dispatch gather)
   void *h;                  // [rows_cap, F]
   void *y;                  // [rows_cap, d]
   int *status;

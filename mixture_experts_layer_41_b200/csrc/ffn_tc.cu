@@ -67,6 +67,8 @@ struct TcParams {
   int n_tiles;              // output tiles per group along N
   __nv_bfloat16 *out;       // [rows_cap, N]
   int *status;
+  const int32_t *gather;    // A row r is token gather[r] of the token matrix (mapA over [T, K], one-row box),
+                            // or nullptr: A row r is row r of mapA
 };
 
 struct SharedState {
@@ -146,6 +148,17 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map
       "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], [%2];" ::"r"(
           dst),
       "l"((uint64_t)map), "r"(bar), "r"(x), "r"(y)
+      : "memory");
+}
+
+// Four rows (r0..r3) of a one-row-box map into four consecutive 128-byte rows
+// at dst; the 128-byte swizzle follows the destination address as for a tile.
+__device__ __forceinline__ void tma_gather4(uint32_t dst, const CUtensorMap *map, uint32_t bar, int x, int r0,
+                                            int r1, int r2, int r3) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5, %6, %7}], [%2];" ::"r"(dst),
+      "l"((uint64_t)map), "r"(bar), "r"(x), "r"(r0), "r"(r1), "r"(r2), "r"(r3)
       : "memory");
 }
 
@@ -281,7 +294,59 @@ tc_grouped_gemm(const __grid_constant__ CUtensorMap mapA, const __grid_constant_
   const int kb_n = (p.K + BK - 1) / BK;
   volatile int *abort_flag = &st->abort_flag;
 
-  if (warp == 0) {
+  if (warp == 0 && p.gather) {
+    // ------------------------------------------------------------ TMA producer, gathered A
+    // Fused dispatch: the A tile's 128 rows are fetched straight from the
+    // token matrix, four per lane with tile::gather4 (one-row boxes); lane 0
+    // waits for the stage, posts the byte count and loads the B halves.
+    uint32_t it = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
+      const TileInfo ti = decode_tile(st, nE, p.n_tiles, tile);
+      // rows past the expert's end repeat its first row (their results are masked)
+      const int row_end = st->off[ti.e + 1];
+      int g[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int r = ti.row0 + lane * 4 + i;
+        g[i] = p.gather[r < row_end ? r : ti.row0];
+      }
+      int b0, b1;
+      if (p.mode == MODE_SWIGLU) {
+        b0 = ti.e * p.b_stride + ti.n * 128;
+        b1 = b0;
+      } else {
+        b0 = ti.e * p.b_stride + ti.n * BN;
+        b1 = b0 + 128;
+      }
+      for (int kb = 0; kb < kb_n; ++kb, ++it) {
+        const int s = it % STAGES;
+        const uint32_t ph = (it / STAGES) & 1u;
+        int good = 1;
+        if (lane == 0) good = wait_bounded(&st->empty[s], ph ^ 1u, abort_flag, p.status, kDevTimeoutProducer);
+        good = __shfl_sync(0xffffffffu, good, 0);
+        if (!good) {
+          ok = false;
+          break;
+        }
+        uint8_t *sa = tiles + (size_t)s * STAGE_BYTES;
+        const uint32_t fb = smem_u32(&st->full[s]);
+        if (lane == 0) mbar_expect_tx(&st->full[s], STAGE_BYTES);
+        __syncwarp();
+        tma_gather4(smem_u32(sa) + (uint32_t)lane * 512u, &mapA, fb, kb * BK, g[0], g[1], g[2], g[3]);
+        if (lane == 0) {
+          tma_load_2d(smem_u32(sa + A_BYTES), &mapB0, fb, kb * BK, b0);
+          tma_load_2d(smem_u32(sa + A_BYTES + BH_BYTES), &mapB1, fb, kb * BK, b1);
+        }
+      }
+    }
+    if (!ok && lane == 0) {
+      const uint32_t first = it > (uint32_t)STAGES ? it - STAGES : 0u;
+      for (uint32_t i = first; i < it; ++i)
+        if (!wait_drain(&st->full[i % STAGES], (i / STAGES) & 1u)) record_status(p.status, kDevTimeoutDrain);
+    }
+    __syncwarp();
+  } else if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
       uint32_t it = 0;
@@ -480,12 +545,15 @@ int sm_count() {
 
 // B0 / B1: expert e's rows start at e * b_stride; a map covers the rows up to
 // the end of the last expert's N.
+// gather (nullable): A row r is token gather[r] of A = [a_rows, K] (the
+// fused dispatch); otherwise A is [rows_cap, K] in row order.
 cudaError_t run_gemm(const void *A, int rows_cap, int K, const void *B0, const void *B1, int b_stride, int N,
                      int mode, const int32_t *offsets, int E, int rows, void *out, int *status,
-                     cudaStream_t s) {
+                     cudaStream_t s, const int32_t *gather = nullptr, int a_rows = 0) {
   CUtensorMap ma, mb0, mb1;
   const int b_rows = ((offsets ? E : 1) - 1) * b_stride + N;
-  cudaError_t err = make_map(&ma, A, (uint64_t)K, (uint64_t)rows_cap, BM);
+  cudaError_t err = gather ? make_map(&ma, A, (uint64_t)K, (uint64_t)a_rows, 1)
+                           : make_map(&ma, A, (uint64_t)K, (uint64_t)rows_cap, BM);
   if (err == cudaSuccess) err = make_map(&mb0, B0, (uint64_t)K, (uint64_t)b_rows, 128);
   if (err == cudaSuccess) err = make_map(&mb1, B1, (uint64_t)K, (uint64_t)b_rows, 128);
   if (err != cudaSuccess) return err;
@@ -501,6 +569,7 @@ cudaError_t run_gemm(const void *A, int rows_cap, int K, const void *B0, const v
   p.n_tiles = mode == MODE_SWIGLU ? (N + 127) / 128 : (N + BN - 1) / BN;
   p.out = static_cast<__nv_bfloat16 *>(out);
   p.status = status;
+  p.gather = gather;
   const int nE = offsets ? E : 1;
   const long long upper = ((long long)(rows_cap + BM - 1) / BM + nE) * p.n_tiles;
   const int sms = sm_count();
@@ -517,10 +586,10 @@ cudaError_t launch_ffn_tc_bf16(const FfnArgs &a, cudaStream_t s) {
   cudaError_t err;
   if (a.act == MOE_ACT_SWIGLU)
     err = run_gemm(a.x, a.rows_cap, a.d, a.w1, a.w2, a.w_stride, a.F, MODE_SWIGLU, a.offsets, a.E, a.rows, a.h,
-                   a.status, s);
+                   a.status, s, a.gather, a.x_rows);
   else
     err = run_gemm(a.x, a.rows_cap, a.d, a.w1, a.w1, a.w_stride, a.F, MODE_RELU, a.offsets, a.E, a.rows, a.h,
-                   a.status, s);
+                   a.status, s, a.gather, a.x_rows);
   if (err != cudaSuccess) return err;
   if (a.mid_event && (err = cudaEventRecord(a.mid_event, s)) != cudaSuccess) return err;
   return run_gemm(a.h, a.rows_cap, a.F, a.w3, a.w3, a.d, a.d, MODE_PLAIN, a.offsets, a.E, a.rows, a.y,

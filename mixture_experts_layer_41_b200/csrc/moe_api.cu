@@ -111,13 +111,17 @@ moe_status do_permute(const moe_config &c, const void *x, const int32_t *ids, co
   return err == cudaSuccess ? MOE_OK : cuda_fail(err, "moe_permute");
 }
 
+// gather (nullable): x_perm is the token matrix itself and row r of the
+// expert-sorted order is token gather[r] (bf16 tensor-core path only).
 moe_status do_ffn(const moe_config &c, const void *x_perm, const int32_t *off, const moe_weights *w, void *y,
-                  void *ws, cudaStream_t s, cudaEvent_t mid = nullptr) {
+                  void *ws, cudaStream_t s, cudaEvent_t mid = nullptr, const int32_t *gather = nullptr) {
   const WsLayout L = ws_layout(c);
   FfnArgs a = ffn_args(c, L, ws);
   a.mid_event = mid;
   a.offsets = off;
   a.x = x_perm;
+  a.gather = gather;
+  a.x_rows = c.num_tokens;
   a.w1 = w->w1;
   a.w2 = w->w2;
   a.w3 = w->w3;
@@ -196,6 +200,7 @@ moe_status moe_validate(const moe_config *cfg) {
   if (c.weight_layout != MOE_LAYOUT_SEPARATE && c.weight_layout != MOE_LAYOUT_FUSED_GATE_UP)
     return MOE_ERR_INVALID_ARG;
   if (c.weight_layout == MOE_LAYOUT_FUSED_GATE_UP && c.act != MOE_ACT_SWIGLU) return MOE_ERR_INVALID_ARG;
+  if (c.fused_gather != 0 && c.fused_gather != 1) return MOE_ERR_INVALID_ARG;
   if (c.act_dtype != MOE_F32 && c.act_dtype != MOE_BF16) return MOE_ERR_INVALID_ARG;
   if (c.weight_dtype != MOE_F32 && c.weight_dtype != MOE_BF16 && c.weight_dtype != MOE_Q4_AFFINE_G64)
     return MOE_ERR_INVALID_ARG;
@@ -495,13 +500,18 @@ static moe_status forward_impl(const moe_config &c, const void *x, const float *
   if ((err = mark(MOE_PHASE_START, s)) != cudaSuccess) return cuda_fail(err, "phase event");
   if ((st = do_route(c, x, w_router, router_bias, ids, wts, psum, ws, s)) != MOE_OK) return st;
   if ((err = mark(MOE_PHASE_ROUTE, s)) != cudaSuccess) return cuda_fail(err, "phase event");
-  void *x_perm = ws_ptr<char>(ws, L.x_perm);
-  if ((st = do_permute(c, x, ids, wts, off, ws_ptr<int32_t>(ws, L.perm_token), ws_ptr<float>(ws, L.perm_w),
+  // with the fused gather, bf16 tensor-core experts read their token rows
+  // straight from x: the permutation is built but no row is copied
+  const bool fused_gather = c.weight_dtype == MOE_BF16 && c.fused_gather;
+  int32_t *perm_token = ws_ptr<int32_t>(ws, L.perm_token);
+  void *x_perm = fused_gather ? nullptr : ws_ptr<char>(ws, L.x_perm);
+  if ((st = do_permute(c, x, ids, wts, off, perm_token, ws_ptr<float>(ws, L.perm_w),
                        ws_ptr<int32_t>(ws, L.slot_row), x_perm, raw, kept, dropped, ws, s)) != MOE_OK)
     return st;
   if ((err = mark(MOE_PHASE_PERMUTE, s)) != cudaSuccess) return cuda_fail(err, "phase event");
   void *y_perm = ws_ptr<char>(ws, L.y_perm);
-  if ((st = do_ffn(c, x_perm, off, w, y_perm, ws, s, g_nevents ? g_events[MOE_PHASE_FFN1] : nullptr)) != MOE_OK)
+  if ((st = do_ffn(c, fused_gather ? x : x_perm, off, w, y_perm, ws, s, g_nevents ? g_events[MOE_PHASE_FFN1] : nullptr,
+                   fused_gather ? perm_token : nullptr)) != MOE_OK)
     return st;
   if ((err = mark(MOE_PHASE_FFN2, s)) != cudaSuccess) return cuda_fail(err, "phase event");
   void *shared = nullptr;

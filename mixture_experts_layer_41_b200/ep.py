@@ -103,7 +103,7 @@ class DeviceOps:
     def _local_cfg(self, rows: int) -> L.moe_config:
         c = self.cfg
         return L.moe_config(rows, c.hidden, c.intermediate, self.e_local, 1, L.MOE_ROUTER_SOFTMAX_TOPK, 1, 1.0,
-                            1, 1, 0.0, c.act, c.act_dtype, c.weight_dtype, 0, 0.0, c.weight_layout)
+                            1, 1, 0.0, c.act, c.act_dtype, c.weight_dtype, 0, 0.0, c.weight_layout, 0)
 
     def dispatch(self, x: torch.Tensor) -> Dispatched:
         c = self.cfg

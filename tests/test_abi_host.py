@@ -190,3 +190,10 @@ def test_device_calls_reject_bad_arguments_before_any_launch():
     bad_layout = _cfg()
     bad_layout.weight_layout = 2
     assert api.moe_validate(bad_layout) == L.MOE_ERR_INVALID_ARG
+    bad_gather = _cfg()
+    bad_gather.fused_gather = 2
+    assert api.moe_validate(bad_gather) == L.MOE_ERR_INVALID_ARG
+    # the fused gather drops the expert-sorted copy from the workspace (bf16 experts only)
+    assert api.moe_workspace_size(_cfg(fused_gather=True)) < api.moe_workspace_size(_cfg())
+    q4 = dict(weight_dtype="q4_affine_g64")
+    assert api.moe_workspace_size(_cfg(fused_gather=True, **q4)) == api.moe_workspace_size(_cfg(**q4))

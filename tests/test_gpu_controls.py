@@ -254,3 +254,32 @@ def test_update_bias_after_forward_moves_toward_balance():
     assert layer.status() == 0
     last = layer.o.raw_counts.cpu().numpy()
     assert last.max() < first.max()
+
+
+# ---------------------------------------------------------------- fused dispatch gather
+
+GATHER = {
+    "mixtral_small": workload("mixtral_prefill", T=700, d=512, F=640),
+    "ragged_nk": workload("mixtral_prefill", T=333, d=200, F=136, E=4, k=2),
+    "relu_capacity": workload("switch_top1", T=257, d=136, F=264, E=8, k=2, capacity_factor=1.25),
+    "deepseek_small": workload("deepseek_v3", T=512, d=448, F=256, E=32, n_group=8, topk_group=4, shared_F=256),
+}
+
+
+@pytest.mark.parametrize("name", sorted(GATHER))
+def test_fused_gather_matches_copy(name):
+    """moe_forward with the expert rows gathered inside the grouped GEMM gives
+    the copy path's output bit for bit, with a smaller workspace."""
+    w = GATHER[name]
+    run = Run(w, seed=21).staged()
+    ref = run.out.clone()
+    cfg = cfg_of(w)
+    cfg.fused_gather = 1
+    assert api.moe_workspace_size(cfg) < api.moe_workspace_size(run.cfg)
+    ws = torch.empty(api.moe_workspace_size(cfg), dtype=torch.uint8, device="cuda")
+    out = torch.empty_like(run.out)
+    api.moe_forward(cfg, run.inp["x"], run.inp["w_router"], run.bias, run.weights, out, run.ids, run.wts,
+                    run.stats, ws)
+    torch.cuda.synchronize()
+    assert api.moe_workspace_status(ws) == 0
+    assert torch.equal(_bits(out), _bits(ref))
