@@ -210,6 +210,15 @@ ROUTER_SHAPES = {
     "split_e128_decode": workload("decode_q4", T=40, d=1024, F=64, k=8, weight_format="dense"),
     "split_e256_sigmoid": workload("deepseek_v3", T=70, d=2048, F=64, shared_F=0),
     "split_e40_f32": workload("tiny_fp32", T=90, d=128, F=8, E=40, k=5, act="relu", capacity_factor=0.0),
+    # tensor-core logits (bf16, T >= 512): a hidden size with a ragged last K-block, expert
+    # counts that leave padded columns in the expert tile, the narrow tile, and the
+    # unnormalised softmax that stays on the CUDA cores
+    "tc_e40_ragged_d": workload("mixtral_prefill", T=700, d=200, F=64, E=40, k=5),
+    "tc_e200_sigmoid": workload("deepseek_v3", T=600, d=448, F=64, E=200, n_group=8, topk_group=4, k=8,
+                                shared_F=0),
+    "tc_e16": workload("mixtral_prefill", T=1000, d=1024, F=64, E=16, k=4),
+    "tc_e64_logit_bias": workload("switch_top1", T=900, d=320, F=64, E=64, k=3),
+    "norm_false_e64": workload("mixtral_prefill", T=800, d=256, F=64, E=64, k=4, norm_topk_prob=False),
 }
 
 
