@@ -32,6 +32,10 @@
  *    the workspace; moe_workspace_status() reads it.
  *  - Calls that take `ws` clear its status word first, so two calls that use
  *    the same workspace must not overlap on the GPU.
+ *  - Environment: MOE_TC_PAIR=1 (read at every launch) runs the bf16 grouped
+ *    FFN without the fused gather on pairs of SMs (256-row tiles, one
+ *    tcgen05 cta_group::2 MMA per pair); the results are the same bits as the
+ *    default one-SM kernel.  Unset or any other value: one SM per tile.
  */
 #ifndef MOE_H
 #define MOE_H

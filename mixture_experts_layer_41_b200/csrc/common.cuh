@@ -198,6 +198,7 @@ struct FfnArgs {
 
 cudaError_t launch_ffn_simt_f32(const FfnArgs &a, cudaStream_t s);
 cudaError_t launch_ffn_tc_bf16(const FfnArgs &a, cudaStream_t s);
+cudaError_t launch_ffn_tc2_bf16(const FfnArgs &a, cudaStream_t s);   // pairs of SMs (cta_group::2), no gather
 cudaError_t launch_ffn_q4(const FfnArgs &a, cudaStream_t s);       // SIMT, any d, F multiple of 64
 bool q4_tc_supported(int d, int F);                                 // the tensor-core 4-bit path's shapes
 cudaError_t launch_ffn_q4_tc(const FfnArgs &a, cudaStream_t s);

@@ -4,6 +4,7 @@
 #include "common.cuh"
 
 #include <math.h>
+#include <stdlib.h>
 #include <stdio.h>
 #include <string.h>
 
@@ -81,10 +82,20 @@ FfnArgs ffn_args(const moe_config &c, const WsLayout &L, void *ws) {
   return a;
 }
 
+// The bf16 grouped GEMM runs on one SM per tile unless MOE_TC_PAIR=1 is set
+// in the environment, which selects the kernel on pairs of SMs (same
+// results bit for bit; measured slower on the dense workloads, so it is not
+// the default).  The fused gather always runs on one SM.
+bool use_pair_gemm(const FfnArgs &a) {
+  if (a.gather) return false;
+  const char *env = getenv("MOE_TC_PAIR");
+  return env && env[0] == '1';
+}
+
 cudaError_t run_ffn(const FfnArgs &a, cudaStream_t s) {
   switch (a.kind) {
     case 0: return launch_ffn_simt_f32(a, s);
-    case 1: return launch_ffn_tc_bf16(a, s);
+    case 1: return use_pair_gemm(a) ? launch_ffn_tc2_bf16(a, s) : launch_ffn_tc_bf16(a, s);
     default: return q4_tc_supported(a.d, a.F) ? launch_ffn_q4_tc(a, s) : launch_ffn_q4(a, s);
   }
 }

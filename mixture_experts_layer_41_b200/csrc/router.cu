@@ -92,6 +92,8 @@ __device__ __forceinline__ double exact_logit(const RouteParams &p, int t, int e
   const uint4 *xr = reinterpret_cast<const uint4 *>(static_cast<const __nv_bfloat16 *>(p.x) + (size_t)t * p.d);
   const float4 *wr = reinterpret_cast<const float4 *>(p.w + (size_t)e * p.d);
   double s = 0.0;
+  // four 16-byte loads of x and eight of w in flight per lane
+#pragma unroll 4
   for (int i = lane; i < p.d / 8; i += 32) {
     const uint4 xv = __ldg(xr + i);
     const float4 w0 = __ldg(wr + 2 * i), w1 = __ldg(wr + 2 * i + 1);
@@ -591,6 +593,7 @@ route_select(RouteParams p) {
     double sacc[4];
 #pragma unroll
     for (int u = 0; u < 4; ++u) sacc[u] = 0.0;
+#pragma unroll 4
     for (int q = 0; q < p.ks; ++q) {
 #pragma unroll
       for (int u = 0; u < 4; ++u) {

@@ -283,3 +283,29 @@ def test_fused_gather_matches_copy(name):
     torch.cuda.synchronize()
     assert api.moe_workspace_status(ws) == 0
     assert torch.equal(_bits(out), _bits(ref))
+
+
+# ---------------------------------------------------------------- bf16 grouped GEMM on pairs of SMs
+
+PAIR = dict(GATHER)
+PAIR["mixtral_tail"] = workload("mixtral_prefill", T=1100, d=512, F=384, E=8, k=2)      # 256-row tiles with tails
+PAIR["one_expert_rows"] = workload("switch_top1", T=130, d=264, F=200, E=2, k=1, capacity_factor=0.0)
+
+
+@pytest.mark.parametrize("name", sorted(PAIR))
+def test_paired_sm_gemm_matches_one_sm(name, monkeypatch):
+    """MOE_TC_PAIR=1 runs the bf16 grouped FFN (and the shared expert) on
+    pairs of SMs with 256-row tiles; each output element is the same chain
+    of K-16 tensor-core steps as on one SM, so the layer output is identical
+    bit for bit, ragged N and K, tails past the last row and all."""
+    w = PAIR[name]
+    monkeypatch.setenv("MOE_TC_PAIR", "0")
+    one = Run(w, seed=22).staged()
+    ref = one.out.clone()
+    monkeypatch.setenv("MOE_TC_PAIR", "1")
+    out = torch.empty_like(ref)
+    api.moe_forward(one.cfg, one.inp["x"], one.inp["w_router"], one.bias, one.weights, out, one.ids, one.wts,
+                    one.stats, one.ws)
+    torch.cuda.synchronize()
+    assert api.moe_workspace_status(one.ws) == 0
+    assert torch.equal(_bits(out), _bits(ref))
