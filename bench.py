@@ -170,6 +170,18 @@ def kernels_per_step(w) -> int:
     return route + permute + ffn + shared + 1       # + combine
 
 
+def ffn_kernel_file(w) -> str:
+    """Source of the grouped FFN kernel moe_forward runs for this workload
+    (the library's selection: 4-bit weights on decode-sized groups, at most
+    16 rows per expert, take the warp-level kernel; larger groups tcgen05;
+    hidden or intermediate sizes off the 128 grid the CUDA-core kernel)."""
+    if w.weight_format == "q4_affine_g64":
+        if w.d % 128 or w.F % 128:
+            return "ffn_q4.cu"
+        return "ffn_q4_mma.cu" if w.T * w.k <= 16 * w.E else "ffn_q4_tc.cu"
+    return "ffn_simt.cu" if w.dtype == "f32" else "ffn_tc.cu"
+
+
 def source_hash(path: str) -> str:
     with open(path, "rb") as fh:
         return hashlib.sha256(fh.read()).hexdigest()[:16]
@@ -433,9 +445,7 @@ def run_ours(args):
     dk = costs[dom]
     t_dom = phases[dom] * 1e-3
     t_tensor, t_hbm = dk["flops"] / tensor_peak, dk["bytes"] / hbm_peak
-    kernel_file = os.path.join(ROOT, "mixture_experts_layer_41_b200", "csrc",
-                               "ffn_q4.cu" if w.weight_format == "q4_affine_g64" else
-                               ("ffn_simt.cu" if w.dtype == "f32" else "ffn_tc.cu"))
+    kernel_file = os.path.join(ROOT, "mixture_experts_layer_41_b200", "csrc", ffn_kernel_file(w))
     traffic = recorded_traffic(kernel_file, f"{w.name}:{dom}")
     if t_tensor >= t_hbm and w.weight_format == "dense" and w.dtype == "bf16":
         roof = {"bound": "tensor", "achieved": dk["flops"] / t_dom / 1e12,

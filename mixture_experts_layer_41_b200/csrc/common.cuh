@@ -37,6 +37,59 @@ __device__ __forceinline__ void record_status(int *status, int code) {
   atomicCAS(status, 0, code);
 }
 
+// Grouped kernels' view of the group offsets, read by ONE full warp into
+// shared memory: off[i] = min(max(0, src[0..i]), rows_cap) (the running
+// maximum, so the copy is non-decreasing and in range) with off[0] = 0, and
+// tile_start[e] = sum over e' < e of units(off[e'+1] - off[e']),
+// tile_start[n] = the total.  src == nullptr stands for one group of `rows`
+// rows ({0, rows}, n = 1).  Loads are coalesced and the scans are warp
+// shuffles, so the cost does not grow with one memory round trip per group.
+// Returns true (on every lane) when src needed any repair.
+template <class Units>
+__device__ __forceinline__ bool warp_group_offsets(const int32_t *src, int n, int rows, int rows_cap, int32_t *off,
+                                                   int32_t *tile_start, Units units) {
+  const unsigned full = 0xffffffffu;
+  const int lane = threadIdx.x & 31;
+  int carry = 0;
+  bool bad = false;
+  for (int base = 0; base <= n; base += 32) {
+    const int i = base + lane;
+    const int v = i <= n ? (src ? src[i] : (i == 0 ? 0 : rows)) : 0;
+    int m = i <= n ? v : 0;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int t = __shfl_up_sync(full, m, o);
+      if (lane >= o) m = max(m, t);
+    }
+    m = max(m, carry);
+    const int val = min(m, rows_cap);
+    if (i <= n) {
+      off[i] = val;
+      if (val != v || (i == 0 && v != 0)) bad = true;
+    }
+    carry = __shfl_sync(full, m, 31);
+  }
+  __syncwarp();
+  if (lane == 0) off[0] = 0;
+  __syncwarp();
+  int total = 0;
+  for (int base = 0; base < n; base += 32) {
+    const int e = base + lane;
+    const int u = e < n ? units(off[e + 1] - off[e]) : 0;
+    int x = u;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int t = __shfl_up_sync(full, x, o);
+      if (lane >= o) x += t;
+    }
+    if (e < n) tile_start[e] = total + x - u;
+    total += __shfl_sync(full, x, 31);
+  }
+  if (lane == 0) tile_start[n] = total;
+  __syncwarp();
+  return __any_sync(full, bad);
+}
+
 size_t route_logits_bytes(const moe_config &c);   // defined in router.cu
 
 // ---------------------------------------------------------------- workspace
@@ -202,6 +255,8 @@ cudaError_t launch_ffn_tc2_bf16(const FfnArgs &a, cudaStream_t s);   // pairs of
 cudaError_t launch_ffn_q4(const FfnArgs &a, cudaStream_t s);       // SIMT, any d, F multiple of 64
 bool q4_tc_supported(int d, int F);                                 // the tensor-core 4-bit path's shapes
 cudaError_t launch_ffn_q4_tc(const FfnArgs &a, cudaStream_t s);
+bool q4_mma_supported(int d, int F);                                // the warp-level 4-bit path's shapes
+cudaError_t launch_ffn_q4_mma(const FfnArgs &a, cudaStream_t s);
 
 // Replaces the text moe_last_error() returns on this thread.
 void set_last_error_text(const char *text);

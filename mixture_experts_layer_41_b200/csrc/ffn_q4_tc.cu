@@ -328,25 +328,10 @@ q4_tc_gemm(const __grid_constant__ CUtensorMap mapC0, const __grid_constant__ CU
                  : "memory");
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
   }
-  if (threadIdx.x == 64) {
-    int prev = 0;
-    bool bad = false;
-    for (int i = 0; i <= nE; ++i) {
-      int v = p.offsets[i];
-      if (i == 0 && v != 0) bad = true;
-      if (v < prev) { v = prev; bad = true; }
-      if (v > p.rows_cap) { v = p.rows_cap; bad = true; }
-      st->off[i] = v;
-      prev = v;
-    }
-    st->off[0] = 0;
-    if (bad) record_status(p.status, kDevBadOffsets);
-    int acc = 0;
-    for (int e = 0; e < nE; ++e) {
-      st->tile_start[e] = acc;
-      acc += ((st->off[e + 1] - st->off[e] + NT - 1) / NT) * m_tiles;
-    }
-    st->tile_start[nE] = acc;
+  if (warp == 2) {
+    const bool bad = warp_group_offsets(p.offsets, nE, 0, p.rows_cap, st->off, st->tile_start,
+                                        [m_tiles](int cnt) { return ((cnt + NT - 1) / NT) * m_tiles; });
+    if (bad && lane == 0) record_status(p.status, kDevBadOffsets);
   }
   tc_fence_before();
   __syncthreads();

@@ -243,25 +243,11 @@ tc2_grouped_gemm(const __grid_constant__ CUtensorMap mapA, const __grid_constant
                  : "memory");
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
   }
-  if (threadIdx.x == 64) {
-    int prev = 0;
-    bool bad = false;
-    for (int i = 0; i <= nE; ++i) {
-      int v = p.offsets ? p.offsets[i] : (i == 0 ? 0 : p.rows);
-      if (i == 0 && v != 0) bad = true;
-      if (v < prev) { v = prev; bad = true; }
-      if (v > p.rows_cap) { v = p.rows_cap; bad = true; }
-      st->off[i] = v;
-      prev = v;
-    }
-    st->off[0] = 0;
-    if (bad && leader) record_status(p.status, kDevBadOffsets);
-    int acc = 0;
-    for (int e = 0; e < nE; ++e) {
-      st->tile_start[e] = acc;
-      acc += ((st->off[e + 1] - st->off[e] + 2 * BM - 1) / (2 * BM)) * p.n_tiles;
-    }
-    st->tile_start[nE] = acc;
+  if (warp == 2) {
+    const int n_tiles = p.n_tiles;
+    const bool bad = warp_group_offsets(p.offsets, nE, p.rows, p.rows_cap, st->off, st->tile_start,
+                                        [n_tiles](int cnt) { return ((cnt + 2 * BM - 1) / (2 * BM)) * n_tiles; });
+    if (bad && leader && lane == 0) record_status(p.status, kDevBadOffsets);
   }
   tc_fence_before();
   __syncthreads();

@@ -92,11 +92,24 @@ bool use_pair_gemm(const FfnArgs &a) {
   return env && env[0] == '1';
 }
 
+// 4-bit weights: decode-sized groups (a few token rows per expert) go to the
+// warp-level kernel, whose 8-token MMA blocks fit them; larger groups to the
+// tcgen05 kernel.  MOE_Q4_KERNEL=mma / tc in the environment forces one.
+bool use_q4_mma(const FfnArgs &a) {
+  if (!q4_mma_supported(a.d, a.F)) return false;
+  const char *env = getenv("MOE_Q4_KERNEL");
+  if (env && strcmp(env, "mma") == 0) return true;
+  if (env && strcmp(env, "tc") == 0) return !q4_tc_supported(a.d, a.F);
+  return (long long)a.rows_cap <= 16LL * a.E;
+}
+
 cudaError_t run_ffn(const FfnArgs &a, cudaStream_t s) {
   switch (a.kind) {
     case 0: return launch_ffn_simt_f32(a, s);
     case 1: return use_pair_gemm(a) ? launch_ffn_tc2_bf16(a, s) : launch_ffn_tc_bf16(a, s);
-    default: return q4_tc_supported(a.d, a.F) ? launch_ffn_q4_tc(a, s) : launch_ffn_q4(a, s);
+    default:
+      if (use_q4_mma(a)) return launch_ffn_q4_mma(a, s);
+      return q4_tc_supported(a.d, a.F) ? launch_ffn_q4_tc(a, s) : launch_ffn_q4(a, s);
   }
 }
 

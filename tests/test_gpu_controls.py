@@ -309,3 +309,49 @@ def test_paired_sm_gemm_matches_one_sm(name, monkeypatch):
     torch.cuda.synchronize()
     assert api.moe_workspace_status(one.ws) == 0
     assert torch.equal(_bits(out), _bits(ref))
+
+
+# ---------------------------------------------------------------- 4-bit FFN kernels
+
+Q4 = {
+    "decode_small": workload("decode_q4", T=16, d=256, F=128, E=16, k=4),
+    "decode_many_rows": workload("decode_q4", T=200, d=256, F=256, E=8, k=2),       # several token passes
+    "ragged_passes": workload("decode_q4", T=90, d=384, F=256, E=4, k=3),           # pass tails in both phases
+    "mostly_empty": workload("decode_q4", T=6, d=512, F=384, E=64, k=2),
+    "decode_like": workload("decode_q4", T=64, d=1024, F=768, E=32, k=8),
+}
+
+
+@pytest.mark.parametrize("kernel", ["mma", "tc"])
+@pytest.mark.parametrize("name", sorted(Q4))
+def test_q4_kernels_match_oracle(name, kernel, monkeypatch):
+    """Both 4-bit grouped FFN kernels (warp-level mma.sync fragments and
+    tcgen05 with the weight operand in TMEM), forced in turn, against the
+    oracle on every token (the GPU's own routing, so only the experts and
+    the combine are compared)."""
+    from gpu_harness import check_output
+    monkeypatch.setenv("MOE_Q4_KERNEL", kernel)
+    run = Run(Q4[name], seed=23).staged()
+    assert run.status() == 0
+    check_output(run)
+
+
+@pytest.mark.parametrize("case", ["bf16", "bf16_pair", "q4_mma", "q4_tc"])
+def test_grouped_ffn_repairs_bad_offsets(case, monkeypatch):
+    """Decreasing group offsets (every value inside [0, T*k]) are clamped to a
+    non-decreasing copy, the call completes, and the workspace reports the
+    device-side failure."""
+    if case.startswith("q4"):
+        w = Q4["decode_like"]
+        monkeypatch.setenv("MOE_Q4_KERNEL", case[3:])
+    else:
+        w = workload("mixtral_prefill", T=300, d=256, F=256, E=8, k=2)
+        monkeypatch.setenv("MOE_TC_PAIR", "1" if case == "bf16_pair" else "0")
+    run = Run(w, seed=24).staged()
+    assert run.status() == 0
+    bad = run.offsets.clone()
+    bad[3] = bad[5] + 7                # a step down after index 3
+    bad[3] = min(int(bad[3]), w.T * w.k)
+    api.moe_grouped_ffn(run.cfg, run.x_perm, bad, run.weights, run.y_perm, run.ws)
+    torch.cuda.synchronize()
+    assert run.status() == L.MOE_ERR_DEVICE
