@@ -127,6 +127,14 @@ inline size_t act_size(const moe_config &c) { return c.act_dtype == MOE_F32 ? 4 
 inline int route_blocks(const moe_config &c) {
   return (c.num_tokens + kRouteTokens - 1) / kRouteTokens;
 }
+// tokens per block of the selection pass over logits partials: 8 when
+// 32-token blocks would leave more than half of the 148 SMs idle
+inline int select_tokens_per_block(int T) { return (T + kRouteTokens - 1) / kRouteTokens < 74 ? 8 : 32; }
+// probability-sum rows any route plan writes (at most one per 8 tokens)
+inline int route_part_rows(const moe_config &c) {
+  const int sel = (c.num_tokens + select_tokens_per_block(c.num_tokens) - 1) / select_tokens_per_block(c.num_tokens);
+  return sel > route_blocks(c) ? sel : route_blocks(c);
+}
 inline int perm_blocks(const moe_config &c) {
   return (c.num_tokens + kPermTokens - 1) / kPermTokens;
 }
@@ -145,7 +153,7 @@ inline WsLayout ws_layout(const moe_config &c) {
   const size_t es = act_size(c);
   const size_t slots = T * K;
   L.status = take(256);
-  L.route_part = take(sizeof(double) * route_blocks(c) * E);
+  L.route_part = take(sizeof(double) * route_part_rows(c) * E);
   L.route_logits = take(route_logits_bytes(c));
   L.blk_counts = take(sizeof(int32_t) * perm_blocks(c) * E);
   L.blk_base = take(sizeof(int32_t) * perm_blocks(c) * E);

@@ -574,21 +574,22 @@ route_tiled(RouteParams p) {
   }
 }
 
-constexpr int SEL_WARPS = 32;   // route_select: one warp per token of a 32-token group
-
-template <int EPL>
-__global__ void __launch_bounds__(32 * SEL_WARPS)
+// route_select: one warp per token, TPB tokens per block (32, or 8 when a
+// 32-token grid would leave more than half of the SMs idle); block b writes
+// probability-sum row b of p.part.
+template <int EPL, int TPB>
+__global__ void __launch_bounds__(32 * TPB)
 route_select(RouteParams p) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
-  double *lgs = reinterpret_cast<double *>(smem_raw);                 // [32][E] summed logits
-  double *dscr = lgs + kRouteTokens * p.E;                           // [SEL_WARPS][kMaxExperts]
+  double *lgs = reinterpret_cast<double *>(smem_raw);                 // [TPB][E] summed logits
+  double *dscr = lgs + TPB * p.E;                                    // [TPB][kMaxExperts]
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int E = p.E;
-  const int tb = blockIdx.x * kRouteTokens;
-  constexpr int NT = 32 * SEL_WARPS;
+  const int tb = blockIdx.x * TPB;
+  constexpr int NT = 32 * TPB;
   // every thread sums the slices of 4 (token, expert) logits at a time, in
   // slice order, with the loads of a slice in flight together
-  const int n = kRouteTokens * E;
+  const int n = TPB * E;
   for (int o0 = threadIdx.x; o0 < n; o0 += 4 * NT) {
     double sacc[4];
 #pragma unroll
@@ -623,7 +624,19 @@ route_select(RouteParams p) {
     }
     select_token<EPL>(p, t, lg, psum, wscr, lane);
   }
-  write_prob_partials<EPL, SEL_WARPS>(p, dscr, psum, tb, 1, lane, warp);
+  // the block's probability sums, warps added in order
+  __syncthreads();
+#pragma unroll
+  for (int j = 0; j < EPL; ++j) {
+    const int e = lane + 32 * j;
+    if (e < E) dscr[warp * E + e] = psum[j];
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += NT) {
+    double sum = 0.0;
+    for (int w = 0; w < TPB; ++w) sum += dscr[w * E + e];
+    p.part[(size_t)blockIdx.x * E + e] = sum;
+  }
 }
 
 // prob_sum[e] = sum over 32-token groups in a fixed order: a block per 32
@@ -662,6 +675,22 @@ cudaError_t launch_tiled(const RouteParams &p, dim3 grid, cudaStream_t s) {
   return cudaGetLastError();
 }
 
+// The selection pass over float64 logits partials [ks][T][E].
+template <int EPL, int TPB>
+cudaError_t launch_select_tpb(const RouteParams &p, cudaStream_t s) {
+  const size_t smem = sizeof(double) * ((size_t)TPB * p.E + (size_t)TPB * kMaxExperts);
+  auto sel = route_select<EPL, TPB>;
+  cudaError_t err = cudaFuncSetAttribute(sel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (err != cudaSuccess) return err;
+  sel<<<(p.T + TPB - 1) / TPB, 32 * TPB, smem, s>>>(p);
+  return cudaGetLastError();
+}
+
+template <int EPL>
+cudaError_t launch_select_epl(const RouteParams &p, cudaStream_t s) {
+  return select_tokens_per_block(p.T) == 8 ? launch_select_tpb<EPL, 8>(p, s) : launch_select_tpb<EPL, 32>(p, s);
+}
+
 template <int EPL, bool BF16>
 cudaError_t launch_wide(const RouteParams &p, const RoutePlan &plan, cudaStream_t s) {
   if (plan.split) {
@@ -669,27 +698,12 @@ cudaError_t launch_wide(const RouteParams &p, const RoutePlan &plan, cudaStream_
     const dim3 grid((p.T + 7) / 8, plan.ks, (p.E + 31) / 32);
     cudaError_t err = launch_tiled<1, 1, BF16, true>(p, grid, s);
     if (err != cudaSuccess) return err;
-    const size_t smem = sizeof(double) * ((size_t)kRouteTokens * p.E + (size_t)SEL_WARPS * kMaxExperts);
-    auto sel = route_select<EPL>;
-    err = cudaFuncSetAttribute(sel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (err != cudaSuccess) return err;
-    sel<<<(p.T + kRouteTokens - 1) / kRouteTokens, 32 * SEL_WARPS, smem, s>>>(p);
-    return cudaGetLastError();
+    return launch_select_epl<EPL>(p, s);
   }
   if (plan.tpw == 8) return launch_tiled<EPL, 8, BF16, false>(p, dim3((p.T + 63) / 64), s);
   return launch_tiled<EPL, 4, BF16, false>(p, dim3((p.T + 31) / 32), s);
 }
 
-// The selection pass over float64 logits partials [ks][T][E].
-template <int EPL>
-cudaError_t launch_select_epl(const RouteParams &p, cudaStream_t s) {
-  const size_t smem = sizeof(double) * ((size_t)kRouteTokens * p.E + (size_t)SEL_WARPS * kMaxExperts);
-  auto sel = route_select<EPL>;
-  cudaError_t err = cudaFuncSetAttribute(sel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  if (err != cudaSuccess) return err;
-  sel<<<(p.T + kRouteTokens - 1) / kRouteTokens, 32 * SEL_WARPS, smem, s>>>(p);
-  return cudaGetLastError();
-}
 
 cudaError_t launch_select(const RouteParams &p, cudaStream_t s) {
   if (p.E <= 32) return launch_select_epl<1>(p, s);
@@ -806,7 +820,11 @@ cudaError_t launch_route(const moe_config &c, const void *x, const float *w_rout
     err = c.act_dtype == MOE_BF16 ? launch_any<true>(p, plan, s) : launch_any<false>(p, plan, s);
   }
   if (err != cudaSuccess) return err;
-  const int nb = route_blocks(c);
+  // probability-sum rows: one per selection block when route_select ran,
+  // else one per 32-token block of the fused router kernels
+  const int nb = plan.tc || plan.split ? (c.num_tokens + select_tokens_per_block(c.num_tokens) - 1) /
+                                             select_tokens_per_block(c.num_tokens)
+                                       : route_blocks(c);
   route_finalize<<<(c.num_experts + 31) / 32, 32 * FIN_WARPS, 0, s>>>(route_part, nb, c.num_experts, prob_sum);
   return cudaGetLastError();
 }
