@@ -32,10 +32,16 @@
  *    the workspace; moe_workspace_status() reads it.
  *  - Calls that take `ws` clear its status word first, so two calls that use
  *    the same workspace must not overlap on the GPU.
- *  - Environment: MOE_TC_PAIR=1 (read at every launch) runs the bf16 grouped
- *    FFN without the fused gather on pairs of SMs (256-row tiles, one
- *    tcgen05 cta_group::2 MMA per pair); the results are the same bits as the
- *    default one-SM kernel.  Unset or any other value: one SM per tile.
+ *  - Environment (read at every launch):
+ *    MOE_TC_PAIR=1 runs the bf16 grouped FFN without the fused gather on
+ *    pairs of SMs (256-row tiles, one tcgen05 cta_group::2 MMA per pair);
+ *    the results are the same bits as the default one-SM kernel.
+ *    MOE_Q4_KERNEL=mma | tc picks the 4-bit grouped FFN kernel: warp-level
+ *    MMA fragments (the default when the groups average at most 16 rows) or
+ *    tcgen05 with the weight operand in tensor memory (the default for
+ *    larger groups).  Both need hidden and intermediate sizes that are
+ *    multiples of 128 (else a CUDA-core kernel runs); their results agree
+ *    within the bf16 output tolerance, not bit for bit.
  */
 #ifndef MOE_H
 #define MOE_H
