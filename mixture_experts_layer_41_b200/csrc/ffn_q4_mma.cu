@@ -31,10 +31,11 @@
 // Per CTA (8 warps, persistent over (expert, token pass, 128-feature block)
 // tasks): the pass's token rows (<= NB_MAX * 8) are staged once in shared
 // memory, each warp owns 16 features (x2 for the gate/up pair) and walks K
-// in 128-element blocks with the next block's codes and scales already in
-// flight into registers (two or more CTAs per SM hide the latency; L2 bulk
-// prefetches and a per-thread cp.async ring of several blocks were measured
-// slower).
+// in 128-element blocks with the codes and scales of the next PF blocks in
+// flight into a register ring (PF = 2 for gate + up, 3 for down, two CTAs
+// per SM; L2 bulk prefetches and a per-thread cp.async ring in shared memory
+// were measured slower).  A pass covers 8 tokens in phase 1 and 16 in phase
+// 2 (decode experts hold ~4); an expert with more takes further passes.
 // Phase 1 writes h = silu(x W_gate^T) * (x W_up^T) in bf16 (row order),
 // phase 2 y = h W_down^T.
 #include "common.cuh"
@@ -141,7 +142,7 @@ __device__ __forceinline__ TaskPos decode_task(const int32_t *off, const int32_t
   return t;
 }
 
-template <int MATS, int NB_MAX>
+template <int MATS, int NB_MAX, int PF>
 __global__ void __launch_bounds__(THREADS, MIN_CTAS)
 q4_mma_gemm(const MmaQ4Params p) {
   extern __shared__ __align__(16) uint8_t smem_raw[];
@@ -173,10 +174,16 @@ q4_mma_gemm(const MmaQ4Params p) {
     const size_t wrow = (size_t)t.e * p.w_stride + f0 + g;           // this thread's first weight row
 
     // the first K-block of this warp's rows is on its way while the tokens are staged
-    Frag cur[MATS], nxt[MATS];
+    // register ring of PF + 1 K-blocks: PF blocks in flight ahead of the one in use
+    Frag buf[PF + 1][MATS];
 #pragma unroll
-    for (int m = 0; m < MATS; ++m)
-      load_frag(cur[m], p.q[m] + wrow * qrow, qrow, p.sc[m] + wrow * srow, p.bi[m] + wrow * srow, srow, 0, c);
+    for (int r = 0; r < PF; ++r)
+      if (r < nblk) {
+#pragma unroll
+        for (int m = 0; m < MATS; ++m)
+          load_frag(buf[r][m], p.q[m] + wrow * qrow, qrow, p.sc[m] + wrow * srow, p.bi[m] + wrow * srow, srow, r,
+                    c);
+      }
 
     // stage the pass's tokens in the operand K order (zero rows past the end)
     __syncthreads();                                    // the previous task's readers are done
@@ -219,52 +226,54 @@ q4_mma_gemm(const MmaQ4Params p) {
     const uint8_t *xb = xs + (size_t)g * row_bytes + c * 16;
 
 #pragma unroll 1
-    for (int blk = 0; blk < nblk; ++blk) {
-      if (blk + 1 < nblk) {
+    for (int blk0 = 0; blk0 < nblk; blk0 += PF + 1) {
 #pragma unroll
-        for (int m = 0; m < MATS; ++m)
-          load_frag(nxt[m], p.q[m] + wrow * qrow, qrow, p.sc[m] + wrow * srow, p.bi[m] + wrow * srow, srow,
-                    blk + 1, c);
-      }
-      uint32_t s2lo[MATS], s2hi[MATS], b2lo[MATS], b2hi[MATS];
+      for (int r = 0; r <= PF; ++r) {                   // slot r holds block blk0 + r
+        const int blk = blk0 + r;
+        if (blk >= nblk) break;
+        if (blk + PF < nblk) {
 #pragma unroll
-      for (int m = 0; m < MATS; ++m) {
-        s2lo[m] = prmt(cur[m].s_lo, 0u, sel);
-        s2hi[m] = prmt(cur[m].s_hi, 0u, sel);
-        b2lo[m] = prmt(cur[m].b_lo, 0u, sel);
-        b2hi[m] = prmt(cur[m].b_hi, 0u, sel);
-      }
+          for (int m = 0; m < MATS; ++m)
+            load_frag(buf[(r + PF) % (PF + 1)][m], p.q[m] + wrow * qrow, qrow, p.sc[m] + wrow * srow,
+                      p.bi[m] + wrow * srow, srow, blk + PF, c);
+        }
+        const Frag *cur = buf[r];
+        uint32_t s2lo[MATS], s2hi[MATS], b2lo[MATS], b2hi[MATS];
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        // B registers of steps 2u and 2u+1 for every 8-token block
-        uint4 bv[NB_MAX];
+        for (int m = 0; m < MATS; ++m) {
+          s2lo[m] = prmt(cur[m].s_lo, 0u, sel);
+          s2hi[m] = prmt(cur[m].s_hi, 0u, sel);
+          b2lo[m] = prmt(cur[m].b_lo, 0u, sel);
+          b2hi[m] = prmt(cur[m].b_hi, 0u, sel);
+        }
 #pragma unroll
-        for (int n = 0; n < NB_MAX; ++n)
-          if (n < nb)
-            bv[n] = *reinterpret_cast<const uint4 *>(xb + (size_t)n * 8 * row_bytes + blk * 256 + u * 64);
+        for (int u = 0; u < 4; ++u) {
+          // B registers of steps 2u and 2u+1 for every 8-token block
+          uint4 bv[NB_MAX];
 #pragma unroll
-        for (int hs = 0; hs < 2; ++hs) {
+          for (int n = 0; n < NB_MAX; ++n)
+            if (n < nb)
+              bv[n] = *reinterpret_cast<const uint4 *>(xb + (size_t)n * 8 * row_bytes + blk * 256 + u * 64);
 #pragma unroll
-          for (int m = 0; m < MATS; ++m) {
-            const uint32_t wl = u == 0 ? cur[m].lo.x : u == 1 ? cur[m].lo.y : u == 2 ? cur[m].lo.z : cur[m].lo.w;
-            const uint32_t wh = u == 0 ? cur[m].hi.x : u == 1 ? cur[m].hi.y : u == 2 ? cur[m].hi.z : cur[m].hi.w;
-            const uint32_t a0 = deq_pair(wl, 2 * hs, s2lo[m], b2lo[m]);
-            const uint32_t a1 = deq_pair(wh, 2 * hs, s2hi[m], b2hi[m]);
-            const uint32_t a2 = deq_pair(wl, 2 * hs + 1, s2lo[m], b2lo[m]);
-            const uint32_t a3 = deq_pair(wh, 2 * hs + 1, s2hi[m], b2hi[m]);
+          for (int hs = 0; hs < 2; ++hs) {
 #pragma unroll
-            for (int n = 0; n < NB_MAX; ++n)
-              if (n < nb) {
-                const uint32_t b0 = hs == 0 ? bv[n].x : bv[n].z;
-                const uint32_t b1 = hs == 0 ? bv[n].y : bv[n].w;
-                mma_bf16(acc[m][n], a0, a1, a2, a3, b0, b1);
-              }
+            for (int m = 0; m < MATS; ++m) {
+              const uint32_t wl = u == 0 ? cur[m].lo.x : u == 1 ? cur[m].lo.y : u == 2 ? cur[m].lo.z : cur[m].lo.w;
+              const uint32_t wh = u == 0 ? cur[m].hi.x : u == 1 ? cur[m].hi.y : u == 2 ? cur[m].hi.z : cur[m].hi.w;
+              const uint32_t a0 = deq_pair(wl, 2 * hs, s2lo[m], b2lo[m]);
+              const uint32_t a1 = deq_pair(wh, 2 * hs, s2hi[m], b2hi[m]);
+              const uint32_t a2 = deq_pair(wl, 2 * hs + 1, s2lo[m], b2lo[m]);
+              const uint32_t a3 = deq_pair(wh, 2 * hs + 1, s2hi[m], b2hi[m]);
+#pragma unroll
+              for (int n = 0; n < NB_MAX; ++n)
+                if (n < nb) {
+                  const uint32_t b0 = hs == 0 ? bv[n].x : bv[n].z;
+                  const uint32_t b1 = hs == 0 ? bv[n].y : bv[n].w;
+                  mma_bf16(acc[m][n], a0, a1, a2, a3, b0, b1);
+                }
+            }
           }
         }
-      }
-      if (blk + 1 < nblk) {
-#pragma unroll
-        for (int m = 0; m < MATS; ++m) cur[m] = nxt[m];
       }
     }
 
@@ -299,7 +308,7 @@ size_t smem_bytes(int E, int ntok, int K) {
   return hdr + (size_t)ntok * ((size_t)K * 2 + 64);
 }
 
-template <int MATS, int NB_MAX>
+template <int MATS, int NB_MAX, int PF>
 cudaError_t run(const FfnArgs &a, const void *tokens, int K, int N, int w_stride, const void *q0, const void *q1,
                 const void *s0, const void *s1, const void *b0, const void *b1, void *out, cudaStream_t s) {
   MmaQ4Params p;
@@ -320,7 +329,7 @@ cudaError_t run(const FfnArgs &a, const void *tokens, int K, int N, int w_stride
   p.out = static_cast<uint16_t *>(out);
   p.status = a.status;
   const size_t smem = smem_bytes(a.E, p.ntok, K);
-  auto kern = q4_mma_gemm<MATS, NB_MAX>;
+  auto kern = q4_mma_gemm<MATS, NB_MAX, PF>;
   cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (err != cudaSuccess) return err;
   int per_sm = 0;
@@ -339,15 +348,15 @@ cudaError_t run(const FfnArgs &a, const void *tokens, int K, int N, int w_stride
 
 bool q4_mma_supported(int d, int F) {
   if (d % FB != 0 || F % FB != 0 || d % KB != 0 || F % KB != 0) return false;
-  // the token tile of a pass (16 rows of d in phase 1, 32 rows of F in phase 2) in shared memory
-  return smem_bytes(kMaxExperts, 16, d) <= 227 * 1024 && smem_bytes(kMaxExperts, 32, F) <= 227 * 1024;
+  // the token tile of a pass (8 rows of d in phase 1, 16 rows of F in phase 2) in shared memory
+  return smem_bytes(kMaxExperts, 8, d) <= 227 * 1024 && smem_bytes(kMaxExperts, 16, F) <= 227 * 1024;
 }
 
 cudaError_t launch_ffn_q4_mma(const FfnArgs &a, cudaStream_t s) {
-  cudaError_t err = run<2, 2>(a, a.x, a.d, a.F, a.w_stride, a.w1, a.w2, a.s1, a.s2, a.b1, a.b2, a.h, s);
+  cudaError_t err = run<2, 1, 2>(a, a.x, a.d, a.F, a.w_stride, a.w1, a.w2, a.s1, a.s2, a.b1, a.b2, a.h, s);
   if (err != cudaSuccess) return err;
   if (a.mid_event && (err = cudaEventRecord(a.mid_event, s)) != cudaSuccess) return err;
-  return run<1, 4>(a, a.h, a.F, a.d, a.d, a.w3, nullptr, a.s3, nullptr, a.b3, nullptr, a.y, s);
+  return run<1, 2, 3>(a, a.h, a.F, a.d, a.d, a.w3, nullptr, a.s3, nullptr, a.b3, nullptr, a.y, s);
 }
 
 }  // namespace moe
