@@ -13,6 +13,7 @@ namespace {
 
 __global__ void __launch_bounds__(kMaxExperts)
 bias_update_kernel(int E, const int32_t *counts, float *bias, float coeff) {
+  pdl_enter();
   __shared__ long long part[kMaxExperts / 32];
   const int e = threadIdx.x, lane = e & 31, warp = e >> 5;
   const long long c = e < E ? (long long)counts[e] : 0;
@@ -32,7 +33,7 @@ bias_update_kernel(int E, const int32_t *counts, float *bias, float coeff) {
 }  // namespace
 
 cudaError_t launch_bias_update(int E, const int32_t *counts, float *expert_bias, float coeff, cudaStream_t s) {
-  bias_update_kernel<<<1, kMaxExperts, 0, s>>>(E, counts, expert_bias, coeff);
+  launch_pdl(bias_update_kernel, 1, kMaxExperts, 0, s, E, counts, expert_bias, coeff);
   return cudaGetLastError();
 }
 

@@ -17,6 +17,7 @@ template <bool BF16>
 __global__ void __launch_bounds__(kThreads)
 combine_kernel(const void *y_perm, const int32_t *slot_row, const float *topk_w,
                const void *shared_out, void *out, int k, int d) {
+  pdl_enter();
   const int t = blockIdx.x;
   __shared__ int rows[kMaxTopK];
   __shared__ float wts[kMaxTopK];
@@ -109,10 +110,10 @@ cudaError_t launch_combine(const moe_config &c, const void *y_perm, const int32_
                            const float *topk_w, const void *shared_out, void *out,
                            cudaStream_t s) {
   if (c.act_dtype == MOE_BF16)
-    combine_kernel<true><<<c.num_tokens, kThreads, 0, s>>>(y_perm, slot_row, topk_w, shared_out,
+    launch_pdl(combine_kernel<true>, c.num_tokens, kThreads, 0, s, y_perm, slot_row, topk_w, shared_out,
                                                             out, c.top_k, c.hidden);
   else
-    combine_kernel<false><<<c.num_tokens, kThreads, 0, s>>>(y_perm, slot_row, topk_w, shared_out,
+    launch_pdl(combine_kernel<false>, c.num_tokens, kThreads, 0, s, y_perm, slot_row, topk_w, shared_out,
                                                              out, c.top_k, c.hidden);
   return cudaGetLastError();
 }

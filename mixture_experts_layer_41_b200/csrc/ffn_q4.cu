@@ -76,6 +76,7 @@ __device__ __forceinline__ float warp_sum_f(float v) {
 
 __global__ void __launch_bounds__(WARPS * 32)
 q4_gemm(Q4Args a) {
+  pdl_enter();
   extern __shared__ __align__(16) unsigned char smem_raw[];
   uint16_t *xs = reinterpret_cast<uint16_t *>(smem_raw);   // [rows_per_pass][K]
   const int e = blockIdx.x;
@@ -139,7 +140,7 @@ cudaError_t run_q4(const Q4Args &base, int N, int K, cudaStream_t s) {
   cudaError_t err = cudaFuncSetAttribute(q4_gemm, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (err != cudaSuccess) return err;
   dim3 grid(a.E, (N + FEAT - 1) / FEAT);
-  q4_gemm<<<grid, WARPS * 32, smem, s>>>(a);
+  launch_pdl(q4_gemm, grid, WARPS * 32, smem, s, a);
   return cudaGetLastError();
 }
 

@@ -145,6 +145,7 @@ __device__ __forceinline__ TaskPos decode_task(const int32_t *off, const int32_t
 template <int MATS, int NB_MAX, int PF>
 __global__ void __launch_bounds__(THREADS, MIN_CTAS)
 q4_mma_gemm(const MmaQ4Params p) {
+  pdl_wait();
   extern __shared__ __align__(16) uint8_t smem_raw[];
   int32_t *off = reinterpret_cast<int32_t *>(smem_raw);              // [E+1]
   int32_t *task_start = off + (p.E + 1);                              // [E+1]
@@ -294,6 +295,7 @@ q4_mma_gemm(const MmaQ4Params p) {
       }
     }
   }
+  pdl_trigger();                         // tasks done: the next kernel may be scheduled
 }
 
 int sm_count() {
@@ -340,7 +342,7 @@ cudaError_t run(const FfnArgs &a, const void *tokens, int K, int N, int w_stride
   const long long upper = ((long long)(a.rows_cap + p.ntok - 1) / p.ntok + a.E) * (N / FB);
   const int slots = per_sm * sm_count();
   const int grid = (int)(upper < slots ? upper : slots);
-  kern<<<grid, THREADS, smem, s>>>(p);
+  launch_plain(kern, grid, THREADS, smem, s, p);
   return cudaGetLastError();
 }
 

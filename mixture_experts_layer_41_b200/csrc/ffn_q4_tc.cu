@@ -284,6 +284,7 @@ template <bool PAIR>
 __global__ void __launch_bounds__(THREADS, 1)
 q4_tc_gemm(const __grid_constant__ CUtensorMap mapC0, const __grid_constant__ CUtensorMap mapC1,
            const __grid_constant__ CUtensorMap mapB, const Q4Params p) {
+  pdl_wait();
   using S = Q4Shape<PAIR>;
   constexpr int MATS = S::MATS, STAGES = S::STAGES, SLOTS = S::SLOTS, GROUPS = S::GROUPS;
   constexpr int WPK = S::WARPS_PER_KB;
@@ -563,6 +564,7 @@ q4_tc_gemm(const __grid_constant__ CUtensorMap mapC0, const __grid_constant__ CU
 
   tc_fence_before();
   __syncthreads();
+  pdl_trigger();                         // tiles done: the next kernel may be scheduled
   if (warp == 1) {
     tc_fence_after();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(512u) : "memory");
@@ -654,7 +656,7 @@ cudaError_t run(const FfnArgs &a, const void *tokens, int K, int N, int w_stride
   const long long upper = ((long long)(a.rows_cap + NT - 1) / NT + a.E) * (N / BM);
   const int sms = sm_count();
   const int grid = (int)(upper < sms ? upper : sms);
-  kern<<<grid, THREADS, smem, s>>>(mc0, mc1, mb, p);
+  launch_plain(kern, grid, THREADS, smem, s, mc0, mc1, mb, p);
   return cudaGetLastError();
 }
 

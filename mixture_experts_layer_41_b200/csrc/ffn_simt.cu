@@ -29,6 +29,7 @@ struct SimtArgs {
 };
 
 __global__ void simt_phase1(SimtArgs a) {
+  pdl_enter();
   __shared__ int32_t off[kMaxExperts + 1];
   const int nE = a.offsets ? a.E : 1;
   for (int i = threadIdx.y * blockDim.x + threadIdx.x; i <= nE; i += blockDim.x * blockDim.y)
@@ -55,6 +56,7 @@ __global__ void simt_phase1(SimtArgs a) {
 }
 
 __global__ void simt_phase2(SimtArgs a) {
+  pdl_enter();
   __shared__ int32_t off[kMaxExperts + 1];
   const int nE = a.offsets ? a.E : 1;
   for (int i = threadIdx.y * blockDim.x + threadIdx.x; i <= nE; i += blockDim.x * blockDim.y)
@@ -90,12 +92,12 @@ cudaError_t launch_ffn_simt_f32(const FfnArgs &f, cudaStream_t s) {
   a.y = static_cast<float *>(f.y);
   const dim3 blk(32, 8);
   const dim3 g1((f.F + 31) / 32, (f.rows_cap + 7) / 8);
-  simt_phase1<<<g1, blk, 0, s>>>(a);
+  launch_pdl(simt_phase1, g1, blk, 0, s, a);
   cudaError_t err = cudaGetLastError();
   if (err != cudaSuccess) return err;
   if (f.mid_event && (err = cudaEventRecord(f.mid_event, s)) != cudaSuccess) return err;
   const dim3 g2((f.d + 31) / 32, (f.rows_cap + 7) / 8);
-  simt_phase2<<<g2, blk, 0, s>>>(a);
+  launch_pdl(simt_phase2, g2, blk, 0, s, a);
   return cudaGetLastError();
 }
 

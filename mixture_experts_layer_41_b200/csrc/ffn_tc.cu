@@ -232,6 +232,7 @@ __device__ __forceinline__ float silu_f(float g) { return g / (1.f + __expf(-g))
 __global__ void __launch_bounds__(THREADS, 1)
 tc_grouped_gemm(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CUtensorMap mapB0,
                 const __grid_constant__ CUtensorMap mapB1, const TcParams p) {
+  pdl_wait();
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   const uint32_t pad = (1024u - (smem_u32(smem_raw) & 1023u)) & 1023u;
   uint8_t *tiles = smem_raw + pad;
@@ -488,6 +489,7 @@ tc_grouped_gemm(const __grid_constant__ CUtensorMap mapA, const __grid_constant_
 
   tc_fence_before();
   __syncthreads();
+  pdl_trigger();                         // tiles done: the next kernel may be scheduled
   if (warp == 1) {
     tc_fence_after();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(TMEM_COLS)
@@ -562,7 +564,7 @@ cudaError_t run_gemm(const void *A, int rows_cap, int K, const void *B0, const v
   const int grid = (int)(upper < sms ? upper : sms);
   err = cudaFuncSetAttribute(tc_grouped_gemm, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
   if (err != cudaSuccess) return err;
-  tc_grouped_gemm<<<grid, THREADS, SMEM_BYTES, s>>>(ma, mb0, mb1, p);
+  launch_plain(tc_grouped_gemm, grid, THREADS, SMEM_BYTES, s, ma, mb0, mb1, p);
   return cudaGetLastError();
 }
 

@@ -208,6 +208,7 @@ __device__ __forceinline__ Tile2 decode_tile2(const Shared2 *st, int nE, int til
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
 tc2_grouped_gemm(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CUtensorMap mapB0,
                  const __grid_constant__ CUtensorMap mapB1, const Tc2Params p) {
+  pdl_wait();
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   const uint32_t pad = (1024u - (smem_u32(smem_raw) & 1023u)) & 1023u;
   uint8_t *tiles = smem_raw + pad;
@@ -426,6 +427,7 @@ tc2_grouped_gemm(const __grid_constant__ CUtensorMap mapA, const __grid_constant
 
   tc_fence_before();
   __syncthreads();
+  pdl_trigger();                         // tiles done: the next kernel may be scheduled
   cluster_sync();                        // the pair's MMAs and remote arrivals are over
   if (warp == 1) {
     tc_fence_after();
@@ -511,7 +513,7 @@ cudaError_t run_gemm2(const void *A, int rows_cap, int K, const void *B0, const 
   if (err != cudaSuccess) return err;
   const int pairs = resident_pairs();
   const int clusters = (int)(upper < pairs ? upper : pairs);
-  tc2_grouped_gemm<<<2 * clusters, THREADS, SMEM_BYTES, s>>>(ma, mb0, mb1, p);
+  launch_plain(tc2_grouped_gemm, 2 * clusters, THREADS, SMEM_BYTES, s, ma, mb0, mb1, p);
   return cudaGetLastError();
 }
 

@@ -25,6 +25,7 @@ constexpr int kWords = kPermTokens / 32;   // mask words per expert
 __global__ void __launch_bounds__(kPermTokens)
 count_kernel(const int32_t *ids, int T, int k, int E, int32_t *blk_counts, int32_t *local_rank,
              int *status) {
+  pdl_enter();
   __shared__ uint32_t mask[kMaxExperts * kWords];
   const int tid = threadIdx.x, lane = tid & 31, word = tid >> 5;
   const int t = blockIdx.x * kPermTokens + tid;
@@ -64,6 +65,7 @@ count_kernel(const int32_t *ids, int T, int k, int E, int32_t *blk_counts, int32
 __global__ void scan_kernel(const int32_t *blk_counts, int nb, int E, long long cap, const int32_t *shard_base,
                             int32_t *blk_base, int32_t *raw_counts, int32_t *kept_counts,
                             int32_t *offsets, int32_t *dropped) {
+  pdl_enter();
   __shared__ int32_t kept_s[kMaxExperts];
   __shared__ int32_t drop_s[kMaxExperts];
   const int e = threadIdx.x;
@@ -100,6 +102,7 @@ scatter_kernel(const int32_t *ids, const float *wts, const int32_t *local_rank,
                const int32_t *blk_base, const int32_t *offsets, int T, int k, int E,
                long long cap, const int32_t *shard_base, const char *x, size_t row_bytes, int32_t *perm_token,
                float *perm_w, int32_t *slot_row, char *x_perm) {
+  pdl_enter();
   const int warp_global = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   if (warp_global >= T * k) return;
@@ -145,10 +148,10 @@ cudaError_t launch_permute(const moe_config &c, const void *x, const int32_t *to
                            int *status, cudaStream_t s, const int32_t *shard_base) {
   const int T = c.num_tokens, k = c.top_k, E = c.num_experts;
   const int nb = perm_blocks(c);
-  count_kernel<<<nb, kPermTokens, 0, s>>>(topk_ids, T, k, E, blk_counts, local_rank, status);
+  launch_pdl(count_kernel, nb, kPermTokens, 0, s, topk_ids, T, k, E, blk_counts, local_rank, status);
   cudaError_t err = cudaGetLastError();
   if (err != cudaSuccess) return err;
-  scan_kernel<<<1, kMaxExperts, 0, s>>>(blk_counts, nb, E, (long long)capacity, shard_base, blk_base,
+  launch_pdl(scan_kernel, 1, kMaxExperts, 0, s, blk_counts, nb, E, (long long)capacity, shard_base, blk_base,
                                         raw_counts, kept_counts, expert_offsets, dropped);
   err = cudaGetLastError();
   if (err != cudaSuccess) return err;
@@ -157,12 +160,12 @@ cudaError_t launch_permute(const moe_config &c, const void *x, const int32_t *to
   const int blocks = (int)((warps * 32 + 255) / 256);
   const bool vec16 = (row_bytes % 16) == 0;
   if (vec16)
-    scatter_kernel<16><<<blocks, 256, 0, s>>>(topk_ids, topk_w, local_rank, blk_base, expert_offsets,
+    launch_pdl(scatter_kernel<16>, blocks, 256, 0, s, topk_ids, topk_w, local_rank, blk_base, expert_offsets,
                                               T, k, E, (long long)capacity, shard_base,
                                               static_cast<const char *>(x), row_bytes, perm_token,
                                               perm_w, slot_row, static_cast<char *>(x_perm));
   else
-    scatter_kernel<4><<<blocks, 256, 0, s>>>(topk_ids, topk_w, local_rank, blk_base, expert_offsets,
+    launch_pdl(scatter_kernel<4>, blocks, 256, 0, s, topk_ids, topk_w, local_rank, blk_base, expert_offsets,
                                              T, k, E, (long long)capacity, shard_base,
                                              static_cast<const char *>(x), row_bytes, perm_token,
                                              perm_w, slot_row, static_cast<char *>(x_perm));

@@ -293,6 +293,7 @@ __device__ __forceinline__ void write_prob_partials(const RouteParams &p, double
 template <int EP, bool BF16, int TPW = 2>
 __global__ void __launch_bounds__(32 * (32 / TPW))
 route_rows(RouteParams p) {
+  pdl_enter();
   constexpr int NW = 32 / TPW;                 // warps per 32-token block
   __shared__ double scratch[NW * 16];          // per-warp probability sums
   __shared__ double wscr_all[NW * 32];         // per-warp selection scores (sigmoid groups)
@@ -409,6 +410,7 @@ __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_gr
 template <int EPL, int TPW, bool BF16, bool SPLIT>
 __global__ void __launch_bounds__(kRouteThreads, 1)
 route_tiled(RouteParams p) {
+  pdl_enter();
   using S = TiledShape<EPL, TPW, BF16>;
   constexpr int TM = S::TM, XS = S::XS, XW = S::XW;
   extern __shared__ __align__(16) unsigned char smem_raw[];
@@ -580,6 +582,7 @@ route_tiled(RouteParams p) {
 template <int EPL, int TPB>
 __global__ void __launch_bounds__(32 * TPB)
 route_select(RouteParams p) {
+  pdl_enter();
   extern __shared__ __align__(16) unsigned char smem_raw[];
   double *lgs = reinterpret_cast<double *>(smem_raw);                 // [TPB][E] summed logits
   double *dscr = lgs + TPB * p.E;                                    // [TPB][kMaxExperts]
@@ -645,6 +648,7 @@ route_select(RouteParams p) {
 // order.  Deterministic for a given T and E.
 constexpr int FIN_WARPS = 8;
 __global__ void __launch_bounds__(32 * FIN_WARPS) route_finalize(const double *part, int nb, int E, float *prob_sum) {
+  pdl_enter();
   __shared__ double ws[FIN_WARPS][32];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int e = blockIdx.x * 32 + lane;
@@ -671,7 +675,7 @@ cudaError_t launch_tiled(const RouteParams &p, dim3 grid, cudaStream_t s) {
   auto kern = route_tiled<EPL, TPW, BF16, SPLIT>;
   cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (err != cudaSuccess) return err;
-  kern<<<grid, kRouteThreads, smem, s>>>(p);
+  launch_pdl(kern, grid, kRouteThreads, smem, s, p);
   return cudaGetLastError();
 }
 
@@ -682,7 +686,7 @@ cudaError_t launch_select_tpb(const RouteParams &p, cudaStream_t s) {
   auto sel = route_select<EPL, TPB>;
   cudaError_t err = cudaFuncSetAttribute(sel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (err != cudaSuccess) return err;
-  sel<<<(p.T + TPB - 1) / TPB, 32 * TPB, smem, s>>>(p);
+  launch_pdl(sel, (p.T + TPB - 1) / TPB, 32 * TPB, smem, s, p);
   return cudaGetLastError();
 }
 
@@ -716,11 +720,11 @@ template <bool BF16>
 cudaError_t launch_any(const RouteParams &p, const RoutePlan &plan, cudaStream_t s) {
   const int nb32 = (p.T + kRouteTokens - 1) / kRouteTokens;
   if (p.E <= 8) {
-    route_rows<8, BF16, 2><<<nb32, 32 * 16, 0, s>>>(p);
+    launch_pdl(route_rows<8, BF16, 2>, nb32, 32 * 16, 0, s, p);
     return cudaGetLastError();
   }
   if (p.E <= 16) {
-    route_rows<16, BF16, 4><<<nb32, 32 * 8, 0, s>>>(p);    // 16 experts x 4 tokens of accumulators
+    launch_pdl(route_rows<16, BF16, 4>, nb32, 32 * 8, 0, s, p);    // 16 experts x 4 tokens of accumulators
     return cudaGetLastError();
   }
   if (p.E <= 64) return launch_wide<2, BF16>(p, plan, s);
@@ -825,7 +829,7 @@ cudaError_t launch_route(const moe_config &c, const void *x, const float *w_rout
   const int nb = plan.tc || plan.split ? (c.num_tokens + select_tokens_per_block(c.num_tokens) - 1) /
                                              select_tokens_per_block(c.num_tokens)
                                        : route_blocks(c);
-  route_finalize<<<(c.num_experts + 31) / 32, 32 * FIN_WARPS, 0, s>>>(route_part, nb, c.num_experts, prob_sum);
+  launch_pdl(route_finalize, (c.num_experts + 31) / 32, 32 * FIN_WARPS, 0, s, route_part, nb, c.num_experts, prob_sum);
   return cudaGetLastError();
 }
 

@@ -186,6 +186,7 @@ __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.
 // Layout [3][e_pad][d].
 __global__ void split_router_weights(const float *__restrict__ w, int E, int e_pad, int d,
                                      __nv_bfloat16 *__restrict__ out) {
+  pdl_enter();
   const size_t n = (size_t)e_pad * d;
   for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (size_t)gridDim.x * blockDim.x) {
     const int e = (int)(i / d);
@@ -205,6 +206,7 @@ template <int NTE>
 __global__ void __launch_bounds__(THREADS, 1)
 route_tc_gemm(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ CUtensorMap mapW,
               const TcRouteParams p) {
+  pdl_enter();
   using S = TcShape<NTE>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   const uint32_t pad = (1024u - (smem_u32(smem_raw) & 1023u)) & 1023u;
@@ -403,7 +405,7 @@ cudaError_t run_tc(const moe_config &c, const void *x, const __nv_bfloat16 *wspl
   err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (err != cudaSuccess) return err;
   const dim3 grid((c.num_tokens + TM - 1) / TM, e_pad / NTE, ks);
-  kern<<<grid, THREADS, smem, s>>>(mx, mw, p);
+  launch_pdl(kern, grid, THREADS, smem, s, mx, mw, p);
   return cudaGetLastError();
 }
 
@@ -432,7 +434,7 @@ cudaError_t launch_route_tc_logits(const moe_config &c, const void *x, const flo
   const TcRoutePlan t = tc_route_plan(c);
   const size_t n = (size_t)t.e_pad * c.hidden;
   const int blocks = (int)((n + 255) / 256 < 1184 ? (n + 255) / 256 : 1184);
-  split_router_weights<<<blocks, 256, 0, s>>>(w_router, c.num_experts, t.e_pad, c.hidden, wsplit);
+  launch_pdl(split_router_weights, blocks, 256, 0, s, w_router, c.num_experts, t.e_pad, c.hidden, wsplit);
   cudaError_t err = cudaGetLastError();
   if (err != cudaSuccess) return err;
   switch (t.nte) {
