@@ -26,11 +26,12 @@
 //   route_select  after a SPLIT pass (8-token x 32-expert x hidden-slice
 //                 blocks, used when T is too small to fill the GPU with
 //                 whole-row blocks, e.g. decode) or the tensor-core pass: sums
-//                 the partial logits of 32 tokens in slice order into shared
-//                 memory, then selects with one warp per token.
-// Every selecting block covers 32-token groups and writes one float64
-// probability sum per (group, expert); route_finalize adds the groups in
-// order, so prob_sum is deterministic.
+//                 the partial logits of its tokens (32, or 8 for small T) in
+//                 slice order into shared memory, then selects with one warp
+//                 per token.
+// Every selecting block writes one float64 probability sum per (block,
+// expert); route_finalize adds the rows in order, so prob_sum is
+// deterministic.
 #include "common.cuh"
 
 #include <math.h>
@@ -580,7 +581,7 @@ route_tiled(RouteParams p) {
 // 32-token grid would leave more than half of the SMs idle); block b writes
 // probability-sum row b of p.part.
 template <int EPL, int TPB>
-__global__ void __launch_bounds__(32 * TPB)
+__global__ void __launch_bounds__(32 * TPB, 1)
 route_select(RouteParams p) {
   pdl_enter();
   extern __shared__ __align__(16) unsigned char smem_raw[];
