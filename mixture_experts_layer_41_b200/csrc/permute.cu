@@ -125,16 +125,33 @@ scatter_kernel(const int32_t *ids, const float *wts, const int32_t *local_rank,
   if (row < 0 || x_perm == nullptr) return;
   const char *src = x + (size_t)t * row_bytes;
   char *dst = x_perm + (size_t)row * row_bytes;
+  // four loads per lane in flight before their stores
   if (VEC_BYTES == 16) {
     const uint4 *s4 = reinterpret_cast<const uint4 *>(src);
     uint4 *d4 = reinterpret_cast<uint4 *>(dst);
     const size_t n = row_bytes / 16;
-    for (size_t i = lane; i < n; i += 32) d4[i] = __ldg(s4 + i);
+    for (size_t i0 = lane; i0 < n; i0 += 4 * 32) {
+      uint4 v[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+        if (i0 + 32 * u < n) v[u] = __ldg(s4 + i0 + 32 * u);
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+        if (i0 + 32 * u < n) d4[i0 + 32 * u] = v[u];
+    }
   } else {
     const uint32_t *s1 = reinterpret_cast<const uint32_t *>(src);
     uint32_t *d1 = reinterpret_cast<uint32_t *>(dst);
     const size_t n = row_bytes / 4;
-    for (size_t i = lane; i < n; i += 32) d1[i] = __ldg(s1 + i);
+    for (size_t i0 = lane; i0 < n; i0 += 4 * 32) {
+      uint32_t v[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+        if (i0 + 32 * u < n) v[u] = __ldg(s1 + i0 + 32 * u);
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+        if (i0 + 32 * u < n) d1[i0 + 32 * u] = v[u];
+    }
   }
 }
 
