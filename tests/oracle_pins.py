@@ -190,6 +190,53 @@ def pin_sigmoid_group_bruteforce(O):
             assert all(sel[ids[t, j]] >= sel[ids[t, j + 1]] for j in range(k - 1))
 
 
+def _group_margin_bruteforce(sel, k, n_group, topk_group):
+    """The parity margin of one token, by enumeration: the smaller of the
+    group margin (topk_group-th best group score minus the next best, over
+    every group; +inf when every group survives) and the expert margin (k-th
+    best selection score minus the (k+1)-th among the experts of the best
+    groups; +inf when the survivors number exactly k)."""
+    E = sel.shape[0]
+    gsize = E // n_group
+    gscore = []
+    for g in range(n_group):
+        vals = sorted(sel[g * gsize:(g + 1) * gsize], reverse=True)
+        gscore.append(vals[0] + vals[1])
+    best_groups = max(itertools.combinations(range(n_group), topk_group),
+                      key=lambda c: sum(gscore[i] for i in c))
+    ranked = sorted(gscore, reverse=True)
+    g_margin = ranked[topk_group - 1] - ranked[topk_group] if topk_group < n_group else math.inf
+    pool = sorted((sel[e] for g in best_groups for e in range(g * gsize, (g + 1) * gsize)), reverse=True)
+    e_margin = pool[k - 1] - pool[k] if k < len(pool) else math.inf
+    return min(g_margin, e_margin), g_margin, e_margin
+
+
+def pin_sigmoid_group_margin(O):
+    """The margin that decides which tokens' ids must match bit for bit
+    ([Edge0] group_select_from_logits: the cut between kept and dropped groups
+    and the cut between the k-th and (k+1)-th expert are both decisions), by
+    brute force over the groups, on the selection score (bias included).
+    Both kinds of cut must be the smaller one on some tokens, so that a margin
+    that leaves one of them out, or is measured on the raw score, fails."""
+    rng = _rng(24)
+    group_decides = expert_decides = 0
+    for (E, n_group, topk_group, k) in ((8, 4, 2, 3), (12, 3, 2, 4), (16, 4, 1, 2), (16, 8, 3, 5),
+                                        (8, 2, 2, 5), (6, 3, 1, 2)):
+        logits = rng.standard_normal((60, E)) * 1.5
+        bias = rng.uniform(-0.4, 0.4, E)
+        _, _, s, margin = O.route_sigmoid_group(logits, k, n_group, topk_group, 2.5, True, bias)
+        for t in range(logits.shape[0]):
+            ref, g_m, e_m = _group_margin_bruteforce(s[t] + bias, k, n_group, topk_group)
+            assert abs(margin[t] - ref) < 1e-13 or (math.isinf(ref) and math.isinf(margin[t])), \
+                (E, n_group, topk_group, k, t, margin[t], ref)
+            group_decides += g_m < e_m
+            expert_decides += e_m < g_m
+    assert group_decides > 20 and expert_decides > 20, (group_decides, expert_decides)
+    # every group kept and exactly k survivors: nothing can flip
+    _, _, _, m = O.route_sigmoid_group(rng.standard_normal((5, 8)), 8, 4, 4, 1.0, True, None)
+    assert np.all(np.isinf(m))
+
+
 def pin_sigmoid_group_reductions(O):
     rng = _rng(5)
     logits = rng.standard_normal((25, 8))

@@ -62,6 +62,23 @@ def m_group_score_top1(O):
     O.route_sigmoid_group = ns["route_sigmoid_group"]
 
 
+def m_margin_without_group_cut(O):
+    src = open(ORACLE_PATH).read().replace("np.minimum(e_margin, g_margin)", "e_margin")
+    ns = {}
+    exec(compile(src, ORACLE_PATH, "exec"), ns)
+    O.route_sigmoid_group = ns["route_sigmoid_group"]
+
+
+def m_margin_on_raw_score(O):
+    src = open(ORACLE_PATH).read().replace(
+        "chosen_sel = np.take_along_axis(masked, ids, axis=-1)",
+        "masked = np.where(emask, s, -np.inf)\n    chosen_sel = np.take_along_axis(masked, ids, axis=-1)")
+    assert src != open(ORACLE_PATH).read()
+    ns = {}
+    exec(compile(src, ORACLE_PATH, "exec"), ns)
+    O.route_sigmoid_group = ns["route_sigmoid_group"]
+
+
 def m_no_routed_scaling(O):
     orig = O.route_sigmoid_group
     O.route_sigmoid_group = lambda l, k, g, tg, rs, norm=True, b=None: orig(l, k, g, tg, 1.0, norm, b)
