@@ -3,8 +3,9 @@
 
 One step = one whole layer forward (route, dispatch, grouped expert FFN,
 shared expert, combine) over one batch of synthetic input already resident
-in HBM.  Default workload: the Mixtral-style prefill layer (T=4096,
-hidden 4096, intermediate 14336, 8 experts, top-2, SwiGLU, bf16).
+in HBM.  Default workload: the DeepSeek-V3-style layer, the largest one that
+fits one GPU (T=16384, hidden 7168, expert width 2048, 256 routed experts
+with sigmoid group-limited top-8 routing, one shared SwiGLU expert, bf16).
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
 
@@ -40,10 +41,11 @@ def parse_args():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--workload", default="mixtral_prefill")
+    ap.add_argument("--workload", default="deepseek_v3")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-hash", action="store_true", help="skip the inputs' SHA-256 digests")
     ap.add_argument("--cpu-sample", type=int, default=0, help="tokens in the oracle sample (0 = auto)")
     return ap.parse_args()
 
@@ -155,21 +157,6 @@ def layer_costs(w, R: int, touched: int) -> dict:
                 ffn2=dict(flops=f2, bytes=w3 + R * w.F * es + R * w.d * es))
 
 
-def kernels_per_step(w) -> int:
-    """Kernels of this library launched by one moe_forward."""
-    if w.dtype == "bf16" and w.T >= 512 and (w.router == "sigmoid_group" or w.norm_topk_prob):
-        route = 4                                   # weight split, tensor-core logits, selection, finalize
-    elif w.E <= 16:
-        route = 2                                   # route_rows + route_finalize
-    else:
-        nb32 = (w.T + 31) // 32
-        route = 3 if nb32 < 148 else 2              # split pass adds route_select
-    permute = 3                                     # count, scan, scatter
-    ffn = 2                                         # two expert GEMM phases
-    shared = 2 if w.shared_F else 0
-    return route + permute + ffn + shared + 1       # + combine
-
-
 def ffn_kernel_file(w) -> str:
     """Source of the grouped FFN kernel moe_forward runs for this workload
     (the library's selection: 4-bit weights on decode-sized groups, at most
@@ -203,9 +190,14 @@ def recorded_traffic(kernel_file: str, workload: str):
 
 # ---------------------------------------------------------------- CPU oracle arm
 
-def oracle_sample_run(w, inp, n_tokens: int, seed: int = 0):
-    """Route every token and evaluate the experts on a seeded sample of
-    ``n_tokens`` tokens with the CPU oracle.  Returns (seconds, tokens, result)."""
+def oracle_sample_run(w, inp, n_tokens: int, seed: int = 0) -> dict:
+    """The CPU oracle on a bounded sample of one layer step: the routing and
+    the dispatch over the whole batch (capacity depends on every token), and
+    the expert MLPs (with the combine and shared expert) on a seeded sample
+    of ``n_tokens`` tokens.  Returns the three times, the sample and the
+    oracle's result.  ``estimate_s`` extrapolates the sampled expert time to
+    the whole batch and adds the whole-batch routing and dispatch once: the
+    oracle's time for the full step."""
     import numpy as np
     from mixture_experts_layer_41_b200.inputs import to_host
     from oracle import moe_oracle as O
@@ -223,12 +215,29 @@ def oracle_sample_run(w, inp, n_tokens: int, seed: int = 0):
 
     shared = {k: host[k] for k in ("ws1", "ws2", "ws3")} if w.shared_F else None
     t0 = time.perf_counter()
+    routing = O.route(host["x"], host["w_router"], top_k=w.k, router=w.router, norm=w.norm_topk_prob,
+                      routed_scaling=w.routed_scaling, n_group=w.n_group, topk_group=w.topk_group,
+                      expert_bias=host.get("expert_bias"), logit_bias=host.get("logit_bias"))
+    t1 = time.perf_counter()
+    O.dispatch(np.asarray(routing["ids"]), w.E, O.capacity(w.T, w.k, w.E, w.capacity_factor), routing["weights"])
+    t2 = time.perf_counter()
     res = O.layer_forward(host["x"], host["w_router"], experts, top_k=w.k, act=w.act,
                           capacity_factor=w.capacity_factor, router=w.router, norm=w.norm_topk_prob,
                           routed_scaling=w.routed_scaling, n_group=w.n_group, topk_group=w.topk_group,
                           expert_bias=host.get("expert_bias"), logit_bias=host.get("logit_bias"),
-                          shared=shared, aux_alpha=w.aux_alpha, tokens=toks)
-    return time.perf_counter() - t0, toks, res
+                          shared=shared, aux_alpha=w.aux_alpha, tokens=toks, routing=routing)
+    t3 = time.perf_counter()
+    route_s, dispatch_s = t1 - t0, t2 - t1
+    experts_s = max(0.0, (t3 - t2) - dispatch_s)      # layer_forward re-runs the whole-batch dispatch
+    estimate_s = route_s + dispatch_s + experts_s * w.T / len(toks)
+    return dict(route_s=route_s, dispatch_s=dispatch_s, experts_s=experts_s, wall_s=t3 - t0,
+                estimate_s=estimate_s, tokens=toks, result=res)
+
+
+def sample_text(w, o: dict) -> str:
+    return (f"oracle routing + dispatch of all {w.T} tokens ({o['route_s'] + o['dispatch_s']:.1f} s) and expert "
+            f"MLPs of {len(o['tokens'])} seeded tokens ({o['experts_s']:.1f} s), extrapolated to {w.T} tokens: "
+            f"value = T / (route + dispatch + experts * T / sample)")
 
 
 def blas_threads() -> int:
@@ -240,15 +249,25 @@ def blas_threads() -> int:
         return os.cpu_count() or 1
 
 
-def auto_sample(w) -> int:
-    # about 10-30 s of oracle work on a few dozen host cores
-    per_tok = 6.0 * w.d * w.F * w.k
-    n = int(4e11 / max(per_tok, 1.0))
-    return max(8, min(w.T, n, 256))
+def auto_sample(w, per_step_s: float = 15.0) -> int:
+    """Tokens in the oracle's expert sample, for about ``per_step_s`` seconds
+    of host work: the oracle widens each touched expert's weights to float64
+    (the dominant cost when the sample touches many experts) and evaluates
+    the k expert MLPs of each sampled token."""
+    per_tok = 6.0 * w.d * w.F * w.k                     # float64 MACs x 2 per sampled token
+    widen = 3.0 * w.d * w.F * 4e-9                      # seconds to widen one expert (~4 ns per element)
+    experts_per_tok = min(w.k, w.E)
+    n = 8
+    while n < w.T:
+        touched = min(w.E, n * experts_per_tok)
+        est = touched * widen + n * per_tok / 2e10
+        if est > per_step_s:
+            break
+        n *= 2
+    return max(4, min(w.T, n // 2 if n > 8 else n))
 
 
 def run_reference(args):
-    import torch
     from mixture_experts_layer_41_b200.inputs import make_inputs, workload
 
     rank = int(os.environ.get("RANK", "0"))
@@ -256,26 +275,60 @@ def run_reference(args):
         return 0
     w = workload(args.workload)
     inp = make_inputs(w, seed=args.seed, device="cpu")
-    n = args.cpu_sample or max(4, auto_sample(w) // 8)
+    n = args.cpu_sample or max(4, auto_sample(w, per_step_s=4.0))
     for _ in range(args.warmup):
         oracle_sample_run(w, inp, n, seed=args.seed)
-    times = []
-    for i in range(args.steps):
-        dt, toks, _ = oracle_sample_run(w, inp, n, seed=args.seed + i)
-        times.append(dt)
-    sec = statistics.mean(times)
-    value = len(toks) / sec
+    runs = [oracle_sample_run(w, inp, n, seed=args.seed + i) for i in range(args.steps)]
+    sec = statistics.mean(o["estimate_s"] for o in runs)
+    value = w.T / sec
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": sec * 1e3, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": w.name, "T": w.T, "d": w.d, "F": w.F, "E": w.E, "top_k": w.k},
+        "config": config_of(w, 1),
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
-                         "sample": f"route all {w.T} tokens, expert MLPs on {len(toks)} sampled tokens per step"},
+                         "sample": sample_text(w, runs[-1]) + "; a fresh token sample each step"},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
     return 0
+
+
+def config_of(w, world: int) -> dict:
+    return {"workload": w.name, "T": w.T, "d": w.d, "F": w.F, "E": w.E, "top_k": w.k, "act": w.act,
+            "router": w.router, "capacity_factor": w.capacity_factor or None, "weights": w.weight_format,
+            "shared_F": w.shared_F, "parallelism": f"replicas x{world}"}
+
+
+def input_hashes(inp: dict) -> dict:
+    """SHA-256 of every input tensor's bytes.  Large tensors are hashed in
+    256 MiB chunks (in parallel); the tensor's digest is then the SHA-256 of
+    its chunks' digests in order."""
+    import concurrent.futures as cf
+    chunk = 256 << 20
+    out = {"scheme": "sha256 of each 256 MiB chunk of the tensor's bytes, then sha256 of the chunk digests"}
+
+    workers = min(16, os.cpu_count() or 4)
+
+    def digest(t):
+        flat = t.detach().contiguous().view(-1).view(torch_uint8())
+        offs = list(range(0, flat.numel(), chunk))
+        parts = []
+        with cf.ThreadPoolExecutor(max_workers=workers) as ex:
+            for i in range(0, len(offs), workers):          # at most `workers` chunks on the host at once
+                host = [flat[o:o + chunk].cpu().numpy() for o in offs[i:i + workers]]
+                parts += list(ex.map(lambda b: hashlib.sha256(b).digest(), host))
+        return hashlib.sha256(b"".join(parts)).hexdigest()
+
+    for k in sorted(inp):
+        if inp[k] is not None:
+            out[k] = digest(inp[k])
+    return out
+
+
+def torch_uint8():
+    import torch
+    return torch.uint8
 
 
 # ---------------------------------------------------------------- GPU arm
@@ -325,6 +378,10 @@ def run_ours(args):
     # warm-up
     for _ in range(args.warmup):
         layer.forward(x)
+    torch.cuda.synchronize()
+    n0 = api.moe_kernel_launches()
+    layer.forward(x)
+    launches_per_step = api.moe_kernel_launches() - n0
     torch.cuda.synchronize()
     st = layer.status()
     if st != 0:
@@ -454,45 +511,53 @@ def run_ours(args):
 
     peaks, peak_src = load_peaks()
     costs = layer_costs(w, R, touched)
-    # The expert GEMMs are timed inside back-to-back layer steps that run long
-    # enough to reach the 1 kW power cap, so the tensor roofline is the
-    # sustained cuBLAS figure; the burst fraction is reported beside it.
-    tensor_peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]) * 1e12
+    # Denominators: the burst bf16 GEMM figure (a timed region of a few
+    # hundred steps is seconds at most; the clocks sampled during it are in
+    # "clocks"), with the fraction of the sustained (power-capped) figure
+    # reported beside it.
+    tensor_peak = peaks["bf16_tflops"] * 1e12
+    sustained = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]) * 1e12
     hbm_peak = peaks["hbm_gbs"] * 1e9
+    tensor_bound = w.weight_format == "dense" and w.dtype == "bf16"
+
+    def phase_roof(name):
+        c = costs[name]
+        t = phases[name] * 1e-3
+        if tensor_bound and c["flops"] / tensor_peak >= c["bytes"] / hbm_peak:
+            a = c["flops"] / t / 1e12
+            return {"bound": "tensor", "achieved": a, "peak": tensor_peak / 1e12, "unit": "TFLOP/s",
+                    "frac": a * 1e12 / tensor_peak, "frac_of_sustained": a * 1e12 / sustained, "ms": phases[name]}
+        a = c["bytes"] / t / 1e9
+        return {"bound": "hbm", "achieved": a, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": a * 1e9 / hbm_peak, "ms": phases[name]}
+
+    gemm_phases = {"ffn1": phase_roof("ffn1"), "ffn2": phase_roof("ffn2")}
     # dominant kernel: the longer expert GEMM phase
     dom = "ffn1" if phases["ffn1"] >= phases["ffn2"] else "ffn2"
     dk = costs[dom]
-    t_dom = phases[dom] * 1e-3
-    t_tensor, t_hbm = dk["flops"] / tensor_peak, dk["bytes"] / hbm_peak
+    roof = {k: v for k, v in gemm_phases[dom].items() if k != "ms"}
     kernel_file = os.path.join(ROOT, "mixture_experts_layer_41_b200", "csrc", ffn_kernel_file(w))
-    traffic = recorded_traffic(kernel_file, f"{w.name}:{dom}")
-    if t_tensor >= t_hbm and w.weight_format == "dense" and w.dtype == "bf16":
-        roof = {"bound": "tensor", "achieved": dk["flops"] / t_dom / 1e12,
-                "peak": tensor_peak / 1e12, "unit": "TFLOP/s",
-                "frac_of_burst_peak": dk["flops"] / t_dom / 1e12 / peaks["bf16_tflops"]}
-    else:
-        roof = {"bound": "hbm", "achieved": dk["bytes"] / t_dom / 1e9, "peak": peaks["hbm_gbs"], "unit": "GB/s"}
-    roof["frac"] = roof["achieved"] / roof["peak"]
-    roof["traffic"] = traffic
+    roof["traffic"] = recorded_traffic(kernel_file, f"{w.name}:{dom}")
     roof["kernel"] = {"ffn1": "grouped expert GEMM, phase 1 (gate/up or in)",
                       "ffn2": "grouped expert GEMM, phase 2 (down or out)"}[dom]
-    roof["peak_source"] = f"{peak_src} ({'bf16 GEMM, sustained' if roof['bound'] == 'tensor' else 'HBM copy'})"
+    roof["peak_source"] = f"{peak_src} ({'bf16 GEMM, burst' if roof['bound'] == 'tensor' else 'HBM copy'})"
     roof["algorithmic"] = {"flop_per_launch": dk["flops"], "bytes_per_launch": dk["bytes"],
                            "ms_per_launch": phases[dom]}
     t_layer_roof = max(costs["flops"] / tensor_peak, costs["bytes"] / hbm_peak)
+    t_layer_roof_sus = max(costs["flops"] / sustained, costs["bytes"] / hbm_peak)
 
     per_gpu = w.T / (ms_max * 1e-3)
     line = {
         "metric": METRIC, "value": per_gpu * world, "unit": UNIT, "n_gpus": world, "steps": K,
         "warmup": args.warmup, "ms_per_step": ms_max, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16" if w.dtype == "bf16" else w.dtype, "data": "synthetic",
-        "config": {"workload": w.name, "T": w.T, "d": w.d, "F": w.F, "E": w.E, "top_k": w.k, "act": w.act,
-                   "router": w.router, "capacity_factor": w.capacity_factor or None,
-                   "weights": w.weight_format, "shared_F": w.shared_F, "parallelism": f"replicas x{world}",
-                   "l2": "inputs larger than L2: every step streams all touched expert weights "
-                         f"({costs['bytes'] / 1e9:.2f} GB) from HBM"},
+        "config": dict(config_of(w, world),
+                       l2="inputs larger than L2: every step streams all touched expert weights "
+                          f"({costs['bytes'] / 1e9:.2f} GB) from HBM"),
         "roofline": roof,
+        "gemm_phases": gemm_phases,
         "layer_roofline": {"frac": t_layer_roof / (ms_max * 1e-3), "roof_ms": t_layer_roof * 1e3,
+                           "frac_of_sustained": t_layer_roof_sus / (ms_max * 1e-3),
                            "flop": costs["flops"], "bytes": costs["bytes"],
                            "tflops": costs["flops"] / (ms_max * 1e-3) / 1e12},
         "phases_ms": {k: round(v, 4) for k, v in phases.items()},
@@ -502,7 +567,8 @@ def run_ours(args):
                 "serial": {"value": world * w.T / (e2e_serial_ms * 1e-3), "ms_per_step": e2e_serial_ms,
                            "streams": 1},
                 "matches_device_out": bool(same)},
-        "gpu_launches": K * kernels_per_step(w),
+        "gpu_launches": K * launches_per_step,
+        "launches_per_step": launches_per_step,
         "launch": "cuda_graph" if graph is not None else "eager",
         "eager_ms_per_step": eager_ms,
         "clocks": clocks,
@@ -510,17 +576,18 @@ def run_ours(args):
 
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         n = args.cpu_sample or auto_sample(w)
-        host_inp = {k: v for k, v in inp.items()}
-        sec, toks, res = oracle_sample_run(w, host_inp, n, seed=args.seed)
+        o = oracle_sample_run(w, dict(inp), n, seed=args.seed)
+        toks = o["tokens"]
         got = layer.o.out.float().cpu().numpy().astype(np.float64)[toks]
-        ref = res["out"][toks]
+        ref = o["result"]["out"][toks]
         err = float(np.abs(got - ref).max() / max(np.abs(ref).max(), 1e-30))
-        line["cpu_baseline"] = {"value": len(toks) / sec, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
-                                "sample": f"route all {w.T} tokens + expert MLPs of {len(toks)} seeded tokens "
-                                          f"({sec:.1f} s)"}
+        line["cpu_baseline"] = {"value": w.T / o["estimate_s"], "unit": UNIT, "cores": blas_threads(),
+                                "kind": "oracle", "sample": sample_text(w, o)}
         line["parity_on_sample"] = {"tokens": int(len(toks)), "rel_err": err,
                                     "tol": 1e-5 if w.dtype == "f32" else 2e-2,
                                     "ok": err <= (1e-5 if w.dtype == "f32" else 2e-2)}
+    if rank == 0 and not args.no_hash:
+        line["inputs_sha256"] = input_hashes(inp)
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:

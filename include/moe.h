@@ -196,9 +196,49 @@ const char *moe_status_string(moe_status s);
 /* Text of the last MOE_ERR_CUDA / MOE_ERR_DEVICE seen by this thread. */
 const char *moe_last_error(void);
 
+/* Kernels this library has launched in this process so far (all threads,
+ * every entry point, including launches captured into a CUDA graph, which a
+ * graph replay then repeats without passing through here).  The difference
+ * across one call is that call's launch count. */
+int64_t moe_kernel_launches(void);
+
 /* Synchronises `stream` and reads the device status word a kernel leaves in
  * `ws` (MOE_OK, or MOE_ERR_DEVICE with the site in moe_last_error()). */
 moe_status moe_workspace_status(const void *ws, moe_stream_t stream);
+
+/* Where moe_forward keeps its intermediates inside `ws` (host only, no device
+ * work), so a caller can read them after the stream is synchronised (for
+ * example the permutation the dispatch built, or the expert-sorted rows the
+ * grouped FFN consumed) and check that nothing is written outside them.
+ * Regions, in moe_forward's terms:
+ *   MOE_WS_OFFSETS     expert_offsets [E+1] int32
+ *   MOE_WS_PERM_TOKEN  perm_token [T*k] int32 (first off[E] valid)
+ *   MOE_WS_PERM_W      perm_w [T*k] f32
+ *   MOE_WS_SLOT_ROW    slot_row [T,k] int32
+ *   MOE_WS_X_PERM      x_perm [T*k, d] act_dtype (0 bytes with the fused gather)
+ *   MOE_WS_H           the grouped FFN intermediate [T*k, F] act_dtype; also
+ *                      the intermediate of moe_grouped_ffn
+ *   MOE_WS_Y_PERM      y_perm [T*k, d] act_dtype
+ *   MOE_WS_SHARED_H    the shared expert's intermediate [T, Fs] (0 bytes without one)
+ *   MOE_WS_SHARED_OUT  the shared expert's output [T, d] (0 bytes without one)
+ * Rows at or past off[E] (and, in x_perm / h / y_perm, every row when the
+ * layer routes nothing) are never written.  *offset is a byte offset from the
+ * start of ws (256-byte aligned) and *bytes the region's size; the layout is
+ * a function of the configuration only.  Returns MOE_ERR_INVALID_ARG for an
+ * unknown region or NULL output, or the moe_validate status. */
+typedef enum moe_ws_region {
+  MOE_WS_OFFSETS = 0,
+  MOE_WS_PERM_TOKEN = 1,
+  MOE_WS_PERM_W = 2,
+  MOE_WS_SLOT_ROW = 3,
+  MOE_WS_X_PERM = 4,
+  MOE_WS_H = 5,
+  MOE_WS_Y_PERM = 6,
+  MOE_WS_SHARED_H = 7,
+  MOE_WS_SHARED_OUT = 8,
+  MOE_WS_REGION_COUNT = 9
+} moe_ws_region;
+moe_status moe_workspace_region(const moe_config *cfg, int32_t region, size_t *offset, size_t *bytes);
 
 /* Optional phase timing.  Registers MOE_PHASE_COUNT CUDA events (cudaEvent_t
  * handles created by the caller, in moe_phase order) that the following
@@ -242,16 +282,22 @@ moe_status moe_route(const moe_config *cfg, const void *x, const float *w_router
  * memory (no page has a counterpart: this exists for library users only).
  * Callers hosted by a framework that owns every device allocation, or on a
  * path where an allocation and the synchronisation it can imply are not
- * allowed, have no `ws` to pass.  Same arguments and results as moe_route,
- * minus ws: the router's one scratch buffer (per-block partial probability
- * sums) is a fixed device array inside the library, 1 MiB on every GPU that
- * loads it, held until the process exits.
+ * allowed, have no `ws` to pass.  Same arguments as moe_route, minus ws: the
+ * router's one scratch buffer (per-block partial probability sums) is a
+ * fixed device array inside the library, 1 MiB on every GPU that loads it,
+ * held until the process exits.
+ * Results agree with moe_route's within the router tolerances (ids on tokens
+ * whose selection margin exceeds 1e-4, weights 1e-6 and prob_sum 1e-5
+ * relative): this call always uses the CUDA-core router with whole-row
+ * blocks, never the split or tensor-core pass (their logits live in the
+ * workspace), so large bf16 batches also route more slowly than moe_route.
  * Limit: ceil(T/32) * E <= 131072 (e.g. T = 16384 with E = 256); larger
  * problems return MOE_ERR_UNSUPPORTED with the reason in moe_last_error().
- * The first call on each device looks up that device's copy of the array
- * (with the device current), so make it before any stream capture.  All
- * calls share the array: calls that overlap on the GPU race, so serialise
- * them.  Each call writes every entry it reads; nothing carries over. */
+ * The first call in each CUDA context of a device looks up that context's
+ * copy of the array (with the device current), so make it before any stream
+ * capture.  All calls share the array: calls that overlap on the GPU race,
+ * so serialise them.  Each call writes every entry it reads; nothing carries
+ * over. */
 moe_status moe_route_noalloc(const moe_config *cfg, const void *x, const float *w_router,
                              const float *router_bias, int32_t *topk_ids, float *topk_w,
                              float *prob_sum, moe_stream_t stream);

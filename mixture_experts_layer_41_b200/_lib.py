@@ -23,6 +23,9 @@ MOE_ERR_DEVICE = 7
 # moe_phase
 MOE_PHASE_START, MOE_PHASE_ROUTE, MOE_PHASE_PERMUTE, MOE_PHASE_FFN1, MOE_PHASE_FFN2, MOE_PHASE_SHARED, \
     MOE_PHASE_COMBINE, MOE_PHASE_COUNT = range(8)
+# moe_ws_region
+MOE_WS_OFFSETS, MOE_WS_PERM_TOKEN, MOE_WS_PERM_W, MOE_WS_SLOT_ROW, MOE_WS_X_PERM, MOE_WS_H, MOE_WS_Y_PERM, \
+    MOE_WS_SHARED_H, MOE_WS_SHARED_OUT, MOE_WS_REGION_COUNT = range(10)
 # moe_router_kind
 MOE_ROUTER_SOFTMAX_TOPK = 0
 MOE_ROUTER_SIGMOID_GROUP = 1
@@ -87,8 +90,10 @@ SIGNATURES = {
                                      C.POINTER(C.c_double), C.POINTER(C.c_int32)]),
     "moe_status_string": (C.c_char_p, [C.c_int]),
     "moe_last_error": (C.c_char_p, []),
+    "moe_kernel_launches": (C.c_int64, []),
     "moe_workspace_status": (C.c_int, [_P, _P]),
     "moe_set_phase_events": (C.c_int, [C.POINTER(C.c_void_p), C.c_int32]),
+    "moe_workspace_region": (C.c_int, [_CFG, C.c_int32, C.POINTER(C.c_size_t), C.POINTER(C.c_size_t)]),
     "moe_route": (C.c_int, [_CFG, _P, _P, _P, _P, _P, _P, _P, C.c_size_t, _P]),
     "moe_route_noalloc": (C.c_int, [_CFG, _P, _P, _P, _P, _P, _P, _P]),
     "moe_route_forced": (C.c_int, [_CFG, _P, _P, _P, _P, _P, _P, _P, _P, C.c_size_t, _P]),

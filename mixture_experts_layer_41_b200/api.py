@@ -85,6 +85,11 @@ def moe_routing_health(cfg: moe_config, kept_counts_host: torch.Tensor, dropped:
                 collapsed=bool(col.value))
 
 
+def moe_kernel_launches() -> int:
+    """Kernels the library has launched in this process so far."""
+    return L.lib().moe_kernel_launches()
+
+
 def moe_status_string(status: int) -> str:
     return L.lib().moe_status_string(status).decode()
 
@@ -103,6 +108,25 @@ def moe_set_phase_events(events) -> None:
 
 def moe_workspace_status(ws: torch.Tensor, stream=None) -> int:
     return L.lib().moe_workspace_status(_p(ws), _s(stream))
+
+
+_REGIONS = {"offsets": L.MOE_WS_OFFSETS, "perm_token": L.MOE_WS_PERM_TOKEN, "perm_w": L.MOE_WS_PERM_W,
+            "slot_row": L.MOE_WS_SLOT_ROW, "x_perm": L.MOE_WS_X_PERM, "h": L.MOE_WS_H, "y_perm": L.MOE_WS_Y_PERM,
+            "shared_h": L.MOE_WS_SHARED_H, "shared_out": L.MOE_WS_SHARED_OUT}
+
+
+def moe_workspace_region(cfg: moe_config, region: str):
+    """(byte offset, bytes) of one of moe_forward's intermediates inside the workspace."""
+    off, n = C.c_size_t(), C.c_size_t()
+    check(L.lib().moe_workspace_region(C.byref(cfg), _REGIONS[region], C.byref(off), C.byref(n)),
+          "moe_workspace_region")
+    return off.value, n.value
+
+
+def workspace_view(cfg: moe_config, ws: torch.Tensor, region: str, dtype: torch.dtype, cols: int = 1):
+    """A tensor view of one workspace region (no copy), [bytes / (cols * itemsize), cols]."""
+    off, n = moe_workspace_region(cfg, region)
+    return ws[off:off + n].view(dtype).view(-1, cols)
 
 
 # ---------------------------------------------------------------- device calls

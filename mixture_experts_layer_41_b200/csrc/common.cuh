@@ -51,9 +51,13 @@ __device__ __forceinline__ void pdl_enter() {
   pdl_trigger();
 }
 
+// Counts every kernel this library launches (moe_kernel_launches).
+void note_launch();
+
 template <typename... KArgs, typename... Args>
 inline cudaError_t launch_kernel(bool pdl, void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
                                  cudaStream_t s, Args &&...args) {
+  note_launch();
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
@@ -161,6 +165,7 @@ struct WsLayout {
   size_t x_stage;      // act[T][d]   (moe_forward_host)
   size_t out_stage;    // act[T][d]
   size_t total;
+  size_t region_bytes[MOE_WS_REGION_COUNT];   // unpadded sizes of the moe_ws_region buffers
 };
 
 inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
@@ -201,10 +206,11 @@ inline WsLayout ws_layout(const moe_config &c) {
   L.blk_counts = take(sizeof(int32_t) * perm_blocks(c) * E);
   L.blk_base = take(sizeof(int32_t) * perm_blocks(c) * E);
   L.local_rank = take(sizeof(int32_t) * slots);
-  L.offsets = take(sizeof(int32_t) * (E + 1));
-  L.perm_token = take(sizeof(int32_t) * slots);
-  L.perm_w = take(sizeof(float) * slots);
-  L.slot_row = take(sizeof(int32_t) * slots);
+  size_t *rb = L.region_bytes;
+  L.offsets = take(rb[MOE_WS_OFFSETS] = sizeof(int32_t) * (E + 1));
+  L.perm_token = take(rb[MOE_WS_PERM_TOKEN] = sizeof(int32_t) * slots);
+  L.perm_w = take(rb[MOE_WS_PERM_W] = sizeof(float) * slots);
+  L.slot_row = take(rb[MOE_WS_SLOT_ROW] = sizeof(int32_t) * slots);
   L.topk_ids = take(sizeof(int32_t) * slots);
   L.topk_w = take(sizeof(float) * slots);
   L.raw_counts = take(sizeof(int32_t) * E);
@@ -212,11 +218,11 @@ inline WsLayout ws_layout(const moe_config &c) {
   L.prob_sum = take(sizeof(float) * E);
   L.dropped = take(sizeof(int32_t));
   // bf16 experts with the fused gather read their rows from x directly: no copy buffer
-  L.x_perm = take(c.weight_dtype == MOE_BF16 && c.fused_gather ? 0 : es * slots * d);
-  L.h = take(es * slots * F);
-  L.y_perm = take(es * slots * d);
-  L.shared_h = take(es * T * Fs);
-  L.shared_out = take(Fs ? es * T * d : 0);
+  L.x_perm = take(rb[MOE_WS_X_PERM] = c.weight_dtype == MOE_BF16 && c.fused_gather ? 0 : es * slots * d);
+  L.h = take(rb[MOE_WS_H] = es * slots * F);
+  L.y_perm = take(rb[MOE_WS_Y_PERM] = es * slots * d);
+  L.shared_h = take(rb[MOE_WS_SHARED_H] = es * T * Fs);
+  L.shared_out = take(rb[MOE_WS_SHARED_OUT] = Fs ? es * T * d : 0);
   L.x_stage = take(es * T * d);
   L.out_stage = take(es * T * d);
   L.total = off;

@@ -22,19 +22,29 @@ __device__ __forceinline__ int group_of(const int32_t *off, int E, int r) {
 
 struct SimtArgs {
   const int32_t *offsets;
-  int E, rows, d, F, act;
+  int E, rows, rows_cap, d, F, act;
   int w_stride;   // rows between experts in w1 / w2
   const float *x, *w1, *w2, *w3;
   float *h, *y;
+  int *status;
 };
+
+// The group offsets in shared memory, clamped to [0, rows_cap] and made
+// non-decreasing by the first warp (a repair records kDevBadOffsets).
+__device__ __forceinline__ void load_offsets(const SimtArgs &a, int nE, int32_t *off) {
+  __shared__ int32_t unused[kMaxExperts + 1];
+  if (threadIdx.y == 0) {
+    const bool bad = warp_group_offsets(a.offsets, nE, a.rows, a.rows_cap, off, unused, [](int) { return 0; });
+    if (bad && threadIdx.x == 0 && a.status) record_status(a.status, kDevBadOffsets);
+  }
+  __syncthreads();
+}
 
 __global__ void simt_phase1(SimtArgs a) {
   pdl_enter();
   __shared__ int32_t off[kMaxExperts + 1];
   const int nE = a.offsets ? a.E : 1;
-  for (int i = threadIdx.y * blockDim.x + threadIdx.x; i <= nE; i += blockDim.x * blockDim.y)
-    off[i] = a.offsets ? a.offsets[i] : (i == 0 ? 0 : a.rows);
-  __syncthreads();
+  load_offsets(a, nE, off);
   const int c = blockIdx.x * blockDim.x + threadIdx.x;
   const int r = blockIdx.y * blockDim.y + threadIdx.y;
   if (c >= a.F || r >= off[nE]) return;
@@ -59,9 +69,7 @@ __global__ void simt_phase2(SimtArgs a) {
   pdl_enter();
   __shared__ int32_t off[kMaxExperts + 1];
   const int nE = a.offsets ? a.E : 1;
-  for (int i = threadIdx.y * blockDim.x + threadIdx.x; i <= nE; i += blockDim.x * blockDim.y)
-    off[i] = a.offsets ? a.offsets[i] : (i == 0 ? 0 : a.rows);
-  __syncthreads();
+  load_offsets(a, nE, off);
   const int c = blockIdx.x * blockDim.x + threadIdx.x;
   const int r = blockIdx.y * blockDim.y + threadIdx.y;
   if (c >= a.d || r >= off[nE]) return;
@@ -80,6 +88,8 @@ cudaError_t launch_ffn_simt_f32(const FfnArgs &f, cudaStream_t s) {
   a.offsets = f.offsets;
   a.E = f.E;
   a.rows = f.rows;
+  a.rows_cap = f.rows_cap;
+  a.status = f.status;
   a.d = f.d;
   a.F = f.F;
   a.act = f.act;

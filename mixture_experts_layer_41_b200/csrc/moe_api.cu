@@ -3,6 +3,7 @@
 // include/moe.h.
 #include "common.cuh"
 
+#include <atomic>
 #include <math.h>
 #include <stdlib.h>
 #include <stdio.h>
@@ -200,6 +201,9 @@ moe_status do_shared(const moe_config &c, const void *x, const moe_weights *w, v
 
 void moe::set_last_error_text(const char *text) { set_error("%s%s", text); }
 
+static std::atomic<long long> g_launches{0};
+void moe::note_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
+
 extern "C" {
 
 int64_t moe_capacity(int32_t num_tokens, int32_t top_k, int32_t num_experts, float capacity_factor) {
@@ -322,6 +326,8 @@ const char *moe_status_string(moe_status s) {
 
 const char *moe_last_error(void) { return g_last_error; }
 
+int64_t moe_kernel_launches(void) { return g_launches.load(std::memory_order_relaxed); }
+
 moe_status moe_workspace_status(const void *ws, moe_stream_t stream) {
   if (!aligned16(ws)) return MOE_ERR_WORKSPACE;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
@@ -345,6 +351,30 @@ moe_status moe_workspace_status(const void *ws, moe_stream_t stream) {
   snprintf(num, sizeof(num), "%d", code);
   set_error("device status %s: %s", num, what);
   return MOE_ERR_DEVICE;
+}
+
+moe_status moe_workspace_region(const moe_config *cfg, int32_t region, size_t *offset, size_t *bytes) {
+  if (!offset || !bytes) return MOE_ERR_INVALID_ARG;
+  moe_status st = moe_validate(cfg);
+  if (st != MOE_OK) return st;
+  const WsLayout L = ws_layout(*cfg);
+  size_t begin = 0, end = 0;
+  switch (region) {
+    case MOE_WS_OFFSETS: begin = L.offsets; end = L.perm_token; break;
+    case MOE_WS_PERM_TOKEN: begin = L.perm_token; end = L.perm_w; break;
+    case MOE_WS_PERM_W: begin = L.perm_w; end = L.slot_row; break;
+    case MOE_WS_SLOT_ROW: begin = L.slot_row; end = L.topk_ids; break;
+    case MOE_WS_X_PERM: begin = L.x_perm; end = L.h; break;
+    case MOE_WS_H: begin = L.h; end = L.y_perm; break;
+    case MOE_WS_Y_PERM: begin = L.y_perm; end = L.shared_h; break;
+    case MOE_WS_SHARED_H: begin = L.shared_h; end = L.shared_out; break;
+    case MOE_WS_SHARED_OUT: begin = L.shared_out; end = L.x_stage; break;
+    default: return MOE_ERR_INVALID_ARG;
+  }
+  *offset = begin;
+  *bytes = L.region_bytes[region];
+  if (begin + *bytes > end) return MOE_ERR_INVALID_ARG;   // layout and sizes disagree: a library bug
+  return MOE_OK;
 }
 
 moe_status moe_set_phase_events(void *const *events, int32_t count) {

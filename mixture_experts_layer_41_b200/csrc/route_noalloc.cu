@@ -13,8 +13,16 @@
 // it, so calls that overlap on the GPU (two streams, two threads) race and
 // must be serialised by the caller.  Each call writes every entry it later
 // reads, so nothing needs clearing between calls.
+//
+// It always runs the CUDA-core router with whole-row blocks: the split and
+// tensor-core passes of moe_route keep their logits in the workspace, which
+// this call does not have.  Its ids, weights and probability sums therefore
+// agree with moe_route's within the router tolerances (ids on tokens whose
+// selection margin is clear, weights 1e-6 and sums 1e-5 relative), not bit
+// for bit, and large bf16 batches route more slowly than through moe_route.
 #include "common.cuh"
 
+#include <cuda.h>
 #include <mutex>
 #include <stdio.h>
 
@@ -25,27 +33,62 @@ constexpr int kMaxDevices = 64;
 
 // Device-side scratch.  In host code this name is only a handle for the CUDA
 // runtime, never a device address: the address comes from
-// cudaGetSymbolAddress below, once per device.
+// cudaGetSymbolAddress below, once per device and CUDA context.
 static __device__ __align__(256) double g_route_partials[kNoAllocPartials];
 
-std::mutex g_mu;
-void *g_addr[kMaxDevices] = {};
+typedef CUresult (*CtxGetCurrentFn)(CUcontext *);
+typedef CUresult (*CtxGetIdFn)(CUcontext, unsigned long long *);
 
-// Address of this device's copy of the scratch array (looked up on the first
-// call made on each device, with that device current).
+struct CachedAddress {
+  unsigned long long ctx_id;   // the context the address belongs to (0: none yet)
+  void *addr;
+};
+
+std::mutex g_mu;
+CachedAddress g_cache[kMaxDevices] = {};
+
+template <class Fn>
+Fn driver_fn(const char *name) {
+  void *p = nullptr;
+  cudaDriverEntryPointQueryResult q;
+  if (cudaGetDriverEntryPoint(name, &p, cudaEnableDefault, &q) != cudaSuccess || q != cudaDriverEntryPointSuccess)
+    return nullptr;
+  return reinterpret_cast<Fn>(p);
+}
+
+// Unique id of the context current on this thread (0 if there is none yet).
+unsigned long long current_context_id() {
+  static CtxGetCurrentFn get_current = driver_fn<CtxGetCurrentFn>("cuCtxGetCurrent");
+  static CtxGetIdFn get_id = driver_fn<CtxGetIdFn>("cuCtxGetId");
+  CUcontext ctx = nullptr;
+  unsigned long long id = 0;
+  if (!get_current || !get_id || get_current(&ctx) != CUDA_SUCCESS || !ctx) return 0;
+  return get_id(ctx, &id) == CUDA_SUCCESS ? id : 0;
+}
+
+// Address of the scratch array in the current device's context.  Looked up
+// with cudaGetSymbolAddress on the first call in each context and cached per
+// device under the context's unique id, so a context created later (after a
+// cudaDeviceReset, or a different context made current by the caller) gets
+// its own lookup instead of a stale address.
 cudaError_t scratch_address(double **out) {
   int dev = 0;
   cudaError_t err = cudaGetDevice(&dev);
   if (err != cudaSuccess) return err;
   if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
   std::lock_guard<std::mutex> lock(g_mu);
-  if (!g_addr[dev]) {
+  unsigned long long id = current_context_id();
+  if (id == 0 || g_cache[dev].ctx_id != id) {
     void *p = nullptr;
-    err = cudaGetSymbolAddress(&p, g_route_partials);
+    err = cudaGetSymbolAddress(&p, g_route_partials);   // binds the device's context if none was current
     if (err != cudaSuccess) return err;
-    g_addr[dev] = p;
+    if (id == 0) id = current_context_id();
+    g_cache[dev].ctx_id = id;   // 0 (no id available): looked up again on the next call
+    g_cache[dev].addr = p;
+    *out = static_cast<double *>(p);
+    return cudaSuccess;
   }
-  *out = static_cast<double *>(g_addr[dev]);
+  *out = static_cast<double *>(g_cache[dev].addr);
   return cudaSuccess;
 }
 

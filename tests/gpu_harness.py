@@ -2,6 +2,8 @@
 against the oracle on the same seeded inputs (GPU tests only)."""
 from __future__ import annotations
 
+import itertools
+
 import numpy as np
 import torch
 
@@ -14,6 +16,17 @@ from oracle import moe_oracle as O
 WEIGHT_RTOL = 1e-6      # routing weights, relative (spec bound)
 PROB_RTOL = 1e-5        # prob_sum, relative
 AUX_RTOL = 1e-5
+# Tokens whose selection margin is within 1e-4 ("unsafe": their ids may
+# legitimately differ) must stay a small minority, so the bit-exact id check
+# covers nearly every token.  The DeepSeek-V3-style workload has about 1.9 %
+# of such tokens by the score density alone (256 sigmoid scores in a narrow
+# band plus the group cut), so the bound is 3 % of T (at least 3 tokens, for
+# batches of a few dozen).  Unsafe tokens are still checked: their choice
+# must be a correct one within the margin, and their weights exact for it.
+UNSAFE_FRACTION = 0.03
+CANARY = 0xA5           # byte written around and inside buffers that must stay untouched
+GUARD_ROWS = 8          # canary rows after each caller-owned output
+GUARD_BYTES = 1 << 16   # canary bytes after the workspace
 
 
 def out_tol(w: Workload) -> float:
@@ -33,7 +46,10 @@ class Run:
         T, k, E, d = w.T, w.k, w.E, w.d
         dt = torch.float32 if w.dtype == "f32" else torch.bfloat16
         i32 = dict(dtype=torch.int32, device=self.dev)
-        self.ws = torch.empty(api.moe_workspace_size(self.cfg), dtype=torch.uint8, device=self.dev)
+        n_ws = api.moe_workspace_size(self.cfg)
+        # the workspace and every row buffer carry a canary tail that no call may touch
+        self.ws_full = torch.full((n_ws + GUARD_BYTES,), CANARY, dtype=torch.uint8, device=self.dev)
+        self.ws = self.ws_full[:n_ws]
         self.ids = torch.empty((T, k), **i32)
         self.wts = torch.empty((T, k), dtype=torch.float32, device=self.dev)
         self.prob_sum = torch.empty(E, dtype=torch.float32, device=self.dev)
@@ -41,12 +57,25 @@ class Run:
         self.perm_token = torch.empty(T * k, **i32)
         self.perm_w = torch.empty(T * k, dtype=torch.float32, device=self.dev)
         self.slot_row = torch.empty((T, k), **i32)
-        self.x_perm = torch.empty((T * k, d), dtype=dt, device=self.dev)
-        self.y_perm = torch.empty((T * k, d), dtype=dt, device=self.dev)
-        self.shared = torch.empty((T, d), dtype=dt, device=self.dev) if w.shared_F else None
-        self.out = torch.empty((T, d), dtype=dt, device=self.dev)
+        self.guarded = {}
+        self.x_perm = self._guarded("x_perm", T * k, d, dt)
+        self.y_perm = self._guarded("y_perm", T * k, d, dt)
+        self.shared = self._guarded("shared", T, d, dt) if w.shared_F else None
+        self.out = self._guarded("out", T, d, dt)
         self.stats = dict(raw_counts=torch.empty(E, **i32), kept_counts=torch.empty(E, **i32),
                           prob_sum=self.prob_sum, dropped=torch.empty(4, **i32))
+
+    def _guarded(self, name, rows, cols, dt):
+        full = torch.empty((rows + GUARD_ROWS, cols), dtype=dt, device=self.dev)
+        full.view(torch.uint8).fill_(CANARY)
+        self.guarded[name] = (full, rows)
+        return full[:rows]
+
+    def fill_canary(self):
+        """Canary bytes over the whole workspace and every caller row buffer."""
+        self.ws_full.fill_(CANARY)
+        for full, _ in self.guarded.values():
+            full.view(torch.uint8).fill_(CANARY)
 
     def staged(self):
         c = self.cfg
@@ -71,43 +100,148 @@ class Run:
         return api.moe_workspace_status(self.ws)
 
 
-def check_route(run: Run, oracle_r: dict) -> dict:
-    """ids bit-exact and weights within 1e-6 relative on tokens whose margin
-    exceeds 1e-4; prob_sum within 1e-5 relative."""
+def _valid_top(scores: np.ndarray, chosen: np.ndarray, pool: np.ndarray, tol: float) -> bool:
+    """``chosen`` is a top-len(chosen) set of ``pool`` under ``scores`` up to
+    ``tol``, listed in descending order up to ``tol``."""
+    rest = np.setdiff1d(pool, chosen)
+    if np.setdiff1d(chosen, pool).size or len(set(chosen.tolist())) != chosen.size:
+        return False
+    if rest.size and scores[chosen].min() < scores[rest].max() - tol:
+        return False
+    return bool(np.all(scores[chosen[:-1]] >= scores[chosen[1:]] - tol))
+
+
+def valid_choice(w: Workload, oracle_r: dict, t: int, chosen: np.ndarray, bias, tol: float) -> bool:
+    """Whether a router's ids for token t are a correct selection when scores
+    may move by ``tol``: the selection rule of the oracle (top-k of the
+    softmax; or, for sigmoid groups, top groups by top-two sums, then top-k
+    of the selection scores inside them) with near-ties resolved either way."""
+    E = w.E
+    if w.router == "softmax_topk":
+        return _valid_top(oracle_r["probs"][t], chosen, np.arange(E), tol)
+    sel = oracle_r["probs"][t] + (bias if bias is not None else 0.0)
+    gsize = E // w.n_group
+    gscore = np.sort(sel.reshape(w.n_group, gsize), axis=1)[:, -2:].sum(axis=1)
+    used = sorted(set((chosen // gsize).tolist()))
+    if len(used) > w.topk_group:
+        return False
+    others = [g for g in range(w.n_group) if g not in used]
+    for extra in itertools.combinations(others, w.topk_group - len(used)):
+        kept = np.array(used + list(extra))
+        if not _valid_top(gscore, kept[np.argsort(-gscore[kept], kind="stable")], np.arange(w.n_group), tol):
+            continue
+        pool = np.concatenate([np.arange(g * gsize, (g + 1) * gsize) for g in kept])
+        if _valid_top(sel, chosen, pool, tol):
+            return True
+    return False
+
+
+def check_route(run: Run, oracle_r: dict, max_unsafe_fraction: float = UNSAFE_FRACTION) -> dict:
+    """ids bit-exact on tokens whose oracle margin exceeds 1e-4; on the rest a
+    correct choice within that margin; weights within 1e-6 relative of the
+    oracle's weights for the GPU's own choice on every token (and of the
+    oracle's own weights where the ids agree); prob_sum within 1e-5
+    relative; tokens within the margin at most UNSAFE_FRACTION of T."""
+    w = run.w
     ids = run.ids.cpu().numpy()
     wts = run.wts.cpu().numpy().astype(np.float64)
     safe = oracle_r["margin"] > O.SAFE_MARGIN
+    n_unsafe = int((~safe).sum())
+    print(f"[route] {w.name} T={w.T}: {n_unsafe} tokens ({n_unsafe / w.T:.2%}) within the 1e-4 margin")
+    assert n_unsafe <= max(3, max_unsafe_fraction * w.T), f"{n_unsafe} of {w.T} tokens within the margin"
     assert np.array_equal(ids[safe], oracle_r["ids"][safe]), "expert ids differ on safe tokens"
+    bias = to_host(run.inp.get("expert_bias")) if w.router == "sigmoid_group" else None
+    bias = O.widen(bias) if bias is not None else None
+    for t in np.nonzero(~safe)[0]:
+        assert valid_choice(w, oracle_r, int(t), ids[t], bias, O.SAFE_MARGIN), \
+            f"token {t}: ids {ids[t]} are not a valid choice (oracle {oracle_r['ids'][t]})"
     ref_w = oracle_r["weights"][safe]
     err = np.abs(wts[safe] - ref_w) / np.maximum(np.abs(ref_w), 1e-30)
     assert err.size == 0 or err.max() <= WEIGHT_RTOL, f"routing weight rel err {err.max():.3e}"
+    # the weights of the GPU's own choice, every token (router replay in the oracle)
+    rep = O.route_forced(to_host(run.inp["x"]), to_host(run.inp["w_router"]), ids, top_k=w.k, router=w.router,
+                         norm=w.norm_topk_prob, routed_scaling=w.routed_scaling,
+                         logit_bias=to_host(run.inp.get("logit_bias")))
+    assert not rep["bad"].any(), "router returned out-of-range or repeated ids"
+    ferr = np.abs(wts - rep["weights"]) / np.maximum(np.abs(rep["weights"]), 1e-30)
+    assert ferr.max() <= WEIGHT_RTOL, f"routing weight rel err {ferr.max():.3e} for the GPU's own ids"
     ps = run.prob_sum.cpu().numpy().astype(np.float64)
     ref_ps = oracle_r["prob_sum"]
     perr = np.abs(ps - ref_ps) / np.maximum(np.abs(ref_ps), 1e-30)
     assert perr.max() <= PROB_RTOL, f"prob_sum rel err {perr.max():.3e}"
-    return dict(n_unsafe=int((~safe).sum()), weight_err=float(err.max()) if err.size else 0.0,
+    return dict(n_unsafe=n_unsafe, weight_err=float(max(ferr.max(), err.max() if err.size else 0.0)),
                 prob_err=float(perr.max()))
 
 
-def check_dispatch(run: Run) -> dict:
-    """The oracle's dispatch of the GPU's own ids and weights, bit-exact."""
+def _untouched(t: torch.Tensor) -> bool:
+    return bool((t.reshape(-1).view(torch.uint8) == CANARY).all().item())
+
+
+def check_canaries(run: Run, routed_rows: int, staged: bool) -> None:
+    """Nothing written outside what the calls promise: the guard rows after
+    each caller buffer, the guard bytes after the workspace, the rows of the
+    expert-sorted buffers past off[E] (caller's in a staged run, the
+    workspace's own in moe_forward), and the workspace buffers a staged run
+    leaves to the caller.  The buffers must have been filled with the canary
+    (Run.fill_canary) before the calls."""
+    cfg = run.cfg
+    for name, (full, rows) in run.guarded.items():
+        assert _untouched(full[rows:]), f"write past the end of {name}"
+    assert _untouched(run.ws_full[run.ws.numel():]), "write past the end of the workspace"
+    R = routed_rows
+    es = run.x_perm.element_size()
+    regions = {"x_perm": run.w.d, "h": run.w.F, "y_perm": run.w.d}
+    for region, cols in regions.items():
+        off, n = api.moe_workspace_region(cfg, region)
+        if n == 0:
+            continue
+        buf = run.ws[off:off + n].view(-1, cols * es)
+        if staged and region != "h":
+            assert _untouched(buf), f"staged calls wrote into the workspace's {region}"
+        else:
+            assert _untouched(buf[R:]), f"write into {region} rows at or past off[E] = {R}"
+    if staged:
+        assert _untouched(run.x_perm[R:]), "write into caller x_perm rows at or past off[E]"
+        assert _untouched(run.y_perm[R:]), "write into caller y_perm rows at or past off[E]"
+        off, n = api.moe_workspace_region(cfg, "shared_out")
+        assert n == 0 or _untouched(run.ws[off:off + n]), "staged calls wrote the workspace's shared_out"
+
+
+def forward_permutation(run: Run) -> dict:
+    """The permutation moe_forward built, read from its workspace."""
+    c, ws, w = run.cfg, run.ws, run.w
+    view = lambda region, dt, cols=1: api.workspace_view(c, ws, region, dt, cols)
+    return dict(offsets=view("offsets", torch.int32).reshape(-1),
+                perm_token=view("perm_token", torch.int32).reshape(-1),
+                perm_w=view("perm_w", torch.float32).reshape(-1),
+                slot_row=view("slot_row", torch.int32, w.k),
+                x_perm=view("x_perm", run.x_perm.dtype, w.d))
+
+
+def check_dispatch(run: Run, src: dict = None) -> dict:
+    """The oracle's dispatch of the GPU's own ids and weights, bit-exact.
+    ``src`` holds the dispatch outputs to check (default: the staged run's
+    caller buffers; forward_permutation(run) for moe_forward's own)."""
     w = run.w
+    if src is None:
+        src = dict(offsets=run.offsets, perm_token=run.perm_token, perm_w=run.perm_w, slot_row=run.slot_row,
+                   x_perm=run.x_perm)
     ids = run.ids.cpu().numpy()
     wts = run.wts.cpu().numpy()
     cap = O.capacity(w.T, w.k, w.E, float(np.float32(w.capacity_factor)))
     ref = O.dispatch(ids, w.E, cap, wts)
-    off = run.offsets.cpu().numpy()
+    off = src["offsets"].cpu().numpy()
     assert np.array_equal(off, ref["expert_offsets"]), "expert_offsets"
     R = int(off[-1])
-    assert np.array_equal(run.perm_token.cpu().numpy()[:R], ref["perm_token"]), "perm_token"
-    assert np.array_equal(run.perm_w.cpu().numpy()[:R], ref["perm_w"].astype(np.float32)), "perm_w"
-    assert np.array_equal(run.slot_row.cpu().numpy(), ref["slot_row"]), "slot_row / drop set"
+    assert np.array_equal(src["perm_token"].cpu().numpy()[:R], ref["perm_token"]), "perm_token"
+    assert np.array_equal(src["perm_w"].cpu().numpy()[:R], ref["perm_w"].astype(np.float32)), "perm_w"
+    assert np.array_equal(src["slot_row"].cpu().numpy(), ref["slot_row"]), "slot_row / drop set"
     assert np.array_equal(run.stats["raw_counts"].cpu().numpy(), ref["raw_counts"]), "raw_counts"
     assert np.array_equal(run.stats["kept_counts"].cpu().numpy(), ref["kept_counts"]), "kept_counts"
     assert int(run.stats["dropped"][0]) == ref["dropped"], "dropped"
     # the gather: x_perm rows are byte copies of the token rows
-    xp = run.x_perm[:R]
-    xs = run.inp["x"][run.perm_token[:R].long()]
+    xp = src["x_perm"][:R]
+    xs = run.inp["x"][src["perm_token"][:R].long()]
     assert torch.equal(xp.view(torch.int16) if xp.dtype == torch.bfloat16 else xp,
                        xs.view(torch.int16) if xs.dtype == torch.bfloat16 else xs), "x_perm gather"
     return dict(R=R, dropped=ref["dropped"], cap=cap, ref=ref)
@@ -153,16 +287,18 @@ def check_aux(run: Run, oracle_r: dict) -> float:
 
 
 def sample_tokens(run: Run, n: int, seed: int = 0) -> np.ndarray:
-    """A seeded subset of tokens that includes every token with a dropped slot
-    (up to n/2 of them) and tokens of the hottest expert."""
+    """A seeded subset of at least n tokens (all of them when T <= n) that
+    holds every token with a dropped slot and every token of the hottest
+    expert (the one with the most routed slots), topped up with tokens drawn
+    uniformly."""
     rng = np.random.default_rng(seed)
     T = run.w.T
+    if T <= n:
+        return np.arange(T)
     slot = run.slot_row.cpu().numpy()
-    dropped = np.nonzero((slot < 0).any(axis=1))[0]
     ids = run.ids.cpu().numpy()
     hot = np.bincount(ids.reshape(-1), minlength=run.w.E).argmax()
-    hot_toks = np.nonzero((ids == hot).any(axis=1))[0]
-    pick = list(dropped[: n // 2]) + list(hot_toks[: n // 4])
-    rest = rng.choice(T, size=min(T, n), replace=False)
-    pick += [t for t in rest if t not in set(pick)]
-    return np.array(sorted(set(int(t) for t in pick[:n])))
+    must = set(np.nonzero((slot < 0).any(axis=1))[0].tolist()) | set(np.nonzero((ids == hot).any(axis=1))[0].tolist())
+    rest = [int(t) for t in rng.permutation(T) if int(t) not in must]
+    pick = sorted(must) + rest[:max(0, n - len(must))]
+    return np.array(sorted(pick))

@@ -197,3 +197,31 @@ def test_device_calls_reject_bad_arguments_before_any_launch():
     assert api.moe_workspace_size(_cfg(fused_gather=True)) < api.moe_workspace_size(_cfg())
     q4 = dict(weight_dtype="q4_affine_g64")
     assert api.moe_workspace_size(_cfg(fused_gather=True, **q4)) == api.moe_workspace_size(_cfg(**q4))
+
+
+@pytest.mark.parametrize("name", sorted(WORKLOADS))
+def test_workspace_regions(name):
+    """moe_workspace_region: the intermediates moe_forward keeps in the
+    workspace lie inside it, in order, without overlap, 256-byte aligned,
+    with the sizes their shapes give."""
+    from mixture_experts_layer_41_b200.inputs import workload
+    w = workload(name)
+    cfg = cfg_of(w)
+    total = api.moe_workspace_size(cfg)
+    es = 4 if w.dtype == "f32" else 2
+    slots = w.T * w.k
+    expect = dict(offsets=4 * (w.E + 1), perm_token=4 * slots, perm_w=4 * slots, slot_row=4 * slots,
+                  x_perm=es * slots * w.d, h=es * slots * w.F, y_perm=es * slots * w.d,
+                  shared_h=es * w.T * w.shared_F, shared_out=es * w.T * w.d if w.shared_F else 0)
+    end = 0
+    for region in ("offsets", "perm_token", "perm_w", "slot_row", "x_perm", "h", "y_perm", "shared_h",
+                   "shared_out"):
+        off, n = api.moe_workspace_region(cfg, region)
+        assert off % 256 == 0 and off >= end, (region, off, end)
+        assert n == expect[region], (region, n, expect[region])
+        end = off + n
+        assert end <= total
+    with pytest.raises(L.MoEError):
+        off, n = C.c_size_t(), C.c_size_t()
+        L.check(L.lib().moe_workspace_region(C.byref(cfg), L.MOE_WS_REGION_COUNT, C.byref(off), C.byref(n)),
+                "region")

@@ -10,8 +10,8 @@ import numpy as np
 import pytest
 import torch
 
-from gpu_harness import (AUX_RTOL, Run, check_aux, check_dispatch, check_output, check_route,
-                         sample_tokens)
+from gpu_harness import (AUX_RTOL, Run, check_aux, check_canaries, check_dispatch, check_output, check_route,
+                         forward_permutation, sample_tokens)
 from mixture_experts_layer_41_b200 import api
 from mixture_experts_layer_41_b200.inputs import workload
 from moe_cases import oracle_route
@@ -47,11 +47,14 @@ def _cuda():
 @pytest.mark.parametrize("name", sorted(SMALL))
 def test_staged_parity(name):
     w = SMALL[name]
-    run = Run(w, seed=1).staged()
+    run = Run(w, seed=1)
+    run.fill_canary()
+    run.staged()
     assert run.status() == 0
     r = oracle_route(w, run.inp)
     info = check_route(run, r)
-    check_dispatch(run)
+    d = check_dispatch(run)
+    check_canaries(run, d["R"], staged=True)
     check_output(run, routing="gpu")
     if info["n_unsafe"] == 0:
         check_output(run, routing="oracle")
@@ -160,33 +163,30 @@ def test_bad_ids_are_reported_not_faulted():
 
 
 # ---------------------------------------------------------------- full sizes
-FULL = {
-    "mixtral_prefill": 48,
-    "switch_top1": 64,
-    "decode_q4": None,       # small enough for the whole output
-    "deepseek_v3": 12,
-}
+# tokens whose output is compared at full size: at least 1024, including
+# every token with a dropped slot and every token of the hottest expert
+FULL_SAMPLE = 1024
+FULL = ["mixtral_prefill", "switch_top1", "decode_q4", "deepseek_v3"]
 
 
-@pytest.mark.parametrize("name", list(FULL))
+@pytest.mark.parametrize("name", FULL)
 def test_full_size_parity(name):
     """Full-size workloads in the launch configuration the bench times
-    (moe_forward): routing and dispatch over the whole batch, the output on
-    a seeded token sample (all tokens for decode)."""
+    (moe_forward on a canary-filled workspace): routing over the whole batch,
+    the dispatch moe_forward built (read from its workspace) bit for bit, no
+    write outside the promised rows, and the output on a seeded sample of at
+    least 1024 tokens (the whole batch for decode)."""
     w = workload(name)
     run = Run(w, seed=0)
+    run.fill_canary()
     run.forward()
     assert run.status() == 0
     r = oracle_route(w, run.inp)
     check_route(run, r)
-    # moe_forward keeps the permutation in the workspace: recompute it staged
-    api.moe_permute(run.cfg, run.inp["x"], run.ids, run.wts, run.offsets, run.perm_token, run.perm_w,
-                    run.slot_row, run.x_perm, run.stats, run.ws)
-    torch.cuda.synchronize()
-    check_dispatch(run)
-    run.forward()
-    n = FULL[name]
-    toks = None if n is None else sample_tokens(run, n)
+    d = check_dispatch(run, forward_permutation(run))
+    check_canaries(run, d["R"], staged=False)
+    toks = sample_tokens(run, FULL_SAMPLE)
+    print(f"[full] {name}: output checked on {len(toks)} tokens, {d['dropped']} dropped slots")
     check_output(run, tokens=toks, routing="gpu")
     assert check_aux(run, r) <= AUX_RTOL
     del run
@@ -222,6 +222,13 @@ ROUTER_SHAPES = {
 }
 
 
+# The router-shape cases put many experts over short hidden sizes, where the
+# softmax probabilities crowd near 1/E and a 1e-4 gap separates fewer tokens
+# (up to about a quarter at E = 96..128 with d = 192..256); every token inside
+# the margin is still checked for a valid choice and exact weights.
+ROUTER_SHAPE_MAX_UNSAFE = 0.35
+
+
 @pytest.mark.parametrize("name", sorted(ROUTER_SHAPES))
 def test_router_shapes(name):
     w = ROUTER_SHAPES[name]
@@ -229,7 +236,7 @@ def test_router_shapes(name):
     api.moe_route(run.cfg, run.inp["x"], run.inp["w_router"], run.bias, run.ids, run.wts, run.prob_sum, run.ws)
     torch.cuda.synchronize()
     assert run.status() == 0
-    check_route(run, oracle_route(w, run.inp))
+    check_route(run, oracle_route(w, run.inp), max_unsafe_fraction=ROUTER_SHAPE_MAX_UNSAFE)
 
 
 def test_token_sharded_capacity_on_one_gpu():

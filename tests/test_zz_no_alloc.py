@@ -14,7 +14,8 @@ import torch
 from mixture_experts_layer_41_b200 import _lib as L
 from mixture_experts_layer_41_b200 import api
 from mixture_experts_layer_41_b200.inputs import make_inputs, workload
-from moe_cases import cfg_of, router_bias_of
+from moe_cases import cfg_of, oracle_route, router_bias_of
+from oracle import moe_oracle as O
 
 pytestmark = pytest.mark.gpu
 
@@ -25,6 +26,10 @@ PROB_RTOL = 1e-5
 def _route_both(w, seed):
     dev = torch.device("cuda")
     inp = make_inputs(w, seed=seed, device=dev)
+    # the two calls take different router passes (moe_route may use the
+    # tensor-core logits, the no-workspace call never does), so ids are
+    # compared only where the oracle's selection margin is clear
+    safe = oracle_route(w, inp)["margin"] > O.SAFE_MARGIN
     cfg = cfg_of(w)
     bias = router_bias_of(w, inp)
     ws = torch.empty(api.moe_workspace_size(cfg), dtype=torch.uint8, device=dev)
@@ -39,14 +44,18 @@ def _route_both(w, seed):
             api.moe_route_noalloc(cfg, inp["x"], inp["w_router"], bias, ids, wts, ps)
         torch.cuda.synchronize()
         out[name] = (ids.cpu().numpy(), wts.cpu().numpy().astype(np.float64), ps.cpu().numpy().astype(np.float64))
+    out["safe"] = safe
     return out
 
 
 def _compare(out):
     ids_a, w_a, p_a = out["ws"]
     ids_b, w_b, p_b = out["noalloc"]
-    assert np.array_equal(ids_a, ids_b)
-    assert np.all(np.abs(w_b - w_a) <= WEIGHT_RTOL * np.abs(w_a))
+    safe = out["safe"]
+    assert safe.mean() > 0.9
+    assert np.array_equal(ids_a[safe], ids_b[safe])
+    same = safe[:, None] & (ids_a == ids_b)
+    assert np.all(np.abs(w_b - w_a)[same] <= WEIGHT_RTOL * np.abs(w_a)[same])
     assert np.all(np.abs(p_b - p_a) <= PROB_RTOL * np.abs(p_a))
 
 
