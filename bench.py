@@ -42,6 +42,9 @@ def parse_args():
     ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default="deepseek_v3")
+    ap.add_argument("--shape", default="",
+                    help="reduced shape for profiling, e.g. E=32,T=2048 (fields of the workload; the line's "
+                         "config then names the reduced shape)")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -152,9 +155,22 @@ def layer_costs(w, R: int, touched: int) -> dict:
     flops = f1 + f2 + fs + router
     xbytes = w.T * w.d * es
     layer_bytes = w1 + w3 + sbytes + 2 * xbytes + w.E * w.d * 4
-    return dict(flops=flops, bytes=layer_bytes,
-                ffn1=dict(flops=f1, bytes=w1 + R * w.d * es + R * w.F * es),
-                ffn2=dict(flops=f2, bytes=w3 + R * w.F * es + R * w.d * es))
+    ffn1 = dict(flops=f1, bytes=w1 + R * w.d * es + R * w.F * es)
+    ffn2 = dict(flops=f2, bytes=w3 + R * w.F * es + R * w.d * es)
+    if shared_in_gemm(w):
+        # the shared expert is one more group of the same two launches
+        ffn1 = dict(flops=f1 + 4.0 * w.T * w.d * w.shared_F,
+                    bytes=ffn1["bytes"] + 2 * w.d * w.shared_F * es + w.T * w.d * es + w.T * w.shared_F * es)
+        ffn2 = dict(flops=f2 + 2.0 * w.T * w.shared_F * w.d,
+                    bytes=ffn2["bytes"] + w.d * w.shared_F * es + w.T * w.shared_F * es + w.T * w.d * es)
+    return dict(flops=flops, bytes=layer_bytes, ffn1=ffn1, ffn2=ffn2)
+
+
+def shared_in_gemm(w) -> bool:
+    """moe_forward runs a bf16 shared expert of the experts' width inside the
+    grouped GEMM launches (unless the routed GEMM is forced onto SM pairs)."""
+    return (w.shared_F > 0 and w.shared_F == w.F and w.dtype == "bf16" and w.weight_format == "dense"
+            and os.environ.get("MOE_TC_PAIR") != "1")
 
 
 def ffn_kernel_file(w) -> str:
@@ -165,7 +181,7 @@ def ffn_kernel_file(w) -> str:
     if w.weight_format == "q4_affine_g64":
         if w.d % 128 or w.F % 128:
             return "ffn_q4.cu"
-        return "ffn_q4_mma.cu" if w.T * w.k <= 16 * w.E else "ffn_q4_tc.cu"
+        return "ffn_q4_i8.cu" if w.T * w.k <= 16 * w.E else "ffn_q4_tc.cu"
     return "ffn_simt.cu" if w.dtype == "f32" else "ffn_tc.cu"
 
 
@@ -273,7 +289,7 @@ def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return 0
-    w = workload(args.workload)
+    w = workload_of(args)
     inp = make_inputs(w, seed=args.seed, device="cpu")
     n = args.cpu_sample or max(4, auto_sample(w, per_step_s=4.0))
     for _ in range(args.warmup):
@@ -292,6 +308,23 @@ def run_reference(args):
     }
     print(json.dumps(line), flush=True)
     return 0
+
+
+def workload_of(args):
+    """The named workload, with --shape overrides (integers, floats or words)."""
+    from mixture_experts_layer_41_b200.inputs import workload
+    kw = {}
+    for item in filter(None, args.shape.split(",")):
+        key, val = item.split("=", 1)
+        for conv in (int, float):
+            try:
+                val = conv(val)
+                break
+            except ValueError:
+                continue
+        kw[key.strip()] = val
+    w = workload(args.workload, **kw)
+    return w.with_(name=w.name + ("[" + args.shape + "]" if args.shape else ""))
 
 
 def config_of(w, world: int) -> dict:
@@ -356,7 +389,7 @@ def run_ours(args):
         if world > 1:
             dist.barrier()
 
-    w = workload(args.workload)
+    w = workload_of(args)
     inp = make_inputs(w, seed=args.seed + rank, device=dev)
     wf = "q4_affine_g64" if w.weight_format == "q4_affine_g64" else w.dtype
     cfg = api.make_config(num_tokens=w.T, hidden=w.d, intermediate=w.F, num_experts=w.E, top_k=w.k,
@@ -539,7 +572,8 @@ def run_ours(args):
     kernel_file = os.path.join(ROOT, "mixture_experts_layer_41_b200", "csrc", ffn_kernel_file(w))
     roof["traffic"] = recorded_traffic(kernel_file, f"{w.name}:{dom}")
     roof["kernel"] = {"ffn1": "grouped expert GEMM, phase 1 (gate/up or in)",
-                      "ffn2": "grouped expert GEMM, phase 2 (down or out)"}[dom]
+                      "ffn2": "grouped expert GEMM, phase 2 (down or out)"}[dom] + \
+        (" with the shared expert as one more group" if shared_in_gemm(w) else "")
     roof["peak_source"] = f"{peak_src} ({'bf16 GEMM, burst' if roof['bound'] == 'tensor' else 'HBM copy'})"
     roof["algorithmic"] = {"flop_per_launch": dk["flops"], "bytes_per_launch": dk["bytes"],
                            "ms_per_launch": phases[dom]}

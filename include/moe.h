@@ -202,6 +202,18 @@ const char *moe_last_error(void);
  * across one call is that call's launch count. */
 int64_t moe_kernel_launches(void);
 
+/* Bound on every on-chip barrier wait of the tensor-core kernels (grouped
+ * GEMMs, the tensor-core router logits), in nanoseconds of the GPU's global
+ * timer, for the launches that follow (process-wide, all threads).  When a
+ * wait runs out, the kernel records where in the workspace status word
+ * (moe_workspace_status: MOE_ERR_DEVICE, "... wait timed out"), lets the
+ * copies and tensor-core work it already issued finish (waiting at most
+ * 200 ms for them), frees its tensor memory and returns, leaving the CUDA
+ * context usable; that call's outputs are then incomplete.  0 restores the
+ * default of 2 s, far above any wait of a healthy launch.  A short limit
+ * makes a launch fail on purpose, which is how the failure path is tested. */
+moe_status moe_set_wait_timeout_ns(uint64_t ns);
+
 /* Synchronises `stream` and reads the device status word a kernel leaves in
  * `ws` (MOE_OK, or MOE_ERR_DEVICE with the site in moe_last_error()). */
 moe_status moe_workspace_status(const void *ws, moe_stream_t stream);
@@ -360,24 +372,41 @@ moe_status moe_permute(const moe_config *cfg, const void *x, const int32_t *topk
 /* Token-sharded dispatch with the in-order capacity rule of the whole batch
  * (blog moe_layer: capacity is "per BATCH"; its in-order cut then spans the
  * token shards held by different GPUs).  A batch split into contiguous token
- * shards keeps, on the shard of rank r, a slot of expert e iff
- * shard_base[e] + (its rank among this shard's slots of e) < capacity, where
- * shard_base[e] is the number of slots of e on the earlier shards -- the one
- * exchange the sharded layer needs (an all-gather of moe_expert_counts).
+ * shards, shard r on rank r, keeps on rank r a slot of expert e iff
+ *   (slots of e on shards 0..r-1) + (its rank among this shard's slots of e) < capacity.
+ * The slot counts of every shard are the one exchange the sharded layer
+ * needs: each rank runs moe_expert_counts on its shard and the ranks
+ * all-gather the results into counts_by_rank.
  *
  * moe_expert_counts: raw per-expert slot counts of this shard's topk_ids
  *   (the histogram of the dispatch, no capacity, no gather).  Out: raw_counts
  *   [E] int32 (device).  Uses ws.
  * moe_permute_shard: moe_permute with capacity = the WHOLE batch's capacity
- *   (moe_capacity(T_total, ...), -1 for none) and shard_base [E] int32
- *   (device, NULL = first shard); cfg->num_tokens is this shard's token count.
- *   Same outputs as moe_permute.  Uses ws. */
+ *   (moe_capacity(T_total, ...), -1 for none) and counts_by_rank [world, E]
+ *   int32 (device; row q = the moe_expert_counts of shard q; may be NULL
+ *   when world == 1 or rank == 0); 0 <= rank < world, else
+ *   MOE_ERR_INVALID_ARG.  cfg->num_tokens is this shard's token count.  The
+ *   library forms the prefix over the earlier ranks itself.  Same outputs
+ *   as moe_permute.  Uses ws. */
 moe_status moe_expert_counts(const moe_config *cfg, const int32_t *topk_ids, int32_t *raw_counts, void *ws,
                              size_t ws_bytes, moe_stream_t stream);
 moe_status moe_permute_shard(const moe_config *cfg, const void *x, const int32_t *topk_ids, const float *topk_w,
-                             const int32_t *shard_base, int64_t capacity, int32_t *expert_offsets,
-                             int32_t *perm_token, float *perm_w, int32_t *slot_row, void *x_perm,
-                             const moe_stats *stats, void *ws, size_t ws_bytes, moe_stream_t stream);
+                             const int32_t *counts_by_rank, int32_t world, int32_t rank, int64_t capacity,
+                             int32_t *expert_offsets, int32_t *perm_token, float *perm_w, int32_t *slot_row,
+                             void *x_perm, const moe_stats *stats, void *ws, size_t ws_bytes, moe_stream_t stream);
+
+/* Expert parallelism ("Mixture-of-Experts" design doc, The pipeline: the
+ * expert-parallel dispatch): rank r of `world` holds experts
+ * [r*experts_per_rank, (r+1)*experts_per_rank).  After the all-to-all of
+ * rows, the received rows are grouped by source rank and, inside a source,
+ * by local expert, with recv_counts[s][e] rows of local expert e from rank s
+ * (recv_counts [world, experts_per_rank] int32, device).  This writes the
+ * local expert id of each of the `rows` received rows into ids [rows] int32
+ * (device), in arrival order, ready for moe_permute with top_k = 1; rows
+ * past the sum of the counts get -1, which moe_permute rejects.
+ * world * experts_per_rank <= 256.  Stream-ordered, no workspace. */
+moe_status moe_ep_local_ids(const int32_t *recv_counts, int32_t world, int32_t experts_per_rank, int32_t rows,
+                            int32_t *ids, moe_stream_t stream);
 
 /* Grouped expert FFN over the ragged groups (design doc: one grouped matmul
  * over the per-expert token groups; blog moe_forward: two GEMMs per expert
@@ -411,6 +440,10 @@ moe_status moe_combine(const moe_config *cfg, const void *y_perm, const int32_t 
                        moe_stream_t stream);
 
 /* The whole layer: route, permute, grouped FFN, shared expert, combine.
+ * With bf16 weights and a shared expert as wide as the routed ones
+ * (shared_intermediate == intermediate), the shared expert runs as one more
+ * group of the grouped FFN's two launches (the same results, bit for bit, as
+ * moe_shared_expert); otherwise it is a launch of its own.
  * topk_ids / topk_w (outputs, [T,k]) and stats may be NULL (kept in ws).
  * Out: out [T,d] act_dtype.  Uses ws. */
 moe_status moe_forward(const moe_config *cfg, const void *x, const float *w_router,

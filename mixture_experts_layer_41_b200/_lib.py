@@ -91,6 +91,7 @@ SIGNATURES = {
     "moe_status_string": (C.c_char_p, [C.c_int]),
     "moe_last_error": (C.c_char_p, []),
     "moe_kernel_launches": (C.c_int64, []),
+    "moe_set_wait_timeout_ns": (C.c_int, [C.c_uint64]),
     "moe_workspace_status": (C.c_int, [_P, _P]),
     "moe_set_phase_events": (C.c_int, [C.POINTER(C.c_void_p), C.c_int32]),
     "moe_workspace_region": (C.c_int, [_CFG, C.c_int32, C.POINTER(C.c_size_t), C.POINTER(C.c_size_t)]),
@@ -100,7 +101,9 @@ SIGNATURES = {
     "moe_update_bias": (C.c_int, [_CFG, _P, _P, C.c_float, _P]),
     "moe_permute": (C.c_int, [_CFG, _P, _P, _P, _P, _P, _P, _P, _P, _S, _P, C.c_size_t, _P]),
     "moe_expert_counts": (C.c_int, [_CFG, _P, _P, _P, C.c_size_t, _P]),
-    "moe_permute_shard": (C.c_int, [_CFG, _P, _P, _P, _P, C.c_int64, _P, _P, _P, _P, _P, _S, _P, C.c_size_t, _P]),
+    "moe_permute_shard": (C.c_int, [_CFG, _P, _P, _P, _P, C.c_int32, C.c_int32, C.c_int64, _P, _P, _P, _P, _P, _S,
+                                    _P, C.c_size_t, _P]),
+    "moe_ep_local_ids": (C.c_int, [_P, C.c_int32, C.c_int32, C.c_int32, _P, _P]),
     "moe_grouped_ffn": (C.c_int, [_CFG, _P, _P, _W, _P, _P, C.c_size_t, _P]),
     "moe_shared_expert": (C.c_int, [_CFG, _P, _W, _P, _P, C.c_size_t, _P]),
     "moe_combine": (C.c_int, [_CFG, _P, _P, _P, _P, _P, _P]),

@@ -90,6 +90,11 @@ def moe_kernel_launches() -> int:
     return L.lib().moe_kernel_launches()
 
 
+def moe_set_wait_timeout_ns(ns: int) -> None:
+    """Bound on the tensor-core kernels' barrier waits (0: the 2 s default)."""
+    check(L.lib().moe_set_wait_timeout_ns(int(ns)), "moe_set_wait_timeout_ns")
+
+
 def moe_status_string(status: int) -> str:
     return L.lib().moe_status_string(status).decode()
 
@@ -184,33 +189,37 @@ def moe_expert_counts(cfg, topk_ids, raw_counts, ws, stream=None):
                                     _s(stream)), "moe_expert_counts")
 
 
-def moe_permute_shard(cfg, x, topk_ids, topk_w, shard_base, capacity, expert_offsets, perm_token, perm_w,
-                      slot_row, x_perm, stats, ws, stream=None):
+def moe_permute_shard(cfg, x, topk_ids, topk_w, counts_by_rank, rank, capacity, expert_offsets, perm_token,
+                      perm_w, slot_row, x_perm, stats, ws, stream=None):
+    """``counts_by_rank``: [world, E] int32 device tensor of every shard's
+    moe_expert_counts (``exchange_counts``), or None for a single shard."""
     st = _stats_struct(stats)
-    check(L.lib().moe_permute_shard(C.byref(cfg), _p(x), _p(topk_ids), _p(topk_w), _p(shard_base), int(capacity),
-                                    _p(expert_offsets), _p(perm_token), _p(perm_w), _p(slot_row), _p(x_perm),
-                                    C.byref(st) if st is not None else None, _p(ws), _nbytes(ws), _s(stream)),
+    world = 1 if counts_by_rank is None else int(counts_by_rank.shape[0])
+    check(L.lib().moe_permute_shard(C.byref(cfg), _p(x), _p(topk_ids), _p(topk_w), _p(counts_by_rank), world,
+                                    int(rank), int(capacity), _p(expert_offsets), _p(perm_token), _p(perm_w),
+                                    _p(slot_row), _p(x_perm), C.byref(st) if st is not None else None, _p(ws),
+                                    _nbytes(ws), _s(stream)),
           "moe_permute_shard")
 
 
-def shard_base_from_counts(counts_by_rank: torch.Tensor, rank: int) -> torch.Tensor:
-    """Slots of each expert on the shards before ``rank``: the exclusive
-    prefix over ranks of the gathered [world, E] raw counts."""
-    if rank == 0:
-        return torch.zeros_like(counts_by_rank[0])
-    return counts_by_rank[:rank].sum(dim=0).to(counts_by_rank.dtype)
-
-
-def exchange_shard_base(raw_counts: torch.Tensor, group=None) -> torch.Tensor:
+def exchange_counts(raw_counts: torch.Tensor, group=None) -> torch.Tensor:
     """The sharded layer's one exchange: all-gather every rank's per-expert
-    raw counts (an E-int32 message per rank) and return this rank's
-    shard_base.  Token shards must be contiguous and in rank order."""
+    raw counts (an E-int32 message per rank) into a [world, E] tensor on the
+    same device.  Token shards must be contiguous and in rank order."""
     import torch.distributed as dist
     world = dist.get_world_size(group)
-    rank = dist.get_rank(group)
-    gathered = [torch.empty_like(raw_counts) for _ in range(world)]
-    dist.all_gather(gathered, raw_counts.contiguous(), group=group)
-    return shard_base_from_counts(torch.stack(gathered), rank)
+    n = raw_counts.numel()
+    gathered = torch.empty(world * n, dtype=raw_counts.dtype, device=raw_counts.device)
+    dist.all_gather_into_tensor(gathered, raw_counts.reshape(-1).contiguous(), group=group)
+    return gathered.view(world, n)
+
+
+def moe_ep_local_ids(recv_counts, rows: int, ids, stream=None):
+    """Local expert id of each received row (arrival order) from the
+    [world, experts_per_rank] received counts."""
+    world, e_local = recv_counts.shape
+    check(L.lib().moe_ep_local_ids(_p(recv_counts), int(world), int(e_local), int(rows), _p(ids), _s(stream)),
+          "moe_ep_local_ids")
 
 
 def moe_grouped_ffn(cfg, x_perm, expert_offsets, weights: dict, y_perm, ws, stream=None):

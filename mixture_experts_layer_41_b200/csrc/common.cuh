@@ -53,6 +53,9 @@ __device__ __forceinline__ void pdl_enter() {
 
 // Counts every kernel this library launches (moe_kernel_launches).
 void note_launch();
+// Bound on every barrier wait of the tensor-core kernels, in ns of
+// %globaltimer (moe_set_wait_timeout_ns; 2 s by default).
+uint64_t wait_timeout_ns();
 
 template <typename... KArgs, typename... Args>
 inline cudaError_t launch_kernel(bool pdl, void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
@@ -138,6 +141,7 @@ __device__ __forceinline__ bool warp_group_offsets(const int32_t *src, int n, in
 }
 
 size_t route_logits_bytes(const moe_config &c);   // defined in router.cu
+size_t q4_i8_token_bytes(int rows, int d, int F);   // defined in ffn_q4_i8.cu
 
 // ---------------------------------------------------------------- workspace
 struct WsLayout {
@@ -164,6 +168,7 @@ struct WsLayout {
   size_t shared_out;   // act[T][d]
   size_t x_stage;      // act[T][d]   (moe_forward_host)
   size_t out_stage;    // act[T][d]
+  size_t q4_tokens;    // quantised token rows of the 4-bit integer-MMA path
   size_t total;
   size_t region_bytes[MOE_WS_REGION_COUNT];   // unpadded sizes of the moe_ws_region buffers
 };
@@ -225,6 +230,7 @@ inline WsLayout ws_layout(const moe_config &c) {
   L.shared_out = take(rb[MOE_WS_SHARED_OUT] = Fs ? es * T * d : 0);
   L.x_stage = take(es * T * d);
   L.out_stage = take(es * T * d);
+  L.q4_tokens = take(c.weight_dtype == MOE_Q4_AFFINE_G64 ? q4_i8_token_bytes((int)slots, (int)d, (int)F) : 0);
   L.total = off;
   return L;
 }
@@ -280,7 +286,11 @@ cudaError_t launch_permute(const moe_config &c, const void *x, const int32_t *to
                            int32_t *perm_token, float *perm_w, int32_t *slot_row, void *x_perm,
                            int32_t *raw_counts, int32_t *kept_counts, int32_t *dropped,
                            int32_t *blk_counts, int32_t *blk_base, int32_t *local_rank,
-                           int *status, cudaStream_t s, const int32_t *shard_base = nullptr);
+                           int *status, cudaStream_t s, const int32_t *counts_by_rank = nullptr,
+                           int rank = 0);
+// Expert parallelism: local expert id of each received row ([world][e_local] counts, device).
+cudaError_t launch_ep_local_ids(const int32_t *recv_counts, int world, int e_local, int rows, int32_t *ids,
+                                cudaStream_t s);
 
 // Two-phase expert FFN over groups.  `offsets` == nullptr means one group of
 // `rows` rows (the shared expert).  Writes the intermediate to `h` and the
@@ -304,6 +314,18 @@ struct FfnArgs {
   void *y;                  // [rows_cap, d]
   int *status;
   cudaEvent_t mid_event;    // recorded between the two phases when not null
+  // bf16 tensor-core path only: the shared expert as one more group of both
+  // phases (0 rows: none).  Its width must equal F.
+  int shared_rows;
+  const void *shared_x;     // [shared_rows, d]
+  const void *shared_w1, *shared_w2, *shared_w3;   // [F, d], [F, d], [d, F]
+  void *shared_h;           // [shared_rows, F]
+  void *shared_y;           // [shared_rows, d]
+  // 4-bit integer-MMA path: workspace for the quantised token rows
+  // (q4_i8_token_bytes), and the views of it the launches share
+  void *q4_scratch;
+  const void *q4_tokens;
+  const float *q4_tscale, *q4_tsum;
 };
 
 cudaError_t launch_ffn_simt_f32(const FfnArgs &a, cudaStream_t s);
@@ -314,6 +336,9 @@ bool q4_tc_supported(int d, int F);                                 // the tenso
 cudaError_t launch_ffn_q4_tc(const FfnArgs &a, cudaStream_t s);
 bool q4_mma_supported(int d, int F);                                // the warp-level 4-bit path's shapes
 cudaError_t launch_ffn_q4_mma(const FfnArgs &a, cudaStream_t s);
+bool q4_i8_supported(int d, int F);                                 // the 8-bit integer MMA path's shapes
+size_t q4_i8_token_bytes(int rows, int d, int F);                   // its workspace
+cudaError_t launch_ffn_q4_i8(const FfnArgs &a, cudaStream_t s);
 
 // Replaces the text moe_last_error() returns on this thread.
 void set_last_error_text(const char *text);

@@ -37,7 +37,7 @@
 // (what the nibble extraction yields without byte permutes): phase 1
 // reorders its token tile in shared memory, and writes h already in that
 // order for phase 2.  Sums over K do not depend on the order.
-// Every mbarrier wait is bounded (2 s of %globaltimer) as in the bf16
+// Every mbarrier wait is bounded by %globaltimer (2 s unless moe_set_wait_timeout_ns says otherwise) as in the bf16
 // grouped GEMM: on expiry the CTA records a status, drains its own TMA/MMA
 // work, frees TMEM and exits.
 #include "common.cuh"
@@ -56,7 +56,6 @@ constexpr int EPI_WARPS = 4;            // one per TMEM lane quarter
 constexpr int THREADS = 32 * (2 + DQ_WARPS + EPI_WARPS);
 constexpr int CODE_BYTES = BM * BK / 2; // 4 KiB of codes per matrix per K-block
 constexpr int B_BYTES = NT * BK * 2;    // 4 KiB token tile per K-block
-constexpr uint64_t TIMEOUT_NS = 2000000000ull;
 constexpr uint64_t DRAIN_NS = 200000000ull;
 
 // kind::f16: D fp32, A/B bf16, K-major, N = 32, M = 128
@@ -76,6 +75,7 @@ struct Q4Shape {
 };
 
 struct Q4Params {
+  uint64_t timeout_ns;        // bound on every barrier wait (moe_set_wait_timeout_ns)
   const int32_t *offsets;   // [E+1]
   int E;
   int rows_cap;
@@ -128,14 +128,15 @@ __device__ __forceinline__ uint64_t global_ns() {
   asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
   return t;
 }
-__device__ __forceinline__ bool wait_bounded(uint64_t *bar, uint32_t parity, volatile int *abort_flag, int *status,
-                                             int code) {
+__device__ __forceinline__ bool wait_bounded(uint64_t *bar, uint32_t parity, volatile int *abort_flag,
+                                             int *status, int code, uint64_t limit_ns) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_ns();
   uint32_t spins = 0;
   while (!mbar_try_wait(bar, parity)) {
     if (*abort_flag) return false;
-    if ((++spins & 31u) == 0 && global_ns() - t0 > TIMEOUT_NS) {
+    // the clock is read every 32 polls, or every poll under a limit below 1 us
+    if (((++spins & 31u) == 0 || limit_ns < 1000u) && global_ns() - t0 > limit_ns) {
       *abort_flag = 1;
       record_status(status, code);
       return false;
@@ -351,7 +352,7 @@ q4_tc_gemm(const __grid_constant__ CUtensorMap mapC0, const __grid_constant__ CU
         const int wrow = ti.e * p.w_stride + ti.m * BM;           // first weight row of the tile
         // scale / bias rows of the tile: contiguous BM * kgroups bf16 per tensor
         const uint32_t sb = tc & 1u;
-        if (!wait_bounded(&st->sc_empty[sb], ((tc >> 1) & 1u) ^ 1u, abort_flag, p.status, kDevTimeoutProducer)) {
+        if (!wait_bounded(&st->sc_empty[sb], ((tc >> 1) & 1u) ^ 1u, abort_flag, p.status, kDevTimeoutProducer, p.timeout_ns)) {
           ok = false;
           break;
         }
@@ -367,7 +368,7 @@ q4_tc_gemm(const __grid_constant__ CUtensorMap mapC0, const __grid_constant__ CU
         for (int kb = 0; kb < kb_n; ++kb, ++it) {
           const int s = it % STAGES;
           const uint32_t ph = (it / STAGES) & 1u;
-          if (!wait_bounded(&st->empty[s], ph ^ 1u, abort_flag, p.status, kDevTimeoutProducer)) {
+          if (!wait_bounded(&st->empty[s], ph ^ 1u, abort_flag, p.status, kDevTimeoutProducer, p.timeout_ns)) {
             ok = false;
             break;
           }
@@ -398,7 +399,7 @@ q4_tc_gemm(const __grid_constant__ CUtensorMap mapC0, const __grid_constant__ CU
       for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x, ++tcount) {
         // accumulator buffer tcount % 2: the epilogue of two tiles ago must be done with it
         const uint32_t abuf = tcount & 1u;
-        if (!wait_bounded(&st->acc_empty[abuf], ((tcount >> 1) & 1u) ^ 1u, abort_flag, p.status, kDevTimeoutMma)) {
+        if (!wait_bounded(&st->acc_empty[abuf], ((tcount >> 1) & 1u) ^ 1u, abort_flag, p.status, kDevTimeoutMma, p.timeout_ns)) {
           ok = false;
           break;
         }
@@ -406,7 +407,7 @@ q4_tc_gemm(const __grid_constant__ CUtensorMap mapC0, const __grid_constant__ CU
         const uint32_t dcol = tmem_base + abuf * S::ACC_COLS;
         for (int kb = 0; kb < kb_n; ++kb, ++it) {
           const uint32_t j = it % SLOTS, use = it / SLOTS;
-          if (!wait_bounded(&st->a_full[j], use & 1u, abort_flag, p.status, kDevTimeoutMma)) {
+          if (!wait_bounded(&st->a_full[j], use & 1u, abort_flag, p.status, kDevTimeoutMma, p.timeout_ns)) {
             ok = false;
             break;
           }
@@ -447,7 +448,7 @@ q4_tc_gemm(const __grid_constant__ CUtensorMap mapC0, const __grid_constant__ CU
     for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x, ++tc) {
       const Tile ti = decode_tile(st, nE, m_tiles, tile);
       const uint32_t sb = tc & 1u;
-      if (!wait_bounded(&st->sc_full[sb], (tc >> 1) & 1u, abort_flag, p.status, kDevTimeoutEpilogue)) {
+      if (!wait_bounded(&st->sc_full[sb], (tc >> 1) & 1u, abort_flag, p.status, kDevTimeoutEpilogue, p.timeout_ns)) {
         ok = false;
         break;
       }
@@ -460,7 +461,7 @@ q4_tc_gemm(const __grid_constant__ CUtensorMap mapC0, const __grid_constant__ CU
         const int s = (int)(it % STAGES);
         const uint32_t ph = (it / STAGES) & 1u;
         const uint32_t j = it % SLOTS, use = it / SLOTS;
-        if (!wait_bounded(&st->full[s], ph, abort_flag, p.status, kDevTimeoutEpilogue)) {
+        if (!wait_bounded(&st->full[s], ph, abort_flag, p.status, kDevTimeoutEpilogue, p.timeout_ns)) {
           ok = false;
           break;
         }
@@ -487,7 +488,7 @@ q4_tc_gemm(const __grid_constant__ CUtensorMap mapC0, const __grid_constant__ CU
           const uint4 d = dequant8(wv[w], s2, b2);
           av[4 * w] = d.x; av[4 * w + 1] = d.y; av[4 * w + 2] = d.z; av[4 * w + 3] = d.w;
         }
-        if (!wait_bounded(&st->a_empty[j], (use & 1u) ^ 1u, abort_flag, p.status, kDevTimeoutEpilogue)) {
+        if (!wait_bounded(&st->a_empty[j], (use & 1u) ^ 1u, abort_flag, p.status, kDevTimeoutEpilogue, p.timeout_ns)) {
           ok = false;
           break;
         }
@@ -516,7 +517,7 @@ q4_tc_gemm(const __grid_constant__ CUtensorMap mapC0, const __grid_constant__ CU
     for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++tc) {
       const Tile ti = decode_tile(st, nE, m_tiles, tile);
       const uint32_t abuf = tc & 1u;
-      if (!wait_bounded(&st->acc_full[abuf], (tc >> 1) & 1u, abort_flag, p.status, kDevTimeoutEpilogue)) break;
+      if (!wait_bounded(&st->acc_full[abuf], (tc >> 1) & 1u, abort_flag, p.status, kDevTimeoutEpilogue, p.timeout_ns)) break;
       tc_fence_after();
       const uint32_t ta = tmem_base + ((uint32_t)(q * 32) << 16) + abuf * S::ACC_COLS;
       const int f = ti.m * BM + row;
@@ -649,6 +650,7 @@ cudaError_t run(const FfnArgs &a, const void *tokens, int K, int N, int w_stride
   p.bi[1] = static_cast<const uint16_t *>(PAIR ? b1 : b0);
   p.out = static_cast<uint16_t *>(out);
   p.status = a.status;
+  p.timeout_ns = wait_timeout_ns();
   const size_t smem = smem_bytes<PAIR>(p.kgroups);
   auto kern = q4_tc_gemm<PAIR>;
   err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);

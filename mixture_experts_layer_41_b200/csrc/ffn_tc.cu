@@ -21,10 +21,17 @@
 //               halves of the B tile), bf16 pack, row-masked 16-byte stores.
 // Tiles run expert by expert, n-tile-major with the m-tiles of an expert
 // innermost, so the CTAs in flight share B (weight) tiles through L2.
+// Optionally one more group follows the experts: the shared expert ("Shared
+// expert" of the MoE documentation: applied to every token with weight 1),
+// whose A rows are the token matrix itself (phase 1) or its own intermediate
+// (phase 2), with its own weights and output; its tiles run m-tile-major with
+// the n-tiles innermost, so each 128-token tile of A is read once from HBM
+// while its weights stay in L2.  The shared expert then costs no launch and
+// no tail of its own.
 // A tile's rows past its expert's end belong to the next expert (or are
 // zero-filled by TMA past the buffer); their results are never stored.
 //
-// Every mbarrier wait is bounded (2 s of %globaltimer): on expiry the thread
+// Every mbarrier wait is bounded by %globaltimer (2 s unless moe_set_wait_timeout_ns says otherwise): on expiry the thread
 // records a status code in the workspace, raises a CTA-wide abort flag, waits
 // (bounded) for its own in-flight copies or MMAs and the CTA frees its TMEM
 // and exits.
@@ -45,7 +52,6 @@ constexpr int BH_BYTES = 128 * BK * 2;        // 16 KiB per B half
 constexpr int STAGE_BYTES = A_BYTES + 2 * BH_BYTES;
 constexpr int THREADS = 192;
 constexpr uint32_t TMEM_COLS = 512;
-constexpr uint64_t TIMEOUT_NS = 2000000000ull;
 constexpr uint64_t DRAIN_NS = 200000000ull;
 
 // kind::f16 instruction descriptor: D fp32, A and B bf16, both K-major,
@@ -56,6 +62,7 @@ constexpr uint32_t IDESC = (1u << 4) | (1u << 7) | (1u << 10) |
 enum Mode { MODE_PLAIN = 0, MODE_RELU = 1, MODE_SWIGLU = 2 };
 
 struct TcParams {
+  uint64_t timeout_ns;        // bound on every barrier wait (moe_set_wait_timeout_ns)
   const int32_t *offsets;   // [E+1] or nullptr (one group of `rows`)
   int E;
   int rows;
@@ -69,6 +76,8 @@ struct TcParams {
   int *status;
   const int32_t *gather;    // A row r is token gather[r] of the token matrix (mapA over [T, K], one-row box),
                             // or nullptr: A row r is row r of mapA
+  int shared_rows;          // rows of the shared-expert group (0: none); A from mapA2, B from mapS0 / mapS1
+  __nv_bfloat16 *out2;      // its output [shared_rows, N]
 };
 
 struct SharedState {
@@ -80,7 +89,7 @@ struct SharedState {
   uint32_t tmem_base;
   int abort_flag;
   int32_t off[kMaxExperts + 1];
-  int32_t tile_start[kMaxExperts + 1];
+  int32_t tile_start[kMaxExperts + 2];   // [nE + 1]: start of the shared-expert group's tiles
 };
 
 constexpr size_t SMEM_BYTES = (size_t)STAGES * STAGE_BYTES + sizeof(SharedState) + 1024;
@@ -117,15 +126,16 @@ __device__ __forceinline__ uint64_t global_ns() {
 }
 
 // Wait for the phase of `bar` with the given parity.  Returns false when the
-// CTA is aborting or after TIMEOUT_NS (then the abort flag and `code` are set).
+// CTA is aborting or after limit_ns (then the abort flag and `code` are set).
 __device__ __forceinline__ bool wait_bounded(uint64_t *bar, uint32_t parity, volatile int *abort_flag,
-                                             int *status, int code) {
+                                             int *status, int code, uint64_t limit_ns) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_ns();
   uint32_t spins = 0;
   while (!mbar_try_wait(bar, parity)) {
     if (*abort_flag) return false;
-    if ((++spins & 31u) == 0 && global_ns() - t0 > TIMEOUT_NS) {
+    // the clock is read every 32 polls, or every poll under a limit below 1 us
+    if (((++spins & 31u) == 0 || limit_ns < 1000u) && global_ns() - t0 > limit_ns) {
       *abort_flag = 1;
       record_status(status, code);
       return false;
@@ -207,31 +217,59 @@ __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.
 // ---------------------------------------------------------------- scheduling
 struct TileInfo {
   int e, row0, rows, n;
+  bool shared;   // a tile of the shared-expert group (e == nE)
 };
 
-__device__ __forceinline__ TileInfo decode_tile(const SharedState *st, int nE, int n_tiles, int tile) {
+__device__ __forceinline__ TileInfo decode_tile(const SharedState *st, int nE, int n_tiles, int shared_rows,
+                                                int tile) {
+  TileInfo ti;
+  if (tile >= st->tile_start[nE]) {
+    // shared-expert group: m-tile-major, n-tiles innermost
+    const int local = tile - st->tile_start[nE];
+    ti.e = nE;
+    ti.shared = true;
+    ti.n = local % n_tiles;
+    ti.row0 = (local / n_tiles) * BM;
+    ti.rows = min(BM, shared_rows - ti.row0);
+    return ti;
+  }
   int lo = 0, hi = nE;   // largest e with tile_start[e] <= tile; tile_start[nE] > tile
   while (hi - lo > 1) {
     const int mid = (lo + hi) >> 1;
     if (st->tile_start[mid] <= tile) lo = mid; else hi = mid;
   }
-  TileInfo ti;
   ti.e = lo;
+  ti.shared = false;
   const int local = tile - st->tile_start[lo];
   const int cnt = st->off[lo + 1] - st->off[lo];
   const int mt = (cnt + BM - 1) / BM;
   ti.n = local / mt;
   ti.row0 = st->off[lo] + (local % mt) * BM;
   ti.rows = min(BM, st->off[lo + 1] - ti.row0);
-  (void)n_tiles;
   return ti;
+}
+
+// B rows of a tile's two 128-row halves: SwiGLU takes the same 128 features
+// of the gate (map 0) and up (map 1) weights; otherwise 256 consecutive rows
+// of one weight.  The shared expert's weights start at row 0 of their maps.
+__device__ __forceinline__ void b_rows(const TcParams &p, const TileInfo &ti, int &b0, int &b1) {
+  const int base = ti.shared ? 0 : ti.e * p.b_stride;
+  if (p.mode == MODE_SWIGLU) {
+    b0 = base + ti.n * 128;
+    b1 = b0;
+  } else {
+    b0 = base + ti.n * BN;
+    b1 = b0 + 128;
+  }
 }
 
 __device__ __forceinline__ float silu_f(float g) { return g / (1.f + __expf(-g)); }
 
 __global__ void __launch_bounds__(THREADS, 1)
 tc_grouped_gemm(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CUtensorMap mapB0,
-                const __grid_constant__ CUtensorMap mapB1, const TcParams p) {
+                const __grid_constant__ CUtensorMap mapB1, const __grid_constant__ CUtensorMap mapA2,
+                const __grid_constant__ CUtensorMap mapS0, const __grid_constant__ CUtensorMap mapS1,
+                const TcParams p) {
   pdl_wait();
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   const uint32_t pad = (1024u - (smem_u32(smem_raw) & 1023u)) & 1023u;
@@ -258,6 +296,11 @@ tc_grouped_gemm(const __grid_constant__ CUtensorMap mapA, const __grid_constant_
     asm volatile("prefetch.tensormap [%0];" ::"l"((uint64_t)&mapA) : "memory");
     asm volatile("prefetch.tensormap [%0];" ::"l"((uint64_t)&mapB0) : "memory");
     asm volatile("prefetch.tensormap [%0];" ::"l"((uint64_t)&mapB1) : "memory");
+    if (p.shared_rows > 0) {
+      asm volatile("prefetch.tensormap [%0];" ::"l"((uint64_t)&mapA2) : "memory");
+      asm volatile("prefetch.tensormap [%0];" ::"l"((uint64_t)&mapS0) : "memory");
+      asm volatile("prefetch.tensormap [%0];" ::"l"((uint64_t)&mapS1) : "memory");
+    }
   }
   if (warp == 1) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
@@ -272,12 +315,13 @@ tc_grouped_gemm(const __grid_constant__ CUtensorMap mapA, const __grid_constant_
     const bool bad = warp_group_offsets(p.offsets, nE, p.rows, p.rows_cap, st->off, st->tile_start,
                                         [n_tiles](int cnt) { return ((cnt + BM - 1) / BM) * n_tiles; });
     if (bad && lane == 0) record_status(p.status, kDevBadOffsets);
+    if (lane == 0) st->tile_start[nE + 1] = st->tile_start[nE] + ((p.shared_rows + BM - 1) / BM) * n_tiles;
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = st->tmem_base;
-  const int total = st->tile_start[nE];
+  const int total = st->tile_start[nE + 1];
   const int kb_n = (p.K + BK - 1) / BK;
   volatile int *abort_flag = &st->abort_flag;
 
@@ -289,28 +333,24 @@ tc_grouped_gemm(const __grid_constant__ CUtensorMap mapA, const __grid_constant_
     uint32_t it = 0;
     bool ok = true;
     for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
-      const TileInfo ti = decode_tile(st, nE, p.n_tiles, tile);
+      const TileInfo ti = decode_tile(st, nE, p.n_tiles, p.shared_rows, tile);
       // rows past the expert's end repeat its first row (their results are masked)
-      const int row_end = st->off[ti.e + 1];
-      int g[4];
+      int g[4] = {0, 0, 0, 0};
+      if (!ti.shared) {
+        const int row_end = st->off[ti.e + 1];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const int r = ti.row0 + lane * 4 + i;
-        g[i] = p.gather[r < row_end ? r : ti.row0];
+        for (int i = 0; i < 4; ++i) {
+          const int r = ti.row0 + lane * 4 + i;
+          g[i] = p.gather[r < row_end ? r : ti.row0];
+        }
       }
       int b0, b1;
-      if (p.mode == MODE_SWIGLU) {
-        b0 = ti.e * p.b_stride + ti.n * 128;
-        b1 = b0;
-      } else {
-        b0 = ti.e * p.b_stride + ti.n * BN;
-        b1 = b0 + 128;
-      }
+      b_rows(p, ti, b0, b1);
       for (int kb = 0; kb < kb_n; ++kb, ++it) {
         const int s = it % STAGES;
         const uint32_t ph = (it / STAGES) & 1u;
         int good = 1;
-        if (lane == 0) good = wait_bounded(&st->empty[s], ph ^ 1u, abort_flag, p.status, kDevTimeoutProducer);
+        if (lane == 0) good = wait_bounded(&st->empty[s], ph ^ 1u, abort_flag, p.status, kDevTimeoutProducer, p.timeout_ns);
         good = __shfl_sync(0xffffffffu, good, 0);
         if (!good) {
           ok = false;
@@ -320,10 +360,16 @@ tc_grouped_gemm(const __grid_constant__ CUtensorMap mapA, const __grid_constant_
         const uint32_t fb = smem_u32(&st->full[s]);
         if (lane == 0) mbar_expect_tx(&st->full[s], STAGE_BYTES);
         __syncwarp();
-        tma_gather4(smem_u32(sa) + (uint32_t)lane * 512u, &mapA, fb, kb * BK, g[0], g[1], g[2], g[3]);
-        if (lane == 0) {
-          tma_load_2d(smem_u32(sa + A_BYTES), &mapB0, fb, kb * BK, b0);
-          tma_load_2d(smem_u32(sa + A_BYTES + BH_BYTES), &mapB1, fb, kb * BK, b1);
+        if (!ti.shared) {
+          tma_gather4(smem_u32(sa) + (uint32_t)lane * 512u, &mapA, fb, kb * BK, g[0], g[1], g[2], g[3]);
+          if (lane == 0) {
+            tma_load_2d(smem_u32(sa + A_BYTES), &mapB0, fb, kb * BK, b0);
+            tma_load_2d(smem_u32(sa + A_BYTES + BH_BYTES), &mapB1, fb, kb * BK, b1);
+          }
+        } else if (lane == 0) {
+          tma_load_2d(smem_u32(sa), &mapA2, fb, kb * BK, ti.row0);
+          tma_load_2d(smem_u32(sa + A_BYTES), &mapS0, fb, kb * BK, b0);
+          tma_load_2d(smem_u32(sa + A_BYTES + BH_BYTES), &mapS1, fb, kb * BK, b1);
         }
       }
     }
@@ -339,28 +385,25 @@ tc_grouped_gemm(const __grid_constant__ CUtensorMap mapA, const __grid_constant_
       uint32_t it = 0;
       bool ok = true;
       for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
-        const TileInfo ti = decode_tile(st, nE, p.n_tiles, tile);
+        const TileInfo ti = decode_tile(st, nE, p.n_tiles, p.shared_rows, tile);
         int b0, b1;
-        if (p.mode == MODE_SWIGLU) {
-          b0 = ti.e * p.b_stride + ti.n * 128;
-          b1 = b0;
-        } else {
-          b0 = ti.e * p.b_stride + ti.n * BN;
-          b1 = b0 + 128;
-        }
+        b_rows(p, ti, b0, b1);
+        const CUtensorMap *ma = ti.shared ? &mapA2 : &mapA;
+        const CUtensorMap *mb0 = ti.shared ? &mapS0 : &mapB0;
+        const CUtensorMap *mb1 = ti.shared ? &mapS1 : &mapB1;
         for (int kb = 0; kb < kb_n; ++kb, ++it) {
           const int s = it % STAGES;
           const uint32_t ph = (it / STAGES) & 1u;
-          if (!wait_bounded(&st->empty[s], ph ^ 1u, abort_flag, p.status, kDevTimeoutProducer)) {
+          if (!wait_bounded(&st->empty[s], ph ^ 1u, abort_flag, p.status, kDevTimeoutProducer, p.timeout_ns)) {
             ok = false;
             break;
           }
           uint8_t *sa = tiles + (size_t)s * STAGE_BYTES;
           const uint32_t fb = smem_u32(&st->full[s]);
           mbar_expect_tx(&st->full[s], STAGE_BYTES);
-          tma_load_2d(smem_u32(sa), &mapA, fb, kb * BK, ti.row0);
-          tma_load_2d(smem_u32(sa + A_BYTES), &mapB0, fb, kb * BK, b0);
-          tma_load_2d(smem_u32(sa + A_BYTES + BH_BYTES), &mapB1, fb, kb * BK, b1);
+          tma_load_2d(smem_u32(sa), ma, fb, kb * BK, ti.row0);
+          tma_load_2d(smem_u32(sa + A_BYTES), mb0, fb, kb * BK, b0);
+          tma_load_2d(smem_u32(sa + A_BYTES + BH_BYTES), mb1, fb, kb * BK, b1);
         }
       }
       if (!ok) {
@@ -378,7 +421,7 @@ tc_grouped_gemm(const __grid_constant__ CUtensorMap mapA, const __grid_constant_
       bool ok = true;
       for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
         const uint32_t buf = tcount & 1u, use = tcount >> 1;
-        if (!wait_bounded(&st->acc_empty[buf], (use & 1u) ^ 1u, abort_flag, p.status, kDevTimeoutMma)) {
+        if (!wait_bounded(&st->acc_empty[buf], (use & 1u) ^ 1u, abort_flag, p.status, kDevTimeoutMma, p.timeout_ns)) {
           ok = false;
           break;
         }
@@ -387,7 +430,7 @@ tc_grouped_gemm(const __grid_constant__ CUtensorMap mapA, const __grid_constant_
         for (int kb = 0; kb < kb_n; ++kb, ++it) {
           const int s = it % STAGES;
           const uint32_t ph = (it / STAGES) & 1u;
-          if (!wait_bounded(&st->full[s], ph, abort_flag, p.status, kDevTimeoutMma)) {
+          if (!wait_bounded(&st->full[s], ph, abort_flag, p.status, kDevTimeoutMma, p.timeout_ns)) {
             ok = false;
             break;
           }
@@ -415,13 +458,13 @@ tc_grouped_gemm(const __grid_constant__ CUtensorMap mapA, const __grid_constant_
     const int rloc = q * 32 + lane;         // row of the tile this thread stores
     uint32_t tcount = 0;
     for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
-      const TileInfo ti = decode_tile(st, nE, p.n_tiles, tile);
+      const TileInfo ti = decode_tile(st, nE, p.n_tiles, p.shared_rows, tile);
       const uint32_t buf = tcount & 1u, use = tcount >> 1;
-      if (!wait_bounded(&st->acc_full[buf], use & 1u, abort_flag, p.status, kDevTimeoutEpilogue)) break;
+      if (!wait_bounded(&st->acc_full[buf], use & 1u, abort_flag, p.status, kDevTimeoutEpilogue, p.timeout_ns)) break;
       tc_fence_after();
       const uint32_t tb = tmem_base + buf * BN + ((uint32_t)(q * 32) << 16);
       const bool valid = rloc < ti.rows;
-      __nv_bfloat16 *orow = p.out + (size_t)(ti.row0 + (valid ? rloc : 0)) * p.N;
+      __nv_bfloat16 *orow = (ti.shared ? p.out2 : p.out) + (size_t)(ti.row0 + (valid ? rloc : 0)) * p.N;
       if (p.mode == MODE_SWIGLU) {
         const int col0 = ti.n * 128;
 #pragma unroll 1
@@ -535,15 +578,33 @@ int sm_count() {
 // the end of the last expert's N.
 // gather (nullable): A row r is token gather[r] of A = [a_rows, K] (the
 // fused dispatch); otherwise A is [rows_cap, K] in row order.
+// shared (nullable): the shared-expert group, one more group after the
+// experts with its own A ([shared->rows, K]), weights ([N, K] each) and output.
+struct SharedGroup {
+  const void *a, *b0, *b1;
+  int rows;
+  void *out;
+};
+
 cudaError_t run_gemm(const void *A, int rows_cap, int K, const void *B0, const void *B1, int b_stride, int N,
                      int mode, const int32_t *offsets, int E, int rows, void *out, int *status,
-                     cudaStream_t s, const int32_t *gather = nullptr, int a_rows = 0) {
-  CUtensorMap ma, mb0, mb1;
-  const int b_rows = ((offsets ? E : 1) - 1) * b_stride + N;
+                     cudaStream_t s, const int32_t *gather = nullptr, int a_rows = 0,
+                     const SharedGroup *shared = nullptr) {
+  CUtensorMap ma, mb0, mb1, ma2, ms0, ms1;
+  const int b_rows_total = ((offsets ? E : 1) - 1) * b_stride + N;
   cudaError_t err = gather ? make_map(&ma, A, (uint64_t)K, (uint64_t)a_rows, 1)
                            : make_map(&ma, A, (uint64_t)K, (uint64_t)rows_cap, BM);
-  if (err == cudaSuccess) err = make_map(&mb0, B0, (uint64_t)K, (uint64_t)b_rows, 128);
-  if (err == cudaSuccess) err = make_map(&mb1, B1, (uint64_t)K, (uint64_t)b_rows, 128);
+  if (err == cudaSuccess) err = make_map(&mb0, B0, (uint64_t)K, (uint64_t)b_rows_total, 128);
+  if (err == cudaSuccess) err = make_map(&mb1, B1, (uint64_t)K, (uint64_t)b_rows_total, 128);
+  if (err == cudaSuccess && shared) {
+    err = make_map(&ma2, shared->a, (uint64_t)K, (uint64_t)shared->rows, BM);
+    if (err == cudaSuccess) err = make_map(&ms0, shared->b0, (uint64_t)K, (uint64_t)N, 128);
+    if (err == cudaSuccess) err = make_map(&ms1, shared->b1, (uint64_t)K, (uint64_t)N, 128);
+  } else {
+    ma2 = ma;
+    ms0 = mb0;
+    ms1 = mb1;
+  }
   if (err != cudaSuccess) return err;
   TcParams p;
   p.offsets = offsets;
@@ -557,14 +618,17 @@ cudaError_t run_gemm(const void *A, int rows_cap, int K, const void *B0, const v
   p.n_tiles = mode == MODE_SWIGLU ? (N + 127) / 128 : (N + BN - 1) / BN;
   p.out = static_cast<__nv_bfloat16 *>(out);
   p.status = status;
+  p.timeout_ns = wait_timeout_ns();
   p.gather = gather;
+  p.shared_rows = shared ? shared->rows : 0;
+  p.out2 = shared ? static_cast<__nv_bfloat16 *>(shared->out) : nullptr;
   const int nE = offsets ? E : 1;
-  const long long upper = ((long long)(rows_cap + BM - 1) / BM + nE) * p.n_tiles;
+  const long long upper = ((long long)(rows_cap + BM - 1) / BM + nE + (p.shared_rows + BM - 1) / BM) * p.n_tiles;
   const int sms = sm_count();
   const int grid = (int)(upper < sms ? upper : sms);
   err = cudaFuncSetAttribute(tc_grouped_gemm, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
   if (err != cudaSuccess) return err;
-  launch_plain(tc_grouped_gemm, grid, THREADS, SMEM_BYTES, s, ma, mb0, mb1, p);
+  launch_plain(tc_grouped_gemm, grid, THREADS, SMEM_BYTES, s, ma, mb0, mb1, ma2, ms0, ms1, p);
   return cudaGetLastError();
 }
 
@@ -572,16 +636,22 @@ cudaError_t run_gemm(const void *A, int rows_cap, int K, const void *B0, const v
 
 cudaError_t launch_ffn_tc_bf16(const FfnArgs &a, cudaStream_t s) {
   cudaError_t err;
+  SharedGroup sh1{}, sh2{};
+  const bool sh = a.shared_rows > 0;
+  if (sh) {
+    sh1 = SharedGroup{a.shared_x, a.shared_w1, a.shared_w2, a.shared_rows, a.shared_h};
+    sh2 = SharedGroup{a.shared_h, a.shared_w3, a.shared_w3, a.shared_rows, a.shared_y};
+  }
   if (a.act == MOE_ACT_SWIGLU)
     err = run_gemm(a.x, a.rows_cap, a.d, a.w1, a.w2, a.w_stride, a.F, MODE_SWIGLU, a.offsets, a.E, a.rows, a.h,
-                   a.status, s, a.gather, a.x_rows);
+                   a.status, s, a.gather, a.x_rows, sh ? &sh1 : nullptr);
   else
     err = run_gemm(a.x, a.rows_cap, a.d, a.w1, a.w1, a.w_stride, a.F, MODE_RELU, a.offsets, a.E, a.rows, a.h,
-                   a.status, s, a.gather, a.x_rows);
+                   a.status, s, a.gather, a.x_rows, sh ? &sh1 : nullptr);
   if (err != cudaSuccess) return err;
   if (a.mid_event && (err = cudaEventRecord(a.mid_event, s)) != cudaSuccess) return err;
   return run_gemm(a.h, a.rows_cap, a.F, a.w3, a.w3, a.d, a.d, MODE_PLAIN, a.offsets, a.E, a.rows, a.y,
-                  a.status, s);
+                  a.status, s, nullptr, 0, sh ? &sh2 : nullptr);
 }
 
 }  // namespace moe

@@ -23,7 +23,7 @@
 //               the even CTA's barrier.
 // No copy multicasts: each CTA loads only its own tiles.
 //
-// Every mbarrier wait is bounded (2 s of %globaltimer); on expiry the thread
+// Every mbarrier wait is bounded by %globaltimer (2 s unless moe_set_wait_timeout_ns says otherwise); on expiry the thread
 // records a status code, raises its CTA's abort flag and drains what it
 // issued; both CTAs meet at the final cluster barrier and free TMEM.
 #include "common.cuh"
@@ -43,7 +43,6 @@ constexpr int B_BYTES = 128 * BK * 2;         // 16 KiB: this CTA's B half
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
 constexpr int THREADS = 192;
 constexpr uint32_t TMEM_COLS = 512;
-constexpr uint64_t TIMEOUT_NS = 2000000000ull;
 constexpr uint64_t DRAIN_NS = 200000000ull;
 
 // kind::f16, D fp32, A/B bf16 K-major, N = 256, M = 256 (pair)
@@ -53,6 +52,7 @@ constexpr uint32_t IDESC = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BN >
 enum Mode { MODE_PLAIN = 0, MODE_RELU = 1, MODE_SWIGLU = 2 };
 
 struct Tc2Params {
+  uint64_t timeout_ns;        // bound on every barrier wait (moe_set_wait_timeout_ns)
   const int32_t *offsets;
   int E, rows, rows_cap, N, b_stride, b_rows, K, mode, n_tiles;
   __nv_bfloat16 *out;
@@ -114,14 +114,15 @@ __device__ __forceinline__ uint64_t global_ns() {
   asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
   return t;
 }
-__device__ __forceinline__ bool wait_bounded(uint64_t *bar, uint32_t parity, volatile int *abort_flag, int *status,
-                                             int code) {
+__device__ __forceinline__ bool wait_bounded(uint64_t *bar, uint32_t parity, volatile int *abort_flag,
+                                             int *status, int code, uint64_t limit_ns) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_ns();
   uint32_t spins = 0;
   while (!mbar_try_wait(bar, parity)) {
     if (*abort_flag) return false;
-    if ((++spins & 31u) == 0 && global_ns() - t0 > TIMEOUT_NS) {
+    // the clock is read every 32 polls, or every poll under a limit below 1 us
+    if (((++spins & 31u) == 0 || limit_ns < 1000u) && global_ns() - t0 > limit_ns) {
       *abort_flag = 1;
       record_status(status, code);
       return false;
@@ -285,7 +286,7 @@ tc2_grouped_gemm(const __grid_constant__ CUtensorMap mapA, const __grid_constant
         for (int kb = 0; kb < kb_n; ++kb, ++it) {
           const int s = it % STAGES;
           const uint32_t ph = (it / STAGES) & 1u;
-          if (!wait_bounded(&st->empty[s], ph ^ 1u, abort_flag, p.status, kDevTimeoutProducer)) {
+          if (!wait_bounded(&st->empty[s], ph ^ 1u, abort_flag, p.status, kDevTimeoutProducer, p.timeout_ns)) {
             ok = false;
             break;
           }
@@ -318,7 +319,7 @@ tc2_grouped_gemm(const __grid_constant__ CUtensorMap mapA, const __grid_constant
       bool ok = true;
       for (int tile = cluster; tile < total && ok; tile += n_clusters) {
         const uint32_t buf = tcount & 1u, use = tcount >> 1;
-        if (!wait_bounded(&st->acc_empty[buf], (use & 1u) ^ 1u, abort_flag, p.status, kDevTimeoutMma)) {
+        if (!wait_bounded(&st->acc_empty[buf], (use & 1u) ^ 1u, abort_flag, p.status, kDevTimeoutMma, p.timeout_ns)) {
           ok = false;
           break;
         }
@@ -327,7 +328,7 @@ tc2_grouped_gemm(const __grid_constant__ CUtensorMap mapA, const __grid_constant
         for (int kb = 0; kb < kb_n; ++kb, ++it) {
           const int s = it % STAGES;
           const uint32_t ph = (it / STAGES) & 1u;
-          if (!wait_bounded(&st->full[s], ph, abort_flag, p.status, kDevTimeoutMma)) {
+          if (!wait_bounded(&st->full[s], ph, abort_flag, p.status, kDevTimeoutMma, p.timeout_ns)) {
             ok = false;
             break;
           }
@@ -356,7 +357,7 @@ tc2_grouped_gemm(const __grid_constant__ CUtensorMap mapA, const __grid_constant
     for (int tile = cluster; tile < total; tile += n_clusters) {
       const Tile2 ti = decode_tile2(st, nE, tile);
       const uint32_t buf = tcount & 1u, use = tcount >> 1;
-      if (!wait_bounded(&st->acc_full[buf], use & 1u, abort_flag, p.status, kDevTimeoutEpilogue)) break;
+      if (!wait_bounded(&st->acc_full[buf], use & 1u, abort_flag, p.status, kDevTimeoutEpilogue, p.timeout_ns)) break;
       tc_fence_after();
       const uint32_t tb = tmem_base + buf * BN + ((uint32_t)(q * 32) << 16);
       const int row = ti.row0 + (int)rank * BM + rloc;
@@ -507,6 +508,7 @@ cudaError_t run_gemm2(const void *A, int rows_cap, int K, const void *B0, const 
   p.n_tiles = mode == MODE_SWIGLU ? (N + 127) / 128 : (N + BN - 1) / BN;
   p.out = static_cast<__nv_bfloat16 *>(out);
   p.status = status;
+  p.timeout_ns = wait_timeout_ns();
   const int nE = offsets ? E : 1;
   const long long upper = ((long long)(rows_cap + 2 * BM - 1) / (2 * BM) + nE) * p.n_tiles;
   err = cudaFuncSetAttribute(tc2_grouped_gemm, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);

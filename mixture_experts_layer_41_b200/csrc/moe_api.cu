@@ -80,6 +80,7 @@ FfnArgs ffn_args(const moe_config &c, const WsLayout &L, void *ws) {
   a.F = c.intermediate;
   a.h = ws_ptr<char>(ws, L.h);
   a.status = ws_ptr<int>(ws, L.status);
+  a.q4_scratch = ws_ptr<char>(ws, L.q4_tokens);
   return a;
 }
 
@@ -87,30 +88,44 @@ FfnArgs ffn_args(const moe_config &c, const WsLayout &L, void *ws) {
 // in the environment, which selects the kernel on pairs of SMs (same
 // results bit for bit; measured slower on the dense workloads, so it is not
 // the default).  The fused gather always runs on one SM.
-bool use_pair_gemm(const FfnArgs &a) {
-  if (a.gather) return false;
+bool pair_env() {
   const char *env = getenv("MOE_TC_PAIR");
   return env && env[0] == '1';
 }
 
+bool use_pair_gemm(const FfnArgs &a) {
+  if (a.gather || a.shared_rows > 0) return false;
+  return pair_env();
+}
+
+// moe_forward runs the shared expert as one more group of the bf16 grouped
+// GEMM (both phases) when it has the experts' width, unless the routed
+// experts are to run on pairs of SMs (that kernel has no shared group).
+bool shared_in_grouped_gemm(const moe_config &c) {
+  return c.shared_intermediate > 0 && c.shared_intermediate == c.intermediate && c.weight_dtype == MOE_BF16 &&
+         c.act_dtype == MOE_BF16 && !(pair_env() && !c.fused_gather);
+}
+
 // 4-bit weights: decode-sized groups (a few token rows per expert) go to the
-// warp-level kernel, whose 8-token MMA blocks fit them; larger groups to the
-// tcgen05 kernel.  MOE_Q4_KERNEL=mma / tc in the environment forces one.
-bool use_q4_mma(const FfnArgs &a) {
-  if (!q4_mma_supported(a.d, a.F)) return false;
+// warp-level integer-MMA kernel, whose 4-token MMA blocks fit them; larger
+// groups to the tcgen05 kernel.  MOE_Q4_KERNEL=i8 / mma / tc in the
+// environment forces one (mma: warp-level bf16 MMAs on dequantised weights).
+cudaError_t run_q4(const FfnArgs &a, cudaStream_t s) {
   const char *env = getenv("MOE_Q4_KERNEL");
-  if (env && strcmp(env, "mma") == 0) return true;
-  if (env && strcmp(env, "tc") == 0) return !q4_tc_supported(a.d, a.F);
-  return (long long)a.rows_cap <= 16LL * a.E;
+  const bool i8 = q4_i8_supported(a.d, a.F), mma = q4_mma_supported(a.d, a.F), tc = q4_tc_supported(a.d, a.F);
+  if (env && strcmp(env, "mma") == 0 && mma) return launch_ffn_q4_mma(a, s);
+  if (env && strcmp(env, "i8") == 0 && i8) return launch_ffn_q4_i8(a, s);
+  if (env && strcmp(env, "tc") == 0 && tc) return launch_ffn_q4_tc(a, s);
+  if (i8 && (long long)a.rows_cap <= 16LL * a.E) return launch_ffn_q4_i8(a, s);
+  if (tc) return launch_ffn_q4_tc(a, s);
+  return i8 ? launch_ffn_q4_i8(a, s) : launch_ffn_q4(a, s);
 }
 
 cudaError_t run_ffn(const FfnArgs &a, cudaStream_t s) {
   switch (a.kind) {
     case 0: return launch_ffn_simt_f32(a, s);
     case 1: return use_pair_gemm(a) ? launch_ffn_tc2_bf16(a, s) : launch_ffn_tc_bf16(a, s);
-    default:
-      if (use_q4_mma(a)) return launch_ffn_q4_mma(a, s);
-      return q4_tc_supported(a.d, a.F) ? launch_ffn_q4_tc(a, s) : launch_ffn_q4(a, s);
+    default: return run_q4(a, s);
   }
 }
 
@@ -138,10 +153,22 @@ moe_status do_permute(const moe_config &c, const void *x, const int32_t *ids, co
 
 // gather (nullable): x_perm is the token matrix itself and row r of the
 // expert-sorted order is token gather[r] (bf16 tensor-core path only).
+// shared_x / shared_out (nullable): the shared expert's tokens and output,
+// computed as one more group of the same two launches.
 moe_status do_ffn(const moe_config &c, const void *x_perm, const int32_t *off, const moe_weights *w, void *y,
-                  void *ws, cudaStream_t s, cudaEvent_t mid = nullptr, const int32_t *gather = nullptr) {
+                  void *ws, cudaStream_t s, cudaEvent_t mid = nullptr, const int32_t *gather = nullptr,
+                  const void *shared_x = nullptr, void *shared_out = nullptr) {
   const WsLayout L = ws_layout(c);
   FfnArgs a = ffn_args(c, L, ws);
+  if (shared_x) {
+    a.shared_rows = c.num_tokens;
+    a.shared_x = shared_x;
+    a.shared_w1 = w->shared1;
+    a.shared_w2 = w->shared2;
+    a.shared_w3 = w->shared3;
+    a.shared_h = ws_ptr<char>(ws, L.shared_h);
+    a.shared_y = shared_out;
+  }
   a.mid_event = mid;
   a.offsets = off;
   a.x = x_perm;
@@ -203,6 +230,10 @@ void moe::set_last_error_text(const char *text) { set_error("%s%s", text); }
 
 static std::atomic<long long> g_launches{0};
 void moe::note_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
+
+static constexpr uint64_t kDefaultWaitNs = 2000000000ull;
+static std::atomic<uint64_t> g_wait_ns{kDefaultWaitNs};
+uint64_t moe::wait_timeout_ns() { return g_wait_ns.load(std::memory_order_relaxed); }
 
 extern "C" {
 
@@ -327,6 +358,11 @@ const char *moe_status_string(moe_status s) {
 const char *moe_last_error(void) { return g_last_error; }
 
 int64_t moe_kernel_launches(void) { return g_launches.load(std::memory_order_relaxed); }
+
+moe_status moe_set_wait_timeout_ns(uint64_t ns) {
+  g_wait_ns.store(ns == 0 ? kDefaultWaitNs : ns, std::memory_order_relaxed);
+  return MOE_OK;
+}
 
 moe_status moe_workspace_status(const void *ws, moe_stream_t stream) {
   if (!aligned16(ws)) return MOE_ERR_WORKSPACE;
@@ -472,16 +508,17 @@ moe_status moe_expert_counts(const moe_config *cfg, const int32_t *topk_ids, int
 }
 
 moe_status moe_permute_shard(const moe_config *cfg, const void *x, const int32_t *topk_ids, const float *topk_w,
-                             const int32_t *shard_base, int64_t capacity, int32_t *expert_offsets,
-                             int32_t *perm_token, float *perm_w, int32_t *slot_row, void *x_perm,
-                             const moe_stats *stats, void *ws, size_t ws_bytes, moe_stream_t stream) {
+                             const int32_t *counts_by_rank, int32_t world, int32_t rank, int64_t capacity,
+                             int32_t *expert_offsets, int32_t *perm_token, float *perm_w, int32_t *slot_row,
+                             void *x_perm, const moe_stats *stats, void *ws, size_t ws_bytes, moe_stream_t stream) {
   moe_status st = moe_validate(cfg);
   if (st != MOE_OK) return st;
   const moe_config &c = *cfg;
-  if (capacity < -1) return MOE_ERR_INVALID_ARG;
+  if (capacity < -1 || world < 1 || rank < 0 || rank >= world) return MOE_ERR_INVALID_ARG;
+  if (world > 1 && !counts_by_rank) return MOE_ERR_INVALID_ARG;
   if (!aligned16(topk_ids) || !aligned16(topk_w) || !aligned16(expert_offsets) || !aligned16(perm_token) ||
       !aligned16(perm_w) || !aligned16(slot_row) || !aligned16_or_null(x) || !aligned16_or_null(x_perm) ||
-      !aligned16_or_null(shard_base))
+      !aligned16_or_null(counts_by_rank))
     return MOE_ERR_INVALID_ARG;
   if ((x == nullptr) != (x_perm == nullptr)) return MOE_ERR_INVALID_ARG;
   if (!stats || !aligned16(stats->raw_counts) || !aligned16(stats->kept_counts) || !aligned16(stats->dropped))
@@ -493,8 +530,19 @@ moe_status moe_permute_shard(const moe_config *cfg, const void *x, const int32_t
   cudaError_t err = launch_permute(c, x, topk_ids, topk_w, capacity, expert_offsets, perm_token, perm_w, slot_row,
                                    x_perm, stats->raw_counts, stats->kept_counts, stats->dropped,
                                    ws_ptr<int32_t>(ws, L.blk_counts), ws_ptr<int32_t>(ws, L.blk_base),
-                                   ws_ptr<int32_t>(ws, L.local_rank), ws_ptr<int>(ws, L.status), s, shard_base);
+                                   ws_ptr<int32_t>(ws, L.local_rank), ws_ptr<int>(ws, L.status), s,
+                                   rank > 0 ? counts_by_rank : nullptr, rank);
   return err == cudaSuccess ? MOE_OK : cuda_fail(err, "moe_permute_shard");
+}
+
+moe_status moe_ep_local_ids(const int32_t *recv_counts, int32_t world, int32_t experts_per_rank, int32_t rows,
+                            int32_t *ids, moe_stream_t stream) {
+  if (world < 1 || experts_per_rank < 1 || (int64_t)world * experts_per_rank > kMaxExperts || rows < 0)
+    return MOE_ERR_INVALID_ARG;
+  if (!aligned16(recv_counts) || (rows > 0 && !aligned16(ids))) return MOE_ERR_INVALID_ARG;
+  cudaError_t err = launch_ep_local_ids(recv_counts, world, experts_per_rank, rows, ids,
+                                        reinterpret_cast<cudaStream_t>(stream));
+  return err == cudaSuccess ? MOE_OK : cuda_fail(err, "moe_ep_local_ids");
 }
 
 moe_status moe_grouped_ffn(const moe_config *cfg, const void *x_perm, const int32_t *expert_offsets,
@@ -564,15 +612,14 @@ static moe_status forward_impl(const moe_config &c, const void *x, const float *
     return st;
   if ((err = mark(MOE_PHASE_PERMUTE, s)) != cudaSuccess) return cuda_fail(err, "phase event");
   void *y_perm = ws_ptr<char>(ws, L.y_perm);
+  void *shared = c.shared_intermediate > 0 ? ws_ptr<char>(ws, L.shared_out) : nullptr;
+  const bool shared_fused = shared && shared_in_grouped_gemm(c);
   if ((st = do_ffn(c, fused_gather ? x : x_perm, off, w, y_perm, ws, s, g_nevents ? g_events[MOE_PHASE_FFN1] : nullptr,
-                   fused_gather ? perm_token : nullptr)) != MOE_OK)
+                   fused_gather ? perm_token : nullptr, shared_fused ? x : nullptr,
+                   shared_fused ? shared : nullptr)) != MOE_OK)
     return st;
   if ((err = mark(MOE_PHASE_FFN2, s)) != cudaSuccess) return cuda_fail(err, "phase event");
-  void *shared = nullptr;
-  if (c.shared_intermediate > 0) {
-    shared = ws_ptr<char>(ws, L.shared_out);
-    if ((st = do_shared(c, x, w, shared, ws, s)) != MOE_OK) return st;
-  }
+  if (shared && !shared_fused && (st = do_shared(c, x, w, shared, ws, s)) != MOE_OK) return st;
   if ((err = mark(MOE_PHASE_SHARED, s)) != cudaSuccess) return cuda_fail(err, "phase event");
   err = launch_combine(c, y_perm, ws_ptr<int32_t>(ws, L.slot_row), wts, shared, out, s);
   if (err != cudaSuccess) return cuda_fail(err, "moe_forward combine");

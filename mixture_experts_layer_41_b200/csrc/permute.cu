@@ -60,23 +60,36 @@ count_kernel(const int32_t *ids, int T, int k, int E, int32_t *blk_counts, int32
 }
 
 // One block of up to 1024 threads, one thread per expert.
-// shard_base (nullable): slots of each expert held by earlier token shards of
-// the same batch; the capacity left for this shard is cap - shard_base[e].
-__global__ void scan_kernel(const int32_t *blk_counts, int nb, int E, long long cap, const int32_t *shard_base,
-                            int32_t *blk_base, int32_t *raw_counts, int32_t *kept_counts,
+// counts_by_rank (nullable): [world, E] raw slot counts of every token shard
+// of the same batch, in token order; the slots of expert e held by the
+// shards before `rank` are the sum of rows 0..rank-1, and the capacity left
+// for this shard is cap minus that.
+__global__ void scan_kernel(const int32_t *blk_counts, int nb, int E, long long cap, const int32_t *counts_by_rank,
+                            int rank, int32_t *blk_base, int32_t *raw_counts, int32_t *kept_counts,
                             int32_t *offsets, int32_t *dropped) {
   pdl_enter();
   __shared__ int32_t kept_s[kMaxExperts];
   __shared__ int32_t drop_s[kMaxExperts];
   const int e = threadIdx.x;
   if (e < E) {
+    // exclusive prefix over the count blocks, 16 loads in flight at a time
     int run = 0;
-    for (int b = 0; b < nb; ++b) {
-      blk_base[(size_t)b * E + e] = run;
-      run += blk_counts[(size_t)b * E + e];
+    for (int b0 = 0; b0 < nb; b0 += 16) {
+      int v[16];
+#pragma unroll
+      for (int u = 0; u < 16; ++u) v[u] = b0 + u < nb ? __ldg(blk_counts + (size_t)(b0 + u) * E + e) : 0;
+#pragma unroll
+      for (int u = 0; u < 16; ++u) {
+        if (b0 + u < nb) blk_base[(size_t)(b0 + u) * E + e] = run;
+        run += v[u];
+      }
     }
     long long room = cap;
-    if (cap >= 0 && shard_base) room = cap - shard_base[e] > 0 ? cap - shard_base[e] : 0;
+    if (cap >= 0 && counts_by_rank) {
+      long long before = 0;
+      for (int r = 0; r < rank; ++r) before += counts_by_rank[(size_t)r * E + e];
+      room = cap - before > 0 ? cap - before : 0;
+    }
     const int kept = (room >= 0 && (long long)run > room) ? (int)room : run;
     raw_counts[e] = run;
     kept_counts[e] = kept;
@@ -99,9 +112,9 @@ __global__ void scan_kernel(const int32_t *blk_counts, int nb, int E, long long 
 template <int VEC_BYTES>
 __global__ void __launch_bounds__(256)
 scatter_kernel(const int32_t *ids, const float *wts, const int32_t *local_rank,
-               const int32_t *blk_base, const int32_t *offsets, int T, int k, int E,
-               long long cap, const int32_t *shard_base, const char *x, size_t row_bytes, int32_t *perm_token,
-               float *perm_w, int32_t *slot_row, char *x_perm) {
+               const int32_t *blk_base, const int32_t *offsets, const int32_t *kept, int T, int k, int E,
+               const char *x, size_t row_bytes, int32_t *perm_token, float *perm_w, int32_t *slot_row,
+               char *x_perm) {
   pdl_enter();
   const int warp_global = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
@@ -111,9 +124,10 @@ scatter_kernel(const int32_t *ids, const float *wts, const int32_t *local_rank,
   const int lr = local_rank[warp_global];
   int row = -1;
   if (e >= 0 && e < E && lr >= 0) {
+    // the slot's rank among its expert's slots in token order; the capacity
+    // cut kept the first kept[e] of them
     const int rank = blk_base[(size_t)(t / kPermTokens) * E + e] + lr;
-    const long long room = (cap >= 0 && shard_base) ? cap - shard_base[e] : cap;
-    if (cap < 0 || (long long)rank < room) row = offsets[e] + rank;
+    if (rank < kept[e]) row = offsets[e] + rank;
   }
   if (lane == 0) {
     slot_row[warp_global] = row;
@@ -155,21 +169,56 @@ scatter_kernel(const int32_t *ids, const float *wts, const int32_t *local_rank,
   }
 }
 
+// Expert parallelism: local expert of every received row.  The rows arrive
+// grouped by source rank, and inside a source by local expert, with
+// recv_counts[s][e] rows of (s, e); row i belongs to the segment whose
+// prefix range holds i.  Rows past the last segment get -1.
+__global__ void __launch_bounds__(256)
+ep_local_ids_kernel(const int32_t *recv_counts, int nseg, int e_local, int rows, int32_t *ids) {
+  pdl_enter();
+  __shared__ int32_t end[kMaxExperts];      // inclusive prefix: segment q holds rows [end[q-1], end[q])
+  if (threadIdx.x == 0) {
+    int acc = 0;
+    for (int q = 0; q < nseg; ++q) {
+      const int c = recv_counts[q];
+      acc += c > 0 ? c : 0;
+      end[q] = acc;
+    }
+  }
+  __syncthreads();
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < rows; i += gridDim.x * blockDim.x) {
+    int lo = 0, hi = nseg;                  // first segment with end > i
+    while (lo < hi) {
+      const int mid = (lo + hi) >> 1;
+      if (end[mid] > i) hi = mid; else lo = mid + 1;
+    }
+    ids[i] = lo < nseg ? lo % e_local : -1;
+  }
+}
+
 }  // namespace
+
+cudaError_t launch_ep_local_ids(const int32_t *recv_counts, int world, int e_local, int rows, int32_t *ids,
+                                cudaStream_t s) {
+  if (rows == 0) return cudaSuccess;
+  const int blocks = (rows + 255) / 256 < 1024 ? (rows + 255) / 256 : 1024;
+  launch_pdl(ep_local_ids_kernel, blocks, 256, 0, s, recv_counts, world * e_local, e_local, rows, ids);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_permute(const moe_config &c, const void *x, const int32_t *topk_ids,
                            const float *topk_w, int64_t capacity, int32_t *expert_offsets,
                            int32_t *perm_token, float *perm_w, int32_t *slot_row, void *x_perm,
                            int32_t *raw_counts, int32_t *kept_counts, int32_t *dropped,
                            int32_t *blk_counts, int32_t *blk_base, int32_t *local_rank,
-                           int *status, cudaStream_t s, const int32_t *shard_base) {
+                           int *status, cudaStream_t s, const int32_t *counts_by_rank, int rank) {
   const int T = c.num_tokens, k = c.top_k, E = c.num_experts;
   const int nb = perm_blocks(c);
   launch_pdl(count_kernel, nb, kPermTokens, 0, s, topk_ids, T, k, E, blk_counts, local_rank, status);
   cudaError_t err = cudaGetLastError();
   if (err != cudaSuccess) return err;
-  launch_pdl(scan_kernel, 1, kMaxExperts, 0, s, blk_counts, nb, E, (long long)capacity, shard_base, blk_base,
-                                        raw_counts, kept_counts, expert_offsets, dropped);
+  launch_pdl(scan_kernel, 1, kMaxExperts, 0, s, blk_counts, nb, E, (long long)capacity, counts_by_rank, rank,
+             blk_base, raw_counts, kept_counts, expert_offsets, dropped);
   err = cudaGetLastError();
   if (err != cudaSuccess) return err;
   const size_t row_bytes = act_size(c) * (size_t)c.hidden;
@@ -178,14 +227,12 @@ cudaError_t launch_permute(const moe_config &c, const void *x, const int32_t *to
   const bool vec16 = (row_bytes % 16) == 0;
   if (vec16)
     launch_pdl(scatter_kernel<16>, blocks, 256, 0, s, topk_ids, topk_w, local_rank, blk_base, expert_offsets,
-                                              T, k, E, (long long)capacity, shard_base,
-                                              static_cast<const char *>(x), row_bytes, perm_token,
-                                              perm_w, slot_row, static_cast<char *>(x_perm));
+               kept_counts, T, k, E, static_cast<const char *>(x), row_bytes, perm_token, perm_w, slot_row,
+               static_cast<char *>(x_perm));
   else
     launch_pdl(scatter_kernel<4>, blocks, 256, 0, s, topk_ids, topk_w, local_rank, blk_base, expert_offsets,
-                                             T, k, E, (long long)capacity, shard_base,
-                                             static_cast<const char *>(x), row_bytes, perm_token,
-                                             perm_w, slot_row, static_cast<char *>(x_perm));
+               kept_counts, T, k, E, static_cast<const char *>(x), row_bytes, perm_token, perm_w, slot_row,
+               static_cast<char *>(x_perm));
   return cudaGetLastError();
 }
 

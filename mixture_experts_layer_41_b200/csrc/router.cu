@@ -643,22 +643,323 @@ route_select(RouteParams p) {
   }
 }
 
+// ---------------------------------------------------------------- tensor-core plan: selection + exact weights
+// After the tensor-core logits (selection grade, within about 1e-5 of the
+// exact value) every token is handled by one warp in two parts:
+//  * selection in fp32 on those logits: softmax top-k (ranked by logit plus
+//    logit bias), or sigmoid scores, selection = score + bias, group top-two
+//    sums, the best topk_group groups and the top-k inside them; the token's
+//    probabilities (softmax p, or raw sigmoid s) feed the block's prob sums;
+//  * the chosen experts' logits recomputed exactly in ONE pass over the
+//    token's row: each 8-element chunk of x is widened to float64 once and
+//    used for up to 8 chosen experts (float64 products of bf16 x fp32 are
+//    exact, summed in float64 per lane in index order), then the eight lane
+//    sums are reduced across the warp by halving exchanges (18 shuffles
+//    instead of 8 full reductions).  Weights and the slot order come from
+//    these exact logits, as in the CUDA-core router.
+// Router replay (forced ids) takes the recorded ids instead of the top-k.
+
+// Exact logits of up to 8 chosen experts (ids[j], valid[j]) of bf16 token t.
+// Returns, on every lane, the sum for slot ((lane >> 4) & 1) * 4 +
+// ((lane >> 3) & 1) * 2 + ((lane >> 2) & 1).
+__device__ __forceinline__ double exact_logits8(const RouteParams &p, int t, const int (&ids)[8],
+                                                const bool (&valid)[8], int lane) {
+  const uint4 *xr = reinterpret_cast<const uint4 *>(static_cast<const __nv_bfloat16 *>(p.x) + (size_t)t * p.d);
+  const float4 *wr[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) wr[j] = reinterpret_cast<const float4 *>(p.w + (size_t)(valid[j] ? ids[j] : 0) * p.d);
+  double acc[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) acc[j] = 0.0;
+  const int nchunk = p.d / 8;
+#pragma unroll 1
+  for (int i = lane; i < nchunk; i += 32) {
+    const uint4 xv = __ldg(xr + i);
+    const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
+    double xd[8];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      xd[2 * u] = (double)__uint_as_float(xw[u] << 16);
+      xd[2 * u + 1] = (double)__uint_as_float(xw[u] & 0xFFFF0000u);
+    }
+    float4 wv[8][2];
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+      if (valid[j]) {
+        wv[j][0] = __ldg(wr[j] + 2 * i);
+        wv[j][1] = __ldg(wr[j] + 2 * i + 1);
+      }
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+      if (valid[j]) {
+        const float wf[8] = {wv[j][0].x, wv[j][0].y, wv[j][0].z, wv[j][0].w,
+                             wv[j][1].x, wv[j][1].y, wv[j][1].z, wv[j][1].w};
+#pragma unroll
+        for (int u = 0; u < 8; ++u) acc[j] = fma(xd[u], (double)wf[u], acc[j]);
+      }
+  }
+  // halving exchanges: lanes split by bit 4, then 3, then 2 keep half of the slots
+  const unsigned full = 0xffffffffu;
+  const int b4 = (lane >> 4) & 1, b3 = (lane >> 3) & 1, b2 = (lane >> 2) & 1;
+  double h4[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const double keep = b4 ? acc[i + 4] : acc[i];
+    const double send = b4 ? acc[i] : acc[i + 4];
+    h4[i] = keep + __shfl_xor_sync(full, send, 16);
+  }
+  double h3[2];
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {
+    const double keep = b3 ? h4[i + 2] : h4[i];
+    const double send = b3 ? h4[i] : h4[i + 2];
+    h3[i] = keep + __shfl_xor_sync(full, send, 8);
+  }
+  double h2 = (b2 ? h3[1] : h3[0]) + __shfl_xor_sync(full, b2 ? h3[0] : h3[1], 4);
+  h2 += __shfl_xor_sync(full, h2, 2);
+  h2 += __shfl_xor_sync(full, h2, 1);
+  return h2;
+}
+
+__device__ __forceinline__ void warp_argmax_f(float &v, int &i) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    const float ov = __shfl_xor_sync(0xffffffffu, v, o);
+    const int oi = __shfl_xor_sync(0xffffffffu, i, o);
+    if (ov > v || (ov == v && oi < i)) { v = ov; i = oi; }
+  }
+}
+
+// TPB tokens per block, WPB warps (TPB / WPB tokens per warp, in order).
+// Shared memory: the block's per-token probabilities [TPB][E] (fp32) and a
+// selection-score row per warp [WPB][E].
+template <int EPL, int TPB, int WPB>
+__global__ void __launch_bounds__(32 * WPB)
+route_select_refine(RouteParams p) {
+  pdl_enter();
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  const int E = p.E;
+  float *pr = reinterpret_cast<float *>(smem_raw);        // [TPB][E]
+  float *scr_all = pr + (size_t)TPB * E;                   // [WPB][E]
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const unsigned full = 0xffffffffu;
+  float *scr = scr_all + (size_t)warp * E;
+  const bool softmax = p.router == MOE_ROUTER_SOFTMAX_TOPK;
+  const int G = E / p.n_group;
+
+  for (int i = 0; i < TPB / WPB; ++i) {
+    const int tl = warp * (TPB / WPB) + i;                 // token within the block
+    const int t = blockIdx.x * TPB + tl;
+    if (t >= p.T) {
+#pragma unroll
+      for (int j = 0; j < EPL; ++j)
+        if (lane + 32 * j < E) pr[tl * E + lane + 32 * j] = 0.f;
+      continue;
+    }
+    // selection-grade logits: the hidden slices added in order
+    float lg[EPL];
+#pragma unroll
+    for (int j = 0; j < EPL; ++j) {
+      const int e = lane + 32 * j;
+      double v = 0.0;
+      if (e < E)
+        for (int q = 0; q < p.ks; ++q) v += p.logits[((size_t)q * p.T + t) * E + e];
+      lg[j] = (float)v;
+    }
+    float score[EPL], prob[EPL];
+    if (softmax) {
+      float m = -INFINITY;
+#pragma unroll
+      for (int j = 0; j < EPL; ++j) {
+        const int e = lane + 32 * j;
+        score[j] = e < E ? lg[j] + (p.bias ? p.bias[e] : 0.f) : -INFINITY;
+        m = fmaxf(m, score[j]);
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(full, m, o));
+      float sum = 0.f;
+#pragma unroll
+      for (int j = 0; j < EPL; ++j) {
+        prob[j] = (lane + 32 * j) < E ? expf(score[j] - m) : 0.f;
+        sum += prob[j];
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(full, sum, o);
+#pragma unroll
+      for (int j = 0; j < EPL; ++j) prob[j] /= sum;
+    } else {
+#pragma unroll
+      for (int j = 0; j < EPL; ++j) {
+        const int e = lane + 32 * j;
+        if (e < E) {
+          prob[j] = 1.f / (1.f + expf(-lg[j]));
+          score[j] = prob[j] + (p.bias ? p.bias[e] : 0.f);
+          scr[e] = score[j];
+        } else {
+          prob[j] = 0.f;
+          score[j] = -INFINITY;
+        }
+      }
+      __syncwarp();
+      // group score: the sum of the group's two largest selection scores
+      float gs = -INFINITY;
+      if (lane < p.n_group) {
+        float b1 = -INFINITY, b2 = -INFINITY;
+        for (int q = 0; q < G; ++q) {
+          const float v = scr[lane * G + q];
+          if (v > b1) { b2 = b1; b1 = v; } else if (v > b2) { b2 = v; }
+        }
+        gs = b1 + b2;
+      }
+      __syncwarp();
+      uint32_t keep = 0;
+      for (int r = 0; r < p.topk_group; ++r) {
+        const bool live = lane < p.n_group && !((keep >> lane) & 1u);
+        float v = live ? gs : -INFINITY;
+        int gi = live ? lane : 0x7fffffff;
+        warp_argmax_f(v, gi);
+        keep |= 1u << (gi & 31);
+      }
+#pragma unroll
+      for (int j = 0; j < EPL; ++j) {
+        const int e = lane + 32 * j;
+        if (e < E && !((keep >> (e / G)) & 1u)) score[j] = -INFINITY;
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < EPL; ++j)
+      if (lane + 32 * j < E) pr[tl * E + lane + 32 * j] = prob[j];
+
+    // the k choices (lane r keeps choice r): top-k by score, ties to the lower
+    // index, or the recorded ids (an id outside [0, E) or already taken is a
+    // bad route: weight 0, status flagged)
+    uint32_t taken = 0;
+    int my_e = -1;
+    bool my_ok = false;
+    for (int r = 0; r < p.k; ++r) {
+      int bi;
+      if (p.forced) {
+        bi = p.forced[(size_t)t * p.k + r];
+      } else {
+        float bv = -INFINITY;
+        bi = 0x7fffffff;
+#pragma unroll
+        for (int j = 0; j < EPL; ++j) {
+          const int e = lane + 32 * j;
+          if (e < E && !((taken >> j) & 1u) && (score[j] > bv || (score[j] == bv && e < bi))) {
+            bv = score[j];
+            bi = e;
+          }
+        }
+        warp_argmax_f(bv, bi);
+      }
+      bool again = false;
+#pragma unroll
+      for (int j = 0; j < EPL; ++j)
+        if (lane + 32 * j == bi && bi >= 0 && bi < E) {
+          again = (taken >> j) & 1u;
+          taken |= 1u << j;
+        }
+      again = __any_sync(full, again);
+      if (p.forced && lane == 0) {
+        if (bi < 0 || bi >= E) record_status(p.status, kDevBadExpertId);
+        else if (again) record_status(p.status, kDevDuplicateId);
+      }
+      if (lane == r) {
+        my_e = bi;
+        my_ok = bi >= 0 && bi < E && !again;
+      }
+    }
+
+    // exact logits of the chosen experts, eight per pass over the row
+    double my_l = 0.0;
+    for (int j0 = 0; j0 < p.k; j0 += 8) {
+      int ids[8];
+      bool valid[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        ids[j] = __shfl_sync(full, my_e, (j0 + j) & 31);
+        valid[j] = __shfl_sync(full, my_ok ? 1 : 0, (j0 + j) & 31) != 0 && j0 + j < p.k;
+      }
+      const double part = exact_logits8(p, t, ids, valid, lane);
+      // slot j of this pass sits on lane ((j >> 2) & 1) * 16 + ((j >> 1) & 1) * 8 + (j & 1) * 4
+      const int j = lane - j0;
+      const int src = j >= 0 && j < 8 ? (((j >> 2) & 1) << 4) | (((j >> 1) & 1) << 3) | ((j & 1) << 2) : 0;
+      const double got = __shfl_sync(full, part, src);
+      if (j >= 0 && j < 8) my_l = got;
+    }
+    // weights from the exact logits; key = the exact selection score (slot order)
+    double wv = 0.0, key = -INFINITY;
+    if (lane < p.k && my_ok) {
+      const double b = p.bias ? (double)p.bias[my_e] : 0.0;
+      if (softmax) {
+        wv = my_l + b;
+        key = wv;
+      } else {
+        wv = 1.0 / (1.0 + exp(-my_l));
+        key = wv + b;
+      }
+    }
+    if (softmax) {
+      double m = lane < p.k && my_ok ? wv : -INFINITY;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) m = fmax(m, __shfl_xor_sync(full, m, o));
+      wv = lane < p.k && my_ok ? exp(wv - m) : 0.0;
+    }
+    double tot = lane < p.k ? wv : 0.0;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) tot += __shfl_xor_sync(full, tot, o);
+    double wout;
+    if (softmax) wout = p.norm ? wv / fmax(tot, 1e-12) : wv;
+    else wout = (p.norm ? wv / (tot + 1e-20) : wv) * p.scaling;
+    int slot = lane;
+    if (!p.forced) {
+      slot = 0;
+      for (int j = 0; j < p.k; ++j) {
+        const double kj = __shfl_sync(full, key, j);
+        const int ej = __shfl_sync(full, my_e, j);
+        if (kj > key || (kj == key && ej < my_e)) ++slot;
+      }
+    }
+    if (lane < p.k) {
+      p.ids[(size_t)t * p.k + slot] = my_e;
+      p.wts[(size_t)t * p.k + slot] = (float)wout;
+    }
+  }
+  // the block's probability sums, tokens added in order
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += 32 * WPB) {
+    double sum = 0.0;
+    for (int tl = 0; tl < TPB; ++tl) sum += (double)pr[tl * E + e];
+    p.part[(size_t)blockIdx.x * E + e] = sum;
+  }
+}
+
 // prob_sum[e] = sum over 32-token groups in a fixed order: a block per 32
-// experts; warp w adds groups w, w + 8, w + 16, ... (four running sums per
-// lane, loads in flight together), then the eight warp sums are added in warp
-// order.  Deterministic for a given T and E.
-constexpr int FIN_WARPS = 8;
+// experts; warp w adds groups w, w + 32, w + 64, ... with eight loads in
+// flight, then the 32 warp sums are added in warp order.  Deterministic for a
+// given T and E.
+constexpr int FIN_WARPS = 32;
+constexpr int FIN_UNROLL = 8;
 __global__ void __launch_bounds__(32 * FIN_WARPS) route_finalize(const double *part, int nb, int E, float *prob_sum) {
   pdl_enter();
   __shared__ double ws[FIN_WARPS][32];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int e = blockIdx.x * 32 + lane;
-  double s[4] = {0.0, 0.0, 0.0, 0.0};
+  double s = 0.0;
   if (e < E) {
-    int b = warp, u = 0;
-    for (; b < nb; b += FIN_WARPS, u = (u + 1) & 3) s[u] += part[(size_t)b * E + e];
+    for (int b0 = warp; b0 < nb; b0 += FIN_WARPS * FIN_UNROLL) {
+      double v[FIN_UNROLL];
+#pragma unroll
+      for (int u = 0; u < FIN_UNROLL; ++u) {
+        const int b = b0 + u * FIN_WARPS;
+        v[u] = b < nb ? part[(size_t)b * E + e] : 0.0;
+      }
+#pragma unroll
+      for (int u = 0; u < FIN_UNROLL; ++u) s += v[u];
+    }
   }
-  ws[warp][lane] = (s[0] + s[1]) + (s[2] + s[3]);
+  ws[warp][lane] = s;
   __syncthreads();
   if (warp == 0 && e < E) {
     double t = 0.0;
@@ -710,7 +1011,29 @@ cudaError_t launch_wide(const RouteParams &p, const RoutePlan &plan, cudaStream_
 }
 
 
+template <int EPL, int TPB, int WPB>
+cudaError_t launch_refine_tpb(const RouteParams &p, cudaStream_t s) {
+  const size_t smem = sizeof(float) * ((size_t)TPB * p.E + (size_t)WPB * p.E);
+  auto kern = route_select_refine<EPL, TPB, WPB>;
+  cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (err != cudaSuccess) return err;
+  launch_pdl(kern, (p.T + TPB - 1) / TPB, 32 * WPB, smem, s, p);
+  return cudaGetLastError();
+}
+
+// tokens per block as the probability-sum rows were sized (select_tokens_per_block)
+template <int EPL>
+cudaError_t launch_refine_epl(const RouteParams &p, cudaStream_t s) {
+  return select_tokens_per_block(p.T) == 8 ? launch_refine_tpb<EPL, 8, 8>(p, s) : launch_refine_tpb<EPL, 32, 16>(p, s);
+}
+
 cudaError_t launch_select(const RouteParams &p, cudaStream_t s) {
+  if (p.refine) {
+    if (p.E <= 32) return launch_refine_epl<1>(p, s);
+    if (p.E <= 64) return launch_refine_epl<2>(p, s);
+    if (p.E <= 128) return launch_refine_epl<4>(p, s);
+    return launch_refine_epl<8>(p, s);
+  }
   if (p.E <= 32) return launch_select_epl<1>(p, s);
   if (p.E <= 64) return launch_select_epl<2>(p, s);
   if (p.E <= 128) return launch_select_epl<4>(p, s);

@@ -2,29 +2,28 @@
 //
 // The gate of the "Mixture of Experts" blog (route / Router.route) and of
 // Edge0 "MoE Spec and Routing" is an fp32 linear map x W_r^T.  For bf16 tokens
-// it runs here as three bf16 tcgen05 GEMMs whose sum is the fp32 product:
-// every fp32 weight w is split into w = hi + mid + lo, three bf16 values
-// carrying successive 8-bit slices of its significand (the residuals are exact
-// in fp32), and a bf16 token times a bf16 slice is exact.  The tensor core
-// then sums products with less than fp32 precision, and an fp32 accumulator
-// left running over thousands of products drifts by more than the 1e-4
-// selection margin (measured at d = 7168); so the accumulator is flushed into
-// float64 registers every FLUSH K-blocks and restarted (double-buffered), which
-// keeps the logit error near 1e-6: far inside the selection margin and the
-// prob-sum bound, but not the 1e-6 bound on the routing weights.  The
-// selection pass therefore recomputes the k chosen logits of every token
-// exactly (float64 products and sums) before weighting.
+// it runs here as two bf16 tcgen05 GEMMs: every fp32 weight w is split into
+// w = hi + lo + r, hi = bf16(w) and lo = bf16(w - hi) carrying the top 16 bits
+// of its significand, and a bf16 token times a bf16 slice is exact.  The
+// dropped residual |r| <= 2^-17 |w| moves a logit at d = 7168 by about 1e-5
+// (rms 8e-6 for the workloads' N(0, 0.02) weights), and the tensor core's own
+// sums, flushed into float64 registers every FLUSH K-blocks (an fp32
+// accumulator left running over thousands of products drifts much further),
+// add about 1e-6: selection-grade logits, far inside the 1e-4 selection margin
+// and the 1e-5 prob-sum bound.  The routing weights need 1e-6 relative, so the
+// selection pass recomputes the k chosen logits of every token exactly
+// (float64 products and sums) before weighting.
 //
 // Grid: (128-token tile, NTE-expert tile, hidden slice).  Per CTA:
 //   warp 0      TMA producer: per K-block the token tile (128 x 64 bf16) and
-//               the three weight-slice tiles (NTE x 64 bf16), 128-byte swizzle;
+//               the two weight-slice tiles (NTE x 64 bf16), 128-byte swizzle;
 //   warp 1      TMEM owner and single-thread MMA issuer (kind::f16, M = 128,
 //               N = NTE, K = 16), fp32 accumulators double-buffered per flush;
 //   warps 2-9   epilogue: two warps per TMEM lane quarter, each half the expert
 //               columns in float64 registers; the slice's sums go to
 //               logits[slice][token][expert].
 // The selection pass then adds the slices in order (route_select).  Every
-// mbarrier wait is bounded (2 s of %globaltimer); on expiry the CTA records a
+// mbarrier wait is bounded by %globaltimer (2 s unless moe_set_wait_timeout_ns says otherwise); on expiry the CTA records a
 // status, drains its own copies and MMAs, frees TMEM and exits.
 #include "common.cuh"
 
@@ -36,18 +35,18 @@ namespace {
 
 constexpr int TM = 128;                 // tokens per tile (MMA M)
 constexpr int BK = 64;                  // K per block
-constexpr int STAGES = 3;
+constexpr int STAGES = 4;
+constexpr int NSPLIT = 2;               // bf16 slices of the fp32 router weight
 constexpr int FLUSH = 2;                // K-blocks per fp32 accumulation before the float64 add
 constexpr int EPI_WARPS = 8;
 constexpr int THREADS = 32 * (2 + EPI_WARPS);
-constexpr uint64_t TIMEOUT_NS = 2000000000ull;
 constexpr uint64_t DRAIN_NS = 200000000ull;
 
 template <int NTE>
 struct TcShape {
   static constexpr int A_BYTES = TM * BK * 2;            // 16 KiB token tile
   static constexpr int B_BYTES = NTE * BK * 2;           // one weight slice tile
-  static constexpr int STAGE_BYTES = A_BYTES + 3 * B_BYTES;
+  static constexpr int STAGE_BYTES = A_BYTES + NSPLIT * B_BYTES;
   static constexpr int CPW = NTE / 2;                    // expert columns per epilogue warp
   static constexpr uint32_t TMEM_COLS = 2 * NTE < 32 ? 32 : 2 * NTE;   // two accumulators
   // kind::f16: D fp32, A/B bf16, both K-major, N = NTE, M = 128
@@ -56,6 +55,7 @@ struct TcShape {
 };
 
 struct TcRouteParams {
+  uint64_t timeout_ns;        // bound on every barrier wait (moe_set_wait_timeout_ns)
   int T, E, d;
   int e_pad;            // weight-slice rows per slice (E rounded up to the expert tile)
   int kb_total;         // K-blocks of the hidden dimension
@@ -99,14 +99,15 @@ __device__ __forceinline__ uint64_t global_ns() {
   asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
   return t;
 }
-__device__ __forceinline__ bool wait_bounded(uint64_t *bar, uint32_t parity, volatile int *abort_flag, int *status,
-                                             int code) {
+__device__ __forceinline__ bool wait_bounded(uint64_t *bar, uint32_t parity, volatile int *abort_flag,
+                                             int *status, int code, uint64_t limit_ns) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_ns();
   uint32_t spins = 0;
   while (!mbar_try_wait(bar, parity)) {
     if (*abort_flag) return false;
-    if ((++spins & 31u) == 0 && global_ns() - t0 > TIMEOUT_NS) {
+    // the clock is read every 32 polls, or every poll under a limit below 1 us
+    if (((++spins & 31u) == 0 || limit_ns < 1000u) && global_ns() - t0 > limit_ns) {
       *abort_flag = 1;
       record_status(status, code);
       return false;
@@ -182,8 +183,8 @@ __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.
 
 // ---------------------------------------------------------------- weight split
 // w (fp32) -> hi, mid, lo (bf16, round to nearest even each) with
-// hi + mid + lo = w: each residual is exact in fp32.  Rows E..e_pad-1 are 0.
-// Layout [3][e_pad][d].
+// hi = bf16(w), lo = bf16(w - hi) (the residual is exact in fp32).  Rows
+// E..e_pad-1 are 0.  Layout [NSPLIT][e_pad][d].
 __global__ void split_router_weights(const float *__restrict__ w, int E, int e_pad, int d,
                                      __nv_bfloat16 *__restrict__ out) {
   pdl_enter();
@@ -192,12 +193,8 @@ __global__ void split_router_weights(const float *__restrict__ w, int E, int e_p
     const int e = (int)(i / d);
     const float v = e < E ? w[i] : 0.f;
     const __nv_bfloat16 hi = __float2bfloat16_rn(v);
-    const float r1 = v - __bfloat162float(hi);
-    const __nv_bfloat16 mid = __float2bfloat16_rn(r1);
-    const float r2 = r1 - __bfloat162float(mid);
     out[i] = hi;
-    out[n + i] = mid;
-    out[2 * n + i] = __float2bfloat16_rn(r2);
+    out[n + i] = __float2bfloat16_rn(v - __bfloat162float(hi));
   }
 }
 
@@ -250,7 +247,7 @@ route_tc_gemm(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ 
       bool ok = true;
       for (; it < kb_n; ++it) {
         const int s = it % STAGES;
-        if (!wait_bounded(&st->empty[s], ((it / STAGES) & 1) ^ 1, abort_flag, p.status, kDevTimeoutProducer)) {
+        if (!wait_bounded(&st->empty[s], ((it / STAGES) & 1) ^ 1, abort_flag, p.status, kDevTimeoutProducer, p.timeout_ns)) {
           ok = false;
           break;
         }
@@ -260,7 +257,7 @@ route_tc_gemm(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ 
         mbar_expect_tx(&st->full[s], S::STAGE_BYTES);
         tma_load_2d(smem_u32(sp), &mapX, fb, kx, t0);
 #pragma unroll
-        for (int part = 0; part < 3; ++part)
+        for (int part = 0; part < NSPLIT; ++part)
           tma_load_2d(smem_u32(sp + S::A_BYTES + part * S::B_BYTES), &mapW, fb, kx, part * p.e_pad + e0);
       }
       if (!ok) {
@@ -277,12 +274,12 @@ route_tc_gemm(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ 
       for (int it = 0; it < kb_n && ok; ++it) {
         const int chunk = it / FLUSH, first = it % FLUSH == 0;
         const uint32_t buf = chunk & 1, use = chunk >> 1;
-        if (first && !wait_bounded(&st->acc_empty[buf], (use & 1) ^ 1, abort_flag, p.status, kDevTimeoutMma)) {
+        if (first && !wait_bounded(&st->acc_empty[buf], (use & 1) ^ 1, abort_flag, p.status, kDevTimeoutMma, p.timeout_ns)) {
           ok = false;
           break;
         }
         const int s = it % STAGES;
-        if (!wait_bounded(&st->full[s], (it / STAGES) & 1, abort_flag, p.status, kDevTimeoutMma)) {
+        if (!wait_bounded(&st->full[s], (it / STAGES) & 1, abort_flag, p.status, kDevTimeoutMma, p.timeout_ns)) {
           ok = false;
           break;
         }
@@ -291,7 +288,7 @@ route_tc_gemm(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ 
         const uint64_t da = sw128_desc(sa);
         const uint32_t dt = tmem_base + buf * NTE;
 #pragma unroll
-        for (int part = 0; part < 3; ++part) {
+        for (int part = 0; part < NSPLIT; ++part) {
           const uint64_t db = sw128_desc(sa + S::A_BYTES + part * S::B_BYTES);
 #pragma unroll
           for (int kk = 0; kk < BK / 16; ++kk)
@@ -318,7 +315,7 @@ route_tc_gemm(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ 
     const int n_chunks = (kb_n + FLUSH - 1) / FLUSH;
     for (int chunk = 0; chunk < n_chunks; ++chunk) {
       const uint32_t buf = chunk & 1, use = chunk >> 1;
-      if (!wait_bounded(&st->acc_full[buf], use & 1, abort_flag, p.status, kDevTimeoutEpilogue)) {
+      if (!wait_bounded(&st->acc_full[buf], use & 1, abort_flag, p.status, kDevTimeoutEpilogue, p.timeout_ns)) {
         ok = false;
         break;
       }
@@ -389,7 +386,7 @@ cudaError_t run_tc(const moe_config &c, const void *x, const __nv_bfloat16 *wspl
   using S = TcShape<NTE>;
   CUtensorMap mx, mw;
   cudaError_t err = make_map(&mx, x, (uint64_t)c.hidden, (uint64_t)c.num_tokens, TM);
-  if (err == cudaSuccess) err = make_map(&mw, wsplit, (uint64_t)c.hidden, (uint64_t)3 * e_pad, NTE);
+  if (err == cudaSuccess) err = make_map(&mw, wsplit, (uint64_t)c.hidden, (uint64_t)NSPLIT * e_pad, NTE);
   if (err != cudaSuccess) return err;
   TcRouteParams p;
   p.T = c.num_tokens;
@@ -400,6 +397,7 @@ cudaError_t run_tc(const moe_config &c, const void *x, const __nv_bfloat16 *wspl
   p.kb_per_slice = kb_per_slice;
   p.logits = logits;
   p.status = status;
+  p.timeout_ns = wait_timeout_ns();
   const size_t smem = 1024 + (size_t)STAGES * S::STAGE_BYTES + sizeof(TcShared);
   auto kern = route_tc_gemm<NTE>;
   err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -425,7 +423,7 @@ TcRoutePlan tc_route_plan(const moe_config &c) {
   ks = ks < 1 ? 1 : (ks > max_ks ? max_ks : ks);
   t.kb_per_slice = (kb_total + ks - 1) / ks;
   t.ks = (kb_total + t.kb_per_slice - 1) / t.kb_per_slice;   // no empty slice
-  t.wsplit_bytes = sizeof(__nv_bfloat16) * 3 * (size_t)t.e_pad * c.hidden;
+  t.wsplit_bytes = sizeof(__nv_bfloat16) * NSPLIT * (size_t)t.e_pad * c.hidden;
   return t;
 }
 

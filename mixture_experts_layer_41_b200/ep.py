@@ -42,27 +42,22 @@ from . import api
 class Dispatched:
     """What a rank sends: expert-sorted rows, the kept count of every expert
     (reshaped [world, E/N]: row q is what rank q receives), and what the local
-    combine needs later."""
-    rows: torch.Tensor          # [R, d]
-    counts: torch.Tensor        # [world, E_local] int32 (host)
+    combine needs later.  ``rows`` may be longer than the kept rows (the
+    dispatch buffer); the first sum(counts) rows are sent."""
+    rows: torch.Tensor          # [>= R, d]
+    counts: torch.Tensor        # [world, E_local] int32 (on the rows' device)
     slot_row: torch.Tensor      # [T, k]
     topk_w: torch.Tensor        # [T, k]
     topk_ids: torch.Tensor      # [T, k]
     x: torch.Tensor             # [T, d] (for the shared expert)
 
 
-def local_expert_ids(recv_counts: torch.Tensor) -> torch.Tensor:
-    """Local expert id of every received row: the rows from source s arrive as
-    recv_counts[s, 0] rows of local expert 0, then recv_counts[s, 1] of expert
-    1, ... (the sender's expert order)."""
-    world, e_local = recv_counts.shape
-    ids = torch.arange(e_local, dtype=torch.int32).repeat(world)
-    return torch.repeat_interleave(ids, recv_counts.reshape(-1).to(torch.int64))
-
-
-def split_sizes(counts: torch.Tensor) -> list:
-    """Rows per peer from a [world, E_local] count table."""
-    return [int(v) for v in counts.sum(dim=1).tolist()]
+def split_sizes_pair(send_counts: torch.Tensor, recv_counts: torch.Tensor):
+    """Rows per peer to send and to receive, from the [world, E_local] count
+    tables: the one device-to-host read the row all-to-all needs (its split
+    sizes are host integers)."""
+    both = torch.stack([send_counts.sum(dim=1), recv_counts.sum(dim=1)]).to(torch.int64).cpu()
+    return [int(v) for v in both[0].tolist()], [int(v) for v in both[1].tolist()]
 
 
 class DeviceOps:
@@ -110,10 +105,8 @@ class DeviceOps:
         api.moe_route(c, x, self.w_router, self.bias, self.ids, self.wts, self.prob_sum, self.ws)
         api.moe_permute(c, x, self.ids, self.wts, self.offsets, self.perm_token, self.perm_w, self.slot_row,
                         self.x_perm, self.stats, self.ws)
-        kept = self.stats["kept_counts"].cpu()
-        rows = int(kept.sum())
-        return Dispatched(self.x_perm[:rows], kept.view(self.world, self.e_local), self.slot_row, self.wts,
-                          self.ids, x)
+        return Dispatched(self.x_perm, self.stats["kept_counts"].view(self.world, self.e_local), self.slot_row,
+                          self.wts, self.ids, x)
 
     def expert(self, rows: torch.Tensor, recv_counts: torch.Tensor) -> torch.Tensor:
         n = rows.shape[0]
@@ -122,7 +115,8 @@ class DeviceOps:
             return out
         cfg = self._local_cfg(n)
         i32 = dict(dtype=torch.int32, device=self.dev)
-        ids = local_expert_ids(recv_counts).to(self.dev).view(n, 1)
+        ids = torch.empty((n, 1), **i32)
+        api.moe_ep_local_ids(recv_counts.to(device=self.dev, dtype=torch.int32).contiguous(), n, ids)
         ones = torch.ones((n, 1), dtype=torch.float32, device=self.dev)
         off = torch.empty(self.e_local + 1, **i32)
         perm_token = torch.empty(n, **i32)
@@ -155,15 +149,14 @@ class DeviceOps:
 
 def exchange_counts(counts: torch.Tensor, group=None) -> torch.Tensor:
     """All-to-all of the [world, E_local] kept-count tables: row q of the result
-    is what rank q sends here, per local expert."""
+    is what rank q sends here, per local expert.  Stays on the tensors'
+    device (NCCL: the GPU; gloo: the host)."""
     import torch.distributed as dist
     world, e_local = counts.shape
     send = counts.reshape(-1).to(torch.int32).contiguous()
     recv = torch.empty_like(send)
-    if _needs_device(group):
-        send, recv = send.cuda(), recv.cuda()
     dist.all_to_all_single(recv, send, group=group)
-    return recv.cpu().view(world, e_local)
+    return recv.view(world, e_local)
 
 
 def exchange_rows(rows: torch.Tensor, send_sizes: Sequence[int], recv_sizes: Sequence[int],
@@ -177,11 +170,6 @@ def exchange_rows(rows: torch.Tensor, send_sizes: Sequence[int], recv_sizes: Seq
     return out
 
 
-def _needs_device(group) -> bool:
-    import torch.distributed as dist
-    return dist.get_backend(group) == "nccl"
-
-
 class EPLayer:
     """One rank's share of an expert-parallel layer: ``forward`` runs the four
     steps with the collectives of ``group``."""
@@ -193,8 +181,8 @@ class EPLayer:
     def forward(self, x: torch.Tensor) -> torch.Tensor:
         disp = self.ops.dispatch(x)
         recv_counts = exchange_counts(disp.counts, self.group)
-        send_sizes, recv_sizes = split_sizes(disp.counts), split_sizes(recv_counts)
-        rows_in = exchange_rows(disp.rows, send_sizes, recv_sizes, self.group)
+        send_sizes, recv_sizes = split_sizes_pair(disp.counts, recv_counts)
+        rows_in = exchange_rows(disp.rows[:sum(send_sizes)], send_sizes, recv_sizes, self.group)
         rows_out = self.ops.expert(rows_in, recv_counts)
         back = exchange_rows(rows_out, recv_sizes, send_sizes, self.group)
         return self.ops.combine(back, disp)
@@ -206,7 +194,7 @@ def emulate(shards: Sequence, xs: Sequence[torch.Tensor]) -> list:
     slicing and concatenating the blocks (for a single device)."""
     world = len(shards)
     disps = [s.dispatch(x) for s, x in zip(shards, xs)]
-    sizes = [split_sizes(dp.counts) for dp in disps]                 # sizes[src][dst]
+    sizes = [split_sizes_pair(dp.counts, dp.counts)[0] for dp in disps]    # sizes[src][dst]
     blocks = []
     for dp, sz in zip(disps, sizes):
         starts = [sum(sz[:q]) for q in range(world)]

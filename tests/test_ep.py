@@ -24,11 +24,41 @@ from oracle import moe_oracle as O
 WORLD = 2
 
 
+def local_expert_ids(recv_counts: torch.Tensor) -> torch.Tensor:
+    """Host reference of moe_ep_local_ids: rows from source s arrive as
+    recv_counts[s, 0] rows of local expert 0, then recv_counts[s, 1] of
+    expert 1, ... (the sender's expert order)."""
+    world, e_local = recv_counts.shape
+    ids = torch.arange(e_local, dtype=torch.int32).repeat(world)
+    return torch.repeat_interleave(ids, recv_counts.reshape(-1).to(torch.int64))
+
+
 def test_local_expert_ids_and_splits():
     counts = torch.tensor([[2, 0, 1], [1, 3, 0]], dtype=torch.int32)
-    ids = ep.local_expert_ids(counts)
-    assert ids.tolist() == [0, 0, 2, 0, 1, 1, 1]
-    assert ep.split_sizes(counts) == [3, 4]
+    assert local_expert_ids(counts).tolist() == [0, 0, 2, 0, 1, 1, 1]
+    recv = torch.tensor([[1, 1, 1], [0, 0, 5]], dtype=torch.int32)
+    assert ep.split_sizes_pair(counts, recv) == ([3, 4], [3, 5])
+
+
+@pytest.mark.gpu
+def test_ep_local_ids_kernel():
+    """moe_ep_local_ids against the host reference, with empty segments,
+    a zero-row call and rows past the counts (-1)."""
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA GPU")
+    from mixture_experts_layer_41_b200 import api
+    gen = torch.Generator().manual_seed(3)
+    for world, e_local in ((2, 4), (4, 32), (8, 32), (1, 7)):
+        counts = torch.randint(0, 40, (world, e_local), generator=gen, dtype=torch.int32)
+        counts[0, 1 % e_local] = 0
+        n = int(counts.sum())
+        ids = torch.full((n + 5, 1), 99, dtype=torch.int32, device="cuda")
+        api.moe_ep_local_ids(counts.cuda(), n + 5, ids)
+        torch.cuda.synchronize()
+        got = ids.view(-1).cpu()
+        assert torch.equal(got[:n], local_expert_ids(counts)), (world, e_local)
+        assert (got[n:] == -1).all()
+        api.moe_ep_local_ids(counts.cuda(), 0, ids)
 
 
 # ---------------------------------------------------------------- host operations on the oracle
@@ -56,7 +86,7 @@ class OracleOps:
                              torch.from_numpy(r["ids"]), x)
 
     def expert(self, rows, recv_counts):
-        ids = ep.local_expert_ids(recv_counts).numpy()
+        ids = local_expert_ids(recv_counts).numpy()
         out = np.zeros(rows.shape, dtype=np.float64)
         rf = rows.numpy()
         for e in range(self.e_local):

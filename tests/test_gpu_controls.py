@@ -322,13 +322,14 @@ Q4 = {
 }
 
 
-@pytest.mark.parametrize("kernel", ["mma", "tc"])
+@pytest.mark.parametrize("kernel", ["i8", "mma", "tc"])
 @pytest.mark.parametrize("name", sorted(Q4))
 def test_q4_kernels_match_oracle(name, kernel, monkeypatch):
-    """Both 4-bit grouped FFN kernels (warp-level mma.sync fragments and
-    tcgen05 with the weight operand in TMEM), forced in turn, against the
-    oracle on every token (the GPU's own routing, so only the experts and
-    the combine are compared)."""
+    """Every 4-bit grouped FFN kernel (warp-level 8-bit integer MMAs on the
+    codes, warp-level bf16 MMAs on dequantised weights, tcgen05 with the
+    weight operand in TMEM), forced in turn, against the oracle on every
+    token (the GPU's own routing, so only the experts and the combine are
+    compared)."""
     from gpu_harness import check_output
     monkeypatch.setenv("MOE_Q4_KERNEL", kernel)
     run = Run(Q4[name], seed=23).staged()
@@ -336,7 +337,7 @@ def test_q4_kernels_match_oracle(name, kernel, monkeypatch):
     check_output(run)
 
 
-@pytest.mark.parametrize("case", ["bf16", "bf16_pair", "q4_mma", "q4_tc"])
+@pytest.mark.parametrize("case", ["bf16", "bf16_pair", "q4_i8", "q4_mma", "q4_tc"])
 def test_grouped_ffn_repairs_bad_offsets(case, monkeypatch):
     """Decreasing group offsets (every value inside [0, T*k]) are clamped to a
     non-decreasing copy, the call completes, and the workspace reports the
@@ -355,3 +356,42 @@ def test_grouped_ffn_repairs_bad_offsets(case, monkeypatch):
     api.moe_grouped_ffn(run.cfg, run.x_perm, bad, run.weights, run.y_perm, run.ws)
     torch.cuda.synchronize()
     assert run.status() == L.MOE_ERR_DEVICE
+
+
+# ---------------------------------------------------------------- bounded-wait failure path
+
+@pytest.mark.parametrize("kernel", ["tc", "q4_tc"])
+def test_barrier_wait_timeout_reports_and_recovers(kernel, monkeypatch):
+    """The tensor-core kernels' failure path, made to run out on purpose: with
+    a 1 ns bound on barrier waits the first wait that is not already
+    satisfied gives up; the call reports MOE_ERR_DEVICE with the waiting
+    site, the kernel lets its issued copies and MMAs land, frees its tensor
+    memory and returns, so the context stays usable; with the default bound
+    restored, the same workspace gives the oracle's result."""
+    if kernel == "tc":
+        w = workload("mixtral_prefill", T=700, d=512, F=640)
+    else:
+        monkeypatch.setenv("MOE_Q4_KERNEL", "tc")
+        # long enough reductions that some barrier wait is still open when it is checked
+        w = workload("decode_q4", T=200, d=2048, F=1024, E=8, k=2)
+    from gpu_harness import check_output
+    run = Run(w, seed=9)
+    c = run.cfg
+    api.moe_route(c, run.inp["x"], run.inp["w_router"], run.bias, run.ids, run.wts, run.prob_sum, run.ws)
+    api.moe_permute(c, run.inp["x"], run.ids, run.wts, run.offsets, run.perm_token, run.perm_w, run.slot_row,
+                    run.x_perm, run.stats, run.ws)
+    torch.cuda.synchronize()
+    assert run.status() == 0
+    try:
+        api.moe_set_wait_timeout_ns(1)
+        api.moe_grouped_ffn(c, run.x_perm, run.offsets, run.weights, run.y_perm, run.ws)
+        st = run.status()
+        text = L.lib().moe_last_error().decode()
+    finally:
+        api.moe_set_wait_timeout_ns(0)
+    assert st == L.MOE_ERR_DEVICE, st
+    assert "timed out" in text, text
+    # the context and the workspace are still good: a normal call succeeds
+    run.staged()
+    assert run.status() == 0
+    check_output(run, routing="gpu")

@@ -241,7 +241,7 @@ def test_router_shapes(name):
 
 def test_token_sharded_capacity_on_one_gpu():
     """Two token shards of one batch, dispatched one after the other on one
-    GPU with moe_expert_counts -> shard_base -> moe_permute_shard: the kept
+    GPU with moe_expert_counts -> the gathered counts -> moe_permute_shard: the kept
     slots and the layer output equal the oracle's whole-batch in-order
     dispatch (the sharded layer's single exchange is the count all-gather)."""
     from mixture_experts_layer_41_b200.inputs import make_inputs, to_host
@@ -272,7 +272,6 @@ def test_token_sharded_capacity_on_one_gpu():
     out = torch.empty((w.T, w.d), dtype=torch.bfloat16, device=dev)
     slot_all = []
     for r, ((lo, hi), (cfg, ws, x, ids, wts)) in enumerate(zip(halves, parts)):
-        base = api.shard_base_from_counts(gathered, r).contiguous()
         n = hi - lo
         i32 = dict(dtype=torch.int32, device=dev)
         off = torch.empty(w.E + 1, **i32)
@@ -283,7 +282,8 @@ def test_token_sharded_capacity_on_one_gpu():
         y_perm = torch.empty_like(x_perm)
         stats = dict(raw_counts=torch.empty(w.E, **i32), kept_counts=torch.empty(w.E, **i32),
                      dropped=torch.empty(4, **i32))
-        api.moe_permute_shard(cfg, x, ids, wts, base, cap, off, perm_token, perm_w, slot_row, x_perm, stats, ws)
+        api.moe_permute_shard(cfg, x, ids, wts, gathered, r, cap, off, perm_token, perm_w, slot_row, x_perm, stats,
+                              ws)
         api.moe_grouped_ffn(cfg, x_perm, off, weights, y_perm, ws)
         api.moe_combine(cfg, y_perm, slot_row, wts, None, out[lo:hi])
         torch.cuda.synchronize()

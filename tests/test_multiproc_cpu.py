@@ -41,7 +41,9 @@ def _shard_worker(rank, port, ids, cap, out_q):
     lo, hi = rank * T // WORLD, (rank + 1) * T // WORLD
     mine = ids[lo:hi]
     raw = torch.from_numpy(np.bincount(mine.reshape(-1), minlength=E).astype(np.int32))
-    base = api.exchange_shard_base(raw).numpy()
+    gathered_counts = api.exchange_counts(raw).numpy()       # [world, E], row q = shard q
+    assert gathered_counts.shape == (WORLD, E) and np.array_equal(gathered_counts[rank], raw.numpy())
+    base = gathered_counts[:rank].sum(axis=0)                # the prefix moe_permute_shard forms
     # this shard's kept slots under the shard rule (plain loops, token order)
     seen = np.zeros(E, dtype=np.int64)
     kept = []
@@ -57,7 +59,7 @@ def _shard_worker(rank, port, ids, cap, out_q):
     t = torch.tensor([1.0 + rank])
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     if rank == 0:
-        out_q.put((gathered, float(t.item()), base.tolist()))
+        out_q.put((gathered, float(t.item()), [int(v) for v in base]))
     dist.barrier()
     dist.destroy_process_group()
 
@@ -87,10 +89,3 @@ def test_sharded_capacity_matches_whole_batch(cf):
     assert tmax == 2.0
     if cap is not None:
         assert len(union) < T * k      # the skew makes the first expert overflow
-
-
-def test_shard_base_prefix():
-    counts = torch.tensor([[3, 0, 2], [1, 4, 0], [2, 2, 2]], dtype=torch.int32)
-    assert api.shard_base_from_counts(counts, 0).tolist() == [0, 0, 0]
-    assert api.shard_base_from_counts(counts, 1).tolist() == [3, 0, 2]
-    assert api.shard_base_from_counts(counts, 2).tolist() == [4, 4, 2]
