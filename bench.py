@@ -49,6 +49,8 @@ def parse_args():
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-hash", action="store_true", help="skip the inputs' SHA-256 digests")
+    ap.add_argument("--fused-gather", action="store_true",
+                    help="bf16 experts read their token rows inside the grouped GEMM (no x_perm copy)")
     ap.add_argument("--cpu-sample", type=int, default=0, help="tokens in the oracle sample (0 = auto)")
     return ap.parse_args()
 
@@ -181,7 +183,10 @@ def ffn_kernel_file(w) -> str:
     if w.weight_format == "q4_affine_g64":
         if w.d % 128 or w.F % 128:
             return "ffn_q4.cu"
-        return "ffn_q4_i8.cu" if w.T * w.k <= 16 * w.E else "ffn_q4_tc.cu"
+        kern = os.environ.get("MOE_Q4_KERNEL", "")
+        if kern in ("mma", "tc"):
+            return {"mma": "ffn_q4_mma.cu", "tc": "ffn_q4_tc.cu"}[kern]
+        return "ffn_q4_mma.cu" if w.T * w.k <= 16 * w.E else "ffn_q4_tc.cu"
     return "ffn_simt.cu" if w.dtype == "f32" else "ffn_tc.cu"
 
 
@@ -397,7 +402,7 @@ def run_ours(args):
                           routed_scaling=w.routed_scaling if w.router == "sigmoid_group" else 1.0,
                           n_group=w.n_group, topk_group=w.topk_group, capacity_factor=w.capacity_factor,
                           act=w.act, act_dtype=w.dtype, weight_dtype=wf, shared_intermediate=w.shared_F,
-                          aux_alpha=w.aux_alpha)
+                          aux_alpha=w.aux_alpha, fused_gather=args.fused_gather)
     weights = {k: inp[k] for k in ("w1", "w2", "w3", "s1", "s2", "s3", "b1", "b2", "b3", "ws1", "ws2", "ws3")
                if inp.get(k) is not None}
     for i in "123":
@@ -587,7 +592,9 @@ def run_ours(args):
         "vs_baseline": None, "dtype": "bf16" if w.dtype == "bf16" else w.dtype, "data": "synthetic",
         "config": dict(config_of(w, world),
                        l2="inputs larger than L2: every step streams all touched expert weights "
-                          f"({costs['bytes'] / 1e9:.2f} GB) from HBM"),
+                          f"({costs['bytes'] / 1e9:.2f} GB) from HBM",
+                       **({"fused_gather": True} if args.fused_gather else {}),
+                       **({"paired_sms": True} if os.environ.get("MOE_TC_PAIR") == "1" else {})),
         "roofline": roof,
         "gemm_phases": gemm_phases,
         "layer_roofline": {"frac": t_layer_roof / (ms_max * 1e-3), "roof_ms": t_layer_roof * 1e3,

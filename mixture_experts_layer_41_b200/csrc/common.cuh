@@ -141,7 +141,6 @@ __device__ __forceinline__ bool warp_group_offsets(const int32_t *src, int n, in
 }
 
 size_t route_logits_bytes(const moe_config &c);   // defined in router.cu
-size_t q4_i8_token_bytes(int rows, int d, int F);   // defined in ffn_q4_i8.cu
 
 // ---------------------------------------------------------------- workspace
 struct WsLayout {
@@ -168,7 +167,6 @@ struct WsLayout {
   size_t shared_out;   // act[T][d]
   size_t x_stage;      // act[T][d]   (moe_forward_host)
   size_t out_stage;    // act[T][d]
-  size_t q4_tokens;    // quantised token rows of the 4-bit integer-MMA path
   size_t total;
   size_t region_bytes[MOE_WS_REGION_COUNT];   // unpadded sizes of the moe_ws_region buffers
 };
@@ -230,7 +228,6 @@ inline WsLayout ws_layout(const moe_config &c) {
   L.shared_out = take(rb[MOE_WS_SHARED_OUT] = Fs ? es * T * d : 0);
   L.x_stage = take(es * T * d);
   L.out_stage = take(es * T * d);
-  L.q4_tokens = take(c.weight_dtype == MOE_Q4_AFFINE_G64 ? q4_i8_token_bytes((int)slots, (int)d, (int)F) : 0);
   L.total = off;
   return L;
 }
@@ -321,11 +318,6 @@ struct FfnArgs {
   const void *shared_w1, *shared_w2, *shared_w3;   // [F, d], [F, d], [d, F]
   void *shared_h;           // [shared_rows, F]
   void *shared_y;           // [shared_rows, d]
-  // 4-bit integer-MMA path: workspace for the quantised token rows
-  // (q4_i8_token_bytes), and the views of it the launches share
-  void *q4_scratch;
-  const void *q4_tokens;
-  const float *q4_tscale, *q4_tsum;
 };
 
 cudaError_t launch_ffn_simt_f32(const FfnArgs &a, cudaStream_t s);
@@ -336,9 +328,6 @@ bool q4_tc_supported(int d, int F);                                 // the tenso
 cudaError_t launch_ffn_q4_tc(const FfnArgs &a, cudaStream_t s);
 bool q4_mma_supported(int d, int F);                                // the warp-level 4-bit path's shapes
 cudaError_t launch_ffn_q4_mma(const FfnArgs &a, cudaStream_t s);
-bool q4_i8_supported(int d, int F);                                 // the 8-bit integer MMA path's shapes
-size_t q4_i8_token_bytes(int rows, int d, int F);                   // its workspace
-cudaError_t launch_ffn_q4_i8(const FfnArgs &a, cudaStream_t s);
 
 // Replaces the text moe_last_error() returns on this thread.
 void set_last_error_text(const char *text);

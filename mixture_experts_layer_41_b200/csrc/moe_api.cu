@@ -80,7 +80,6 @@ FfnArgs ffn_args(const moe_config &c, const WsLayout &L, void *ws) {
   a.F = c.intermediate;
   a.h = ws_ptr<char>(ws, L.h);
   a.status = ws_ptr<int>(ws, L.status);
-  a.q4_scratch = ws_ptr<char>(ws, L.q4_tokens);
   return a;
 }
 
@@ -107,18 +106,19 @@ bool shared_in_grouped_gemm(const moe_config &c) {
 }
 
 // 4-bit weights: decode-sized groups (a few token rows per expert) go to the
-// warp-level integer-MMA kernel, whose 4-token MMA blocks fit them; larger
-// groups to the tcgen05 kernel.  MOE_Q4_KERNEL=i8 / mma / tc in the
-// environment forces one (mma: warp-level bf16 MMAs on dequantised weights).
-cudaError_t run_q4(const FfnArgs &a, cudaStream_t s) {
+// warp-level kernel, whose 8-token MMA blocks fit them; larger groups to the
+// tcgen05 kernel.  MOE_Q4_KERNEL=mma / tc in the environment forces one.
+bool use_q4_mma(const FfnArgs &a) {
+  if (!q4_mma_supported(a.d, a.F)) return false;
   const char *env = getenv("MOE_Q4_KERNEL");
-  const bool i8 = q4_i8_supported(a.d, a.F), mma = q4_mma_supported(a.d, a.F), tc = q4_tc_supported(a.d, a.F);
-  if (env && strcmp(env, "mma") == 0 && mma) return launch_ffn_q4_mma(a, s);
-  if (env && strcmp(env, "i8") == 0 && i8) return launch_ffn_q4_i8(a, s);
-  if (env && strcmp(env, "tc") == 0 && tc) return launch_ffn_q4_tc(a, s);
-  if (i8 && (long long)a.rows_cap <= 16LL * a.E) return launch_ffn_q4_i8(a, s);
-  if (tc) return launch_ffn_q4_tc(a, s);
-  return i8 ? launch_ffn_q4_i8(a, s) : launch_ffn_q4(a, s);
+  if (env && strcmp(env, "mma") == 0) return true;
+  if (env && strcmp(env, "tc") == 0) return !q4_tc_supported(a.d, a.F);
+  return (long long)a.rows_cap <= 16LL * a.E;
+}
+
+cudaError_t run_q4(const FfnArgs &a, cudaStream_t s) {
+  if (use_q4_mma(a)) return launch_ffn_q4_mma(a, s);
+  return q4_tc_supported(a.d, a.F) ? launch_ffn_q4_tc(a, s) : launch_ffn_q4(a, s);
 }
 
 cudaError_t run_ffn(const FfnArgs &a, cudaStream_t s) {

@@ -580,16 +580,16 @@ route_tiled(RouteParams p) {
 // route_select: one warp per token, TPB tokens per block (32, or 8 when a
 // 32-token grid would leave more than half of the SMs idle); block b writes
 // probability-sum row b of p.part.
+// The selection of block-tile `tile` (tokens tile*TPB ..): sums the float64
+// partial logits of its tokens in slice order, selects with one warp per
+// token and writes probability-sum row `tile`.
 template <int EPL, int TPB>
-__global__ void __launch_bounds__(32 * TPB, 1)
-route_select(RouteParams p) {
-  pdl_enter();
-  extern __shared__ __align__(16) unsigned char smem_raw[];
+__device__ __forceinline__ void select_tile(const RouteParams &p, int tile, unsigned char *smem_raw) {
   double *lgs = reinterpret_cast<double *>(smem_raw);                 // [TPB][E] summed logits
   double *dscr = lgs + TPB * p.E;                                    // [TPB][kMaxExperts]
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int E = p.E;
-  const int tb = blockIdx.x * TPB;
+  const int tb = tile * TPB;
   constexpr int NT = 32 * TPB;
   // every thread sums the slices of 4 (token, expert) logits at a time, in
   // slice order, with the loads of a slice in flight together
@@ -639,8 +639,16 @@ route_select(RouteParams p) {
   for (int e = threadIdx.x; e < E; e += NT) {
     double sum = 0.0;
     for (int w = 0; w < TPB; ++w) sum += dscr[w * E + e];
-    p.part[(size_t)blockIdx.x * E + e] = sum;
+    p.part[(size_t)tile * E + e] = sum;
   }
+}
+
+template <int EPL, int TPB>
+__global__ void __launch_bounds__(32 * TPB, 1)
+route_select(RouteParams p) {
+  pdl_enter();
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  select_tile<EPL, TPB>(p, blockIdx.x, smem_raw);
 }
 
 // ---------------------------------------------------------------- tensor-core plan: selection + exact weights
@@ -659,6 +667,23 @@ route_select(RouteParams p) {
 //    these exact logits, as in the CUDA-core router.
 // Router replay (forced ids) takes the recorded ids instead of the top-k.
 
+// A float32 w as the float64 w * 2^-896, built with integer operations
+// (shifts and one multiply-add) instead of a float conversion: the fp32
+// exponent and significand bits are placed in the float64 fields unchanged,
+// without the exponent re-bias, and the sign moved to bit 63.  Exact for every
+// finite w, subnormals and zeros included (the 2^-896 scale maps the fp32
+// range onto the float64 normal range); a sum of products with these values
+// is multiplied by 2^896 at the end.  Half of the chosen logits' weights are
+// converted this way and half with the conversion instruction, so the
+// integer and the conversion pipes share the work.
+__device__ __forceinline__ double f32_as_f64_scaled(float w) {
+  const uint32_t u = __float_as_uint(w);
+  const uint32_t t = u >> 3;                       // sign lands in bit 28
+  const uint32_t hi = t + (u >> 31) * 0x70000000u; // ... moved to bit 31
+  return __hiloint2double((int)hi, (int)(u << 29));
+}
+constexpr double kTwoTo896 = 0x1p896;
+
 // Exact logits of up to 8 chosen experts (ids[j], valid[j]) of bf16 token t.
 // Returns, on every lane, the sum for slot ((lane >> 4) & 1) * 4 +
 // ((lane >> 3) & 1) * 2 + ((lane >> 2) & 1).
@@ -676,27 +701,41 @@ __device__ __forceinline__ double exact_logits8(const RouteParams &p, int t, con
   for (int i = lane; i < nchunk; i += 32) {
     const uint4 xv = __ldg(xr + i);
     const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
+    // the token's 8 elements, widened once for all chosen experts
     double xd[8];
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
       xd[2 * u] = (double)__uint_as_float(xw[u] << 16);
       xd[2 * u + 1] = (double)__uint_as_float(xw[u] & 0xFFFF0000u);
     }
-    float4 wv[8][2];
 #pragma unroll
-    for (int j = 0; j < 8; ++j)
-      if (valid[j]) {
-        wv[j][0] = __ldg(wr[j] + 2 * i);
-        wv[j][1] = __ldg(wr[j] + 2 * i + 1);
+    for (int h = 0; h < 8; h += 4) {               // four chosen experts' loads in flight at a time
+    float4 wv[4][2];
+#pragma unroll
+    for (int jj = 0; jj < 4; ++jj)
+      if (valid[h + jj]) {
+        wv[jj][0] = __ldg(wr[h + jj] + 2 * i);
+        wv[jj][1] = __ldg(wr[h + jj] + 2 * i + 1);
       }
 #pragma unroll
-    for (int j = 0; j < 8; ++j)
-      if (valid[j]) {
-        const float wf[8] = {wv[j][0].x, wv[j][0].y, wv[j][0].z, wv[j][0].w,
-                             wv[j][1].x, wv[j][1].y, wv[j][1].z, wv[j][1].w};
-#pragma unroll
-        for (int u = 0; u < 8; ++u) acc[j] = fma(xd[u], (double)wf[u], acc[j]);
+    for (int jj = 0; jj < 4; ++jj)
+      if (valid[h + jj]) {
+        const int j = h + jj;
+        // elements 0-3 against the integer-built w * 2^-896 (their sum is
+        // scaled back by 2^896, exactly), elements 4-7 against the converted w;
+        // every product is exact in float64
+        double lo = 0.0;
+        lo = fma(xd[0], f32_as_f64_scaled(wv[jj][0].x), lo);
+        lo = fma(xd[1], f32_as_f64_scaled(wv[jj][0].y), lo);
+        lo = fma(xd[2], f32_as_f64_scaled(wv[jj][0].z), lo);
+        lo = fma(xd[3], f32_as_f64_scaled(wv[jj][0].w), lo);
+        acc[j] = fma(lo, kTwoTo896, acc[j]);
+        acc[j] = fma(xd[4], (double)wv[jj][1].x, acc[j]);
+        acc[j] = fma(xd[5], (double)wv[jj][1].y, acc[j]);
+        acc[j] = fma(xd[6], (double)wv[jj][1].z, acc[j]);
+        acc[j] = fma(xd[7], (double)wv[jj][1].w, acc[j]);
       }
+    }
   }
   // halving exchanges: lanes split by bit 4, then 3, then 2 keep half of the slots
   const unsigned full = 0xffffffffu;
@@ -1138,6 +1177,7 @@ cudaError_t launch_route(const moe_config &c, const void *x, const float *w_rout
   p.logits = logits;
   p.ks = plan.ks;
   p.kchunk = plan.kchunk;
+
   cudaError_t err;
   if (plan.tc) {
     __nv_bfloat16 *wsplit =

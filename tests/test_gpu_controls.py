@@ -322,14 +322,13 @@ Q4 = {
 }
 
 
-@pytest.mark.parametrize("kernel", ["i8", "mma", "tc"])
+@pytest.mark.parametrize("kernel", ["mma", "tc"])
 @pytest.mark.parametrize("name", sorted(Q4))
 def test_q4_kernels_match_oracle(name, kernel, monkeypatch):
-    """Every 4-bit grouped FFN kernel (warp-level 8-bit integer MMAs on the
-    codes, warp-level bf16 MMAs on dequantised weights, tcgen05 with the
-    weight operand in TMEM), forced in turn, against the oracle on every
-    token (the GPU's own routing, so only the experts and the combine are
-    compared)."""
+    """Both 4-bit grouped FFN kernels (warp-level mma.sync fragments and
+    tcgen05 with the weight operand in TMEM), forced in turn, against the
+    oracle on every token (the GPU's own routing, so only the experts and
+    the combine are compared)."""
     from gpu_harness import check_output
     monkeypatch.setenv("MOE_Q4_KERNEL", kernel)
     run = Run(Q4[name], seed=23).staged()
@@ -337,7 +336,7 @@ def test_q4_kernels_match_oracle(name, kernel, monkeypatch):
     check_output(run)
 
 
-@pytest.mark.parametrize("case", ["bf16", "bf16_pair", "q4_i8", "q4_mma", "q4_tc"])
+@pytest.mark.parametrize("case", ["bf16", "bf16_pair", "q4_mma", "q4_tc"])
 def test_grouped_ffn_repairs_bad_offsets(case, monkeypatch):
     """Decreasing group offsets (every value inside [0, T*k]) are clamped to a
     non-decreasing copy, the call completes, and the workspace reports the
