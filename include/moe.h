@@ -233,6 +233,13 @@ moe_status moe_workspace_status(const void *ws, moe_stream_t stream);
  *   MOE_WS_Y_PERM      y_perm [T*k, d] act_dtype
  *   MOE_WS_SHARED_H    the shared expert's intermediate [T, Fs] (0 bytes without one)
  *   MOE_WS_SHARED_OUT  the shared expert's output [T, d] (0 bytes without one)
+ *   MOE_WS_ROUTER_LOGITS  the router's float64 logits partials [ks][T][E] when
+ *                      its plan computes them in the workspace (bf16 batches of
+ *                      512 tokens or more, or the split CUDA-core pass; the
+ *                      logit of (t, e) is the sum over the ks slices), else 0
+ *                      bytes.  On the integer tensor-core plan each logit is
+ *                      within |dx_t|_1 |w_e|_inf + |xhat_t|_2 |dw_e|_2 +
+ *                      |x2_t|_2 |w3_e|_2 of x_t . w_e (see moe_route).
  * Rows at or past off[E] (and, in x_perm / h / y_perm, every row when the
  * layer routes nothing) are never written.  *offset is a byte offset from the
  * start of ws (256-byte aligned) and *bytes the region's size; the layout is
@@ -248,7 +255,8 @@ typedef enum moe_ws_region {
   MOE_WS_Y_PERM = 6,
   MOE_WS_SHARED_H = 7,
   MOE_WS_SHARED_OUT = 8,
-  MOE_WS_REGION_COUNT = 9
+  MOE_WS_ROUTER_LOGITS = 9,
+  MOE_WS_REGION_COUNT = 10
 } moe_ws_region;
 moe_status moe_workspace_region(const moe_config *cfg, int32_t region, size_t *offset, size_t *bytes);
 

@@ -25,7 +25,7 @@ MOE_PHASE_START, MOE_PHASE_ROUTE, MOE_PHASE_PERMUTE, MOE_PHASE_FFN1, MOE_PHASE_F
     MOE_PHASE_COMBINE, MOE_PHASE_COUNT = range(8)
 # moe_ws_region
 MOE_WS_OFFSETS, MOE_WS_PERM_TOKEN, MOE_WS_PERM_W, MOE_WS_SLOT_ROW, MOE_WS_X_PERM, MOE_WS_H, MOE_WS_Y_PERM, \
-    MOE_WS_SHARED_H, MOE_WS_SHARED_OUT, MOE_WS_REGION_COUNT = range(10)
+    MOE_WS_SHARED_H, MOE_WS_SHARED_OUT, MOE_WS_ROUTER_LOGITS, MOE_WS_REGION_COUNT = range(11)
 # moe_router_kind
 MOE_ROUTER_SOFTMAX_TOPK = 0
 MOE_ROUTER_SIGMOID_GROUP = 1

@@ -117,7 +117,8 @@ def moe_workspace_status(ws: torch.Tensor, stream=None) -> int:
 
 _REGIONS = {"offsets": L.MOE_WS_OFFSETS, "perm_token": L.MOE_WS_PERM_TOKEN, "perm_w": L.MOE_WS_PERM_W,
             "slot_row": L.MOE_WS_SLOT_ROW, "x_perm": L.MOE_WS_X_PERM, "h": L.MOE_WS_H, "y_perm": L.MOE_WS_Y_PERM,
-            "shared_h": L.MOE_WS_SHARED_H, "shared_out": L.MOE_WS_SHARED_OUT}
+            "shared_h": L.MOE_WS_SHARED_H, "shared_out": L.MOE_WS_SHARED_OUT,
+            "router_logits": L.MOE_WS_ROUTER_LOGITS}
 
 
 def moe_workspace_region(cfg: moe_config, region: str):

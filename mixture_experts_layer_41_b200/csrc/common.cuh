@@ -140,7 +140,8 @@ __device__ __forceinline__ bool warp_group_offsets(const int32_t *src, int n, in
   return __any_sync(full, bad);
 }
 
-size_t route_logits_bytes(const moe_config &c);   // defined in router.cu
+size_t route_logits_bytes(const moe_config &c);       // defined in router.cu
+size_t route_logits_f64_bytes(const moe_config &c);   // its float64 logits partials [ks][T][E]
 
 // ---------------------------------------------------------------- workspace
 struct WsLayout {
@@ -206,6 +207,7 @@ inline WsLayout ws_layout(const moe_config &c) {
   L.status = take(256);
   L.route_part = take(sizeof(double) * route_part_rows(c) * E);
   L.route_logits = take(route_logits_bytes(c));
+  L.region_bytes[MOE_WS_ROUTER_LOGITS] = route_logits_f64_bytes(c);
   L.blk_counts = take(sizeof(int32_t) * perm_blocks(c) * E);
   L.blk_base = take(sizeof(int32_t) * perm_blocks(c) * E);
   L.local_rank = take(sizeof(int32_t) * slots);
@@ -253,7 +255,8 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 // selection pass -- for batches too small to fill the GPU with whole rows.
 struct RoutePlan {
   bool split;
-  bool tc;          // bf16 tokens: logits on the tensor cores (router_tc.cu), then the selection pass
+  bool tc;          // bf16 tokens: selection-grade logits on the bf16 tensor cores (router_tc.cu), exact re-weighting
+  bool i8;          // bf16 tokens: bounded-error logits on the integer tensor cores (router_i8.cu)
   int ks, kchunk;
   int tpw;          // tokens per warp of the tiled kernel (4 or 8)
 };
@@ -268,6 +271,32 @@ TcRoutePlan tc_route_plan(const moe_config &c);
 // Splits w_router into wsplit and writes float64 logits partials [ks][T][E].
 cudaError_t launch_route_tc_logits(const moe_config &c, const void *x, const float *w_router,
                                    __nv_bfloat16 *wsplit, double *logits, int *status, cudaStream_t s);
+
+// Integer tensor-core logits: expert tile width, padded sizes, hidden slices.
+struct I8RoutePlan {
+  int n, e_pad, d_pad, ks, kb_per_slice;
+};
+// Its workspace: float64 logits partials [ks][T][E], the weight's digit planes
+// [4][e_pad][d_pad], the scale exponents and the error-bound norms.
+struct I8RouteBuffers {
+  double *logits;
+  int8_t *wdig;
+  int *sx, *sw;
+  double *xst;    // [T][4]: |dx|_1, |xhat|_2, |x2|_2, 0
+  double *wst;    // [e_pad][4]: |w|_inf, |dw|_2, |w3|_2, 0
+  int *xcnt;      // [T] elements each token row's digits round (dx != 0)
+  int *xidx;      // [T][round_list] the first round_list of them: index
+  double *xdx;    // [T][round_list] and dx (x - xhat)
+  int round_list;
+  int *flag_count; // tokens listed for the exact recomputation (zeroed by the preparation pass)
+  int *flag_list;  // [T]
+};
+bool i8_route_supported(const moe_config &c);
+I8RoutePlan i8_route_plan(const moe_config &c);
+size_t i8_route_bytes(const moe_config &c, const I8RoutePlan &t);
+I8RouteBuffers i8_route_buffers(const moe_config &c, const I8RoutePlan &t, void *base);
+cudaError_t launch_route_i8_logits(const moe_config &c, const void *x, const float *w_router,
+                                   const I8RoutePlan &t, const I8RouteBuffers &b, int *status, cudaStream_t s);
 
 // logits == nullptr forbids the split pass (no workspace for it).
 cudaError_t launch_route(const moe_config &c, const void *x, const float *w_router,

@@ -405,6 +405,7 @@ moe_status moe_workspace_region(const moe_config *cfg, int32_t region, size_t *o
     case MOE_WS_Y_PERM: begin = L.y_perm; end = L.shared_h; break;
     case MOE_WS_SHARED_H: begin = L.shared_h; end = L.shared_out; break;
     case MOE_WS_SHARED_OUT: begin = L.shared_out; end = L.x_stage; break;
+    case MOE_WS_ROUTER_LOGITS: begin = L.route_logits; end = L.blk_counts; break;
     default: return MOE_ERR_INVALID_ARG;
   }
   *offset = begin;

@@ -35,6 +35,8 @@
 #include "common.cuh"
 
 #include <math.h>
+#include <stdlib.h>
+#include <string.h>
 
 namespace moe {
 namespace {
@@ -59,6 +61,22 @@ struct RouteParams {
   const int32_t *forced;   // [T][k] replayed expert ids, or null to select
   int *status;             // device status word (bad / repeated forced ids)
   int refine;              // logits are selection-grade only: weight from exact chosen logits
+  // approx: the logits carry a bound per (token, expert),
+  //   xst[t] . wst[e] = |dx_t|_1 |w_e|_inf + |xhat_t|_2 |dw_e|_2 + |x2_t|_2 |w3_e|_2
+  // (router_i8.cu); a token's chosen logits are recomputed exactly when a
+  // chosen bound exceeds tau or two chosen experts' keys lie within their
+  // bounds of each other.
+  int approx;
+  const double *xst, *wst;
+  double tau;
+  // the x-rounding term is corrected exactly (sum of dx * w over the listed
+  // rounded elements) when a token lists all of them (xcnt <= round_list)
+  const int *xcnt, *xidx;
+  const double *xdx;
+  int round_list;
+  // tokens whose chosen logits need the exact recomputation are appended
+  // here (the count zeroed by the preparation pass) for route_refine_listed
+  int *flag_count, *flag_list;
 };
 
 __device__ __forceinline__ void argmax_merge(double &v, int &i, double ov, int oi) {
@@ -86,34 +104,103 @@ __device__ __forceinline__ double warp_max(double v) {
   return v;
 }
 
-// Exact logit of bf16 token t and expert e: every product is exact in
-// float64 (8-bit by 24-bit significands), summed per lane in index order and
-// then across the warp.  d % 8 == 0 (bf16 rows are 16-byte vectors).
-__device__ __forceinline__ double exact_logit(const RouteParams &p, int t, int e, int lane) {
+// A float32 w as the float64 w * 2^-896, built with integer operations
+// (shifts and one multiply-add) instead of a float conversion: the fp32
+// exponent and significand bits are placed in the float64 fields unchanged,
+// without the exponent re-bias, and the sign moved to bit 63.  Exact for every
+// finite w, subnormals and zeros included (the 2^-896 scale maps the fp32
+// range onto the float64 normal range); a sum of products with these values
+// is multiplied by 2^896 at the end.  Half of the chosen logits' weights are
+// converted this way and half with the conversion instruction, so the
+// integer and the conversion pipes share the work.
+__device__ __forceinline__ double f32_as_f64_scaled(float w) {
+  const uint32_t u = __float_as_uint(w);
+  const uint32_t t = u >> 3;                       // sign lands in bit 28
+  const uint32_t hi = t + (u >> 31) * 0x70000000u; // ... moved to bit 31
+  return __hiloint2double((int)hi, (int)(u << 29));
+}
+constexpr double kTwoTo896 = 0x1p896;
+
+// Exact logits of up to 8 chosen experts (ids[j], valid[j]) of bf16 token t.
+// Returns, on every lane, the sum for slot ((lane >> 4) & 1) * 4 +
+// ((lane >> 3) & 1) * 2 + ((lane >> 2) & 1).
+__device__ __noinline__ double exact_logits8(const RouteParams &p, int t, const int (&ids)[8],
+                                                const bool (&valid)[8], int lane) {
   const uint4 *xr = reinterpret_cast<const uint4 *>(static_cast<const __nv_bfloat16 *>(p.x) + (size_t)t * p.d);
-  const float4 *wr = reinterpret_cast<const float4 *>(p.w + (size_t)e * p.d);
-  double s = 0.0;
-  // four 16-byte loads of x and eight of w in flight per lane
-#pragma unroll 4
-  for (int i = lane; i < p.d / 8; i += 32) {
+  const float4 *wr[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) wr[j] = reinterpret_cast<const float4 *>(p.w + (size_t)(valid[j] ? ids[j] : 0) * p.d);
+  double acc[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) acc[j] = 0.0;
+  const int nchunk = p.d / 8;
+#pragma unroll 1
+  for (int i = lane; i < nchunk; i += 32) {
     const uint4 xv = __ldg(xr + i);
-    const float4 w0 = __ldg(wr + 2 * i), w1 = __ldg(wr + 2 * i + 1);
     const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
-    const float wf[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+    // the token's 8 elements, widened once for all chosen experts
+    double xd[8];
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
-      s = fma((double)__uint_as_float(xw[u] << 16), (double)wf[2 * u], s);
-      s = fma((double)__uint_as_float(xw[u] & 0xFFFF0000u), (double)wf[2 * u + 1], s);
+      xd[2 * u] = (double)__uint_as_float(xw[u] << 16);
+      xd[2 * u + 1] = (double)__uint_as_float(xw[u] & 0xFFFF0000u);
+    }
+#pragma unroll
+    for (int h = 0; h < 8; h += 4) {               // four chosen experts' loads in flight at a time
+    float4 wv[4][2];
+#pragma unroll
+    for (int jj = 0; jj < 4; ++jj)
+      if (valid[h + jj]) {
+        wv[jj][0] = __ldg(wr[h + jj] + 2 * i);
+        wv[jj][1] = __ldg(wr[h + jj] + 2 * i + 1);
+      }
+#pragma unroll
+    for (int jj = 0; jj < 4; ++jj)
+      if (valid[h + jj]) {
+        const int j = h + jj;
+        // elements 0-3 against the integer-built w * 2^-896 (their sum is
+        // scaled back by 2^896, exactly), elements 4-7 against the converted w;
+        // every product is exact in float64
+        double lo = 0.0;
+        lo = fma(xd[0], f32_as_f64_scaled(wv[jj][0].x), lo);
+        lo = fma(xd[1], f32_as_f64_scaled(wv[jj][0].y), lo);
+        lo = fma(xd[2], f32_as_f64_scaled(wv[jj][0].z), lo);
+        lo = fma(xd[3], f32_as_f64_scaled(wv[jj][0].w), lo);
+        acc[j] = fma(lo, kTwoTo896, acc[j]);
+        acc[j] = fma(xd[4], (double)wv[jj][1].x, acc[j]);
+        acc[j] = fma(xd[5], (double)wv[jj][1].y, acc[j]);
+        acc[j] = fma(xd[6], (double)wv[jj][1].z, acc[j]);
+        acc[j] = fma(xd[7], (double)wv[jj][1].w, acc[j]);
+      }
     }
   }
-  return warp_sum(s);
+  // halving exchanges: lanes split by bit 4, then 3, then 2 keep half of the slots
+  const unsigned full = 0xffffffffu;
+  const int b4 = (lane >> 4) & 1, b3 = (lane >> 3) & 1, b2 = (lane >> 2) & 1;
+  double h4[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const double keep = b4 ? acc[i + 4] : acc[i];
+    const double send = b4 ? acc[i] : acc[i + 4];
+    h4[i] = keep + __shfl_xor_sync(full, send, 16);
+  }
+  double h3[2];
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {
+    const double keep = b3 ? h4[i + 2] : h4[i];
+    const double send = b3 ? h4[i] : h4[i + 2];
+    h3[i] = keep + __shfl_xor_sync(full, send, 8);
+  }
+  double h2 = (b2 ? h3[1] : h3[0]) + __shfl_xor_sync(full, b2 ? h3[0] : h3[1], 4);
+  h2 += __shfl_xor_sync(full, h2, 2);
+  h2 += __shfl_xor_sync(full, h2, 1);
+  return h2;
 }
 
 // Scores, selection and weights of token t, whose logits (without bias) sit
 // in l[j] for expert lane + 32 j.  Adds the token's probabilities to psum.
-// wscr: this warp's shared scratch row of kMaxExperts doubles.  With
-// p.refine the logits only choose the experts (and give the probability
-// sums); the chosen experts' logits are recomputed exactly for the weights.
+// wscr: this warp's shared scratch row of kMaxExperts doubles.  (The
+// tensor-core plans select in route_select_refine instead.)
 template <int EPL>
 __device__ __forceinline__ void select_token(const RouteParams &p, int t, const double (&lg)[EPL],
                                              double (&psum)[EPL], double *wscr, int lane) {
@@ -189,8 +276,7 @@ __device__ __forceinline__ void select_token(const RouteParams &p, int t, const 
   // taken gets weight 0 and flags the status word)
   uint32_t taken = 0;
   int my_e = -1;
-  double my_w = 0.0, my_key = 0.0;
-  bool my_ok = false;
+  double my_w = 0.0;
   for (int r = 0; r < p.k; ++r) {
     int bi = 0x7fffffff;
     if (p.forced) {
@@ -219,48 +305,15 @@ __device__ __forceinline__ void select_token(const RouteParams &p, int t, const 
       else if (lane == 0 && again) record_status(p.status, kDevDuplicateId);
     }
     wv = __shfl_sync(0xffffffffu, wv, bi & 31);
-    double key = 0.0;
-    if (p.refine && bi >= 0 && bi < E && !again) {
-      // softmax keeps the exact logit (with the logit bias) for the
-      // renormalisation below; sigmoid scores it at once (its bias only
-      // selects).  key: the exact selection score, for the slot order
-      const double l = exact_logit(p, t, bi, lane);
-      const double b = p.bias ? (double)p.bias[bi] : 0.0;
-      if (p.router == MOE_ROUTER_SOFTMAX_TOPK) {
-        wv = l + b;
-        key = wv;
-      } else {
-        wv = 1.0 / (1.0 + exp(-l));
-        key = wv + b;
-      }
-    }
-    if (lane == r) { my_e = bi; my_w = wv; my_key = key; my_ok = bi >= 0 && bi < E && !again; }
-  }
-  if (p.refine && p.router == MOE_ROUTER_SOFTMAX_TOPK) {
-    // renormalised softmax over the chosen experts from their exact logits:
-    // p_j / sum_sel p = exp(l_j - m) / sum_sel exp(l_i - m)
-    const double m = warp_max(lane < p.k && my_ok ? my_w : -INFINITY);
-    my_w = lane < p.k && my_ok ? exp(my_w - m) : 0.0;
+    if (lane == r) { my_e = bi; my_w = wv; }
   }
   const double tot = warp_sum(lane < p.k ? my_w : 0.0);
   double wout;
   if (p.router == MOE_ROUTER_SOFTMAX_TOPK) wout = p.norm ? my_w / fmax(tot, 1e-12) : my_w;
   else wout = (p.norm ? my_w / (tot + 1e-20) : my_w) * p.scaling;
-  // slot order: the approximate logits chose the set; with refinement the
-  // chosen experts are ranked again by their exact scores (descending, ties
-  // to the lower index), as a selection on exact logits would order them
-  int slot = lane;
-  if (p.refine && !p.forced) {
-    slot = 0;
-    for (int j = 0; j < p.k; ++j) {
-      const double kj = __shfl_sync(0xffffffffu, my_key, j);
-      const int ej = __shfl_sync(0xffffffffu, my_e, j);
-      if (kj > my_key || (kj == my_key && ej < my_e)) ++slot;
-    }
-  }
   if (lane < p.k) {
-    p.ids[(size_t)t * p.k + slot] = my_e;
-    p.wts[(size_t)t * p.k + slot] = (float)wout;
+    p.ids[(size_t)t * p.k + lane] = my_e;
+    p.wts[(size_t)t * p.k + lane] = (float)wout;
   }
 }
 
@@ -583,14 +636,15 @@ route_tiled(RouteParams p) {
 // The selection of block-tile `tile` (tokens tile*TPB ..): sums the float64
 // partial logits of its tokens in slice order, selects with one warp per
 // token and writes probability-sum row `tile`.
-template <int EPL, int TPB>
+// TPB tokens per block, WPB warps (tokens warp, warp + WPB, ... in order).
+template <int EPL, int TPB, int WPB>
 __device__ __forceinline__ void select_tile(const RouteParams &p, int tile, unsigned char *smem_raw) {
   double *lgs = reinterpret_cast<double *>(smem_raw);                 // [TPB][E] summed logits
   double *dscr = lgs + TPB * p.E;                                    // [TPB][kMaxExperts]
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int E = p.E;
   const int tb = tile * TPB;
-  constexpr int NT = 32 * TPB;
+  constexpr int NT = 32 * WPB;
   // every thread sums the slices of 4 (token, expert) logits at a time, in
   // slice order, with the loads of a slice in flight together
   const int n = TPB * E;
@@ -618,15 +672,17 @@ __device__ __forceinline__ void select_tile(const RouteParams &p, int tile, unsi
 #pragma unroll
   for (int j = 0; j < EPL; ++j) psum[j] = 0.0;
   double *wscr = dscr + warp * kMaxExperts;
-  const int t = tb + warp;
-  if (t < p.T) {
+  for (int i = warp; i < TPB; i += WPB) {
+    const int t = tb + i;
+    if (t >= p.T) break;
     double lg[EPL];
 #pragma unroll
     for (int j = 0; j < EPL; ++j) {
       const int e = lane + 32 * j;
-      lg[j] = e < E ? lgs[warp * E + e] : 0.0;
+      lg[j] = e < E ? lgs[i * E + e] : 0.0;
     }
     select_token<EPL>(p, t, lg, psum, wscr, lane);
+    __syncwarp();
   }
   // the block's probability sums, warps added in order
   __syncthreads();
@@ -638,17 +694,17 @@ __device__ __forceinline__ void select_tile(const RouteParams &p, int tile, unsi
   __syncthreads();
   for (int e = threadIdx.x; e < E; e += NT) {
     double sum = 0.0;
-    for (int w = 0; w < TPB; ++w) sum += dscr[w * E + e];
+    for (int w = 0; w < WPB; ++w) sum += dscr[w * E + e];
     p.part[(size_t)tile * E + e] = sum;
   }
 }
 
-template <int EPL, int TPB>
-__global__ void __launch_bounds__(32 * TPB, 1)
+template <int EPL, int TPB, int WPB>
+__global__ void __launch_bounds__(32 * WPB, 1)
 route_select(RouteParams p) {
   pdl_enter();
   extern __shared__ __align__(16) unsigned char smem_raw[];
-  select_tile<EPL, TPB>(p, blockIdx.x, smem_raw);
+  select_tile<EPL, TPB, WPB>(p, blockIdx.x, smem_raw);
 }
 
 // ---------------------------------------------------------------- tensor-core plan: selection + exact weights
@@ -667,113 +723,21 @@ route_select(RouteParams p) {
 //    these exact logits, as in the CUDA-core router.
 // Router replay (forced ids) takes the recorded ids instead of the top-k.
 
-// A float32 w as the float64 w * 2^-896, built with integer operations
-// (shifts and one multiply-add) instead of a float conversion: the fp32
-// exponent and significand bits are placed in the float64 fields unchanged,
-// without the exponent re-bias, and the sign moved to bit 63.  Exact for every
-// finite w, subnormals and zeros included (the 2^-896 scale maps the fp32
-// range onto the float64 normal range); a sum of products with these values
-// is multiplied by 2^896 at the end.  Half of the chosen logits' weights are
-// converted this way and half with the conversion instruction, so the
-// integer and the conversion pipes share the work.
-__device__ __forceinline__ double f32_as_f64_scaled(float w) {
-  const uint32_t u = __float_as_uint(w);
-  const uint32_t t = u >> 3;                       // sign lands in bit 28
-  const uint32_t hi = t + (u >> 31) * 0x70000000u; // ... moved to bit 31
-  return __hiloint2double((int)hi, (int)(u << 29));
-}
-constexpr double kTwoTo896 = 0x1p896;
-
-// Exact logits of up to 8 chosen experts (ids[j], valid[j]) of bf16 token t.
-// Returns, on every lane, the sum for slot ((lane >> 4) & 1) * 4 +
-// ((lane >> 3) & 1) * 2 + ((lane >> 2) & 1).
-__device__ __forceinline__ double exact_logits8(const RouteParams &p, int t, const int (&ids)[8],
-                                                const bool (&valid)[8], int lane) {
-  const uint4 *xr = reinterpret_cast<const uint4 *>(static_cast<const __nv_bfloat16 *>(p.x) + (size_t)t * p.d);
-  const float4 *wr[8];
-#pragma unroll
-  for (int j = 0; j < 8; ++j) wr[j] = reinterpret_cast<const float4 *>(p.w + (size_t)(valid[j] ? ids[j] : 0) * p.d);
-  double acc[8];
-#pragma unroll
-  for (int j = 0; j < 8; ++j) acc[j] = 0.0;
-  const int nchunk = p.d / 8;
-#pragma unroll 1
-  for (int i = lane; i < nchunk; i += 32) {
-    const uint4 xv = __ldg(xr + i);
-    const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
-    // the token's 8 elements, widened once for all chosen experts
-    double xd[8];
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      xd[2 * u] = (double)__uint_as_float(xw[u] << 16);
-      xd[2 * u + 1] = (double)__uint_as_float(xw[u] & 0xFFFF0000u);
-    }
-#pragma unroll
-    for (int h = 0; h < 8; h += 4) {               // four chosen experts' loads in flight at a time
-    float4 wv[4][2];
-#pragma unroll
-    for (int jj = 0; jj < 4; ++jj)
-      if (valid[h + jj]) {
-        wv[jj][0] = __ldg(wr[h + jj] + 2 * i);
-        wv[jj][1] = __ldg(wr[h + jj] + 2 * i + 1);
-      }
-#pragma unroll
-    for (int jj = 0; jj < 4; ++jj)
-      if (valid[h + jj]) {
-        const int j = h + jj;
-        // elements 0-3 against the integer-built w * 2^-896 (their sum is
-        // scaled back by 2^896, exactly), elements 4-7 against the converted w;
-        // every product is exact in float64
-        double lo = 0.0;
-        lo = fma(xd[0], f32_as_f64_scaled(wv[jj][0].x), lo);
-        lo = fma(xd[1], f32_as_f64_scaled(wv[jj][0].y), lo);
-        lo = fma(xd[2], f32_as_f64_scaled(wv[jj][0].z), lo);
-        lo = fma(xd[3], f32_as_f64_scaled(wv[jj][0].w), lo);
-        acc[j] = fma(lo, kTwoTo896, acc[j]);
-        acc[j] = fma(xd[4], (double)wv[jj][1].x, acc[j]);
-        acc[j] = fma(xd[5], (double)wv[jj][1].y, acc[j]);
-        acc[j] = fma(xd[6], (double)wv[jj][1].z, acc[j]);
-        acc[j] = fma(xd[7], (double)wv[jj][1].w, acc[j]);
-      }
-    }
-  }
-  // halving exchanges: lanes split by bit 4, then 3, then 2 keep half of the slots
-  const unsigned full = 0xffffffffu;
-  const int b4 = (lane >> 4) & 1, b3 = (lane >> 3) & 1, b2 = (lane >> 2) & 1;
-  double h4[4];
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const double keep = b4 ? acc[i + 4] : acc[i];
-    const double send = b4 ? acc[i] : acc[i + 4];
-    h4[i] = keep + __shfl_xor_sync(full, send, 16);
-  }
-  double h3[2];
-#pragma unroll
-  for (int i = 0; i < 2; ++i) {
-    const double keep = b3 ? h4[i + 2] : h4[i];
-    const double send = b3 ? h4[i] : h4[i + 2];
-    h3[i] = keep + __shfl_xor_sync(full, send, 8);
-  }
-  double h2 = (b2 ? h3[1] : h3[0]) + __shfl_xor_sync(full, b2 ? h3[0] : h3[1], 4);
-  h2 += __shfl_xor_sync(full, h2, 2);
-  h2 += __shfl_xor_sync(full, h2, 1);
-  return h2;
-}
-
+// Warp arg-max of (v, i), ties to the lower index: two warp reductions on
+// an order-preserving integer image of v.
 __device__ __forceinline__ void warp_argmax_f(float &v, int &i) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    const float ov = __shfl_xor_sync(0xffffffffu, v, o);
-    const int oi = __shfl_xor_sync(0xffffffffu, i, o);
-    if (ov > v || (ov == v && oi < i)) { v = ov; i = oi; }
-  }
+  const uint32_t u = __float_as_uint(v);
+  const uint32_t key = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+  const uint32_t kmax = __reduce_max_sync(0xffffffffu, key);
+  i = __reduce_min_sync(0xffffffffu, key == kmax ? i : 0x7fffffff);
+  v = __uint_as_float((kmax & 0x80000000u) ? (kmax & 0x7fffffffu) : ~kmax);
 }
 
 // TPB tokens per block, WPB warps (TPB / WPB tokens per warp, in order).
 // Shared memory: the block's per-token probabilities [TPB][E] (fp32) and a
 // selection-score row per warp [WPB][E].
 template <int EPL, int TPB, int WPB>
-__global__ void __launch_bounds__(32 * WPB)
+__global__ void __launch_bounds__(32 * WPB, WPB <= 8 ? 2 : 1)
 route_select_refine(RouteParams p) {
   pdl_enter();
   extern __shared__ __align__(16) unsigned char smem_raw[];
@@ -795,16 +759,31 @@ route_select_refine(RouteParams p) {
         if (lane + 32 * j < E) pr[tl * E + lane + 32 * j] = 0.f;
       continue;
     }
-    // selection-grade logits: the hidden slices added in order
+    // the logits: the hidden slices added in order, the loads of four
+    // slices (all of the token's experts) in flight together; the float64
+    // sums stay for the chosen experts
     float lg[EPL];
+    double lgd[EPL];
 #pragma unroll
-    for (int j = 0; j < EPL; ++j) {
-      const int e = lane + 32 * j;
-      double v = 0.0;
-      if (e < E)
-        for (int q = 0; q < p.ks; ++q) v += p.logits[((size_t)q * p.T + t) * E + e];
-      lg[j] = (float)v;
+    for (int j = 0; j < EPL; ++j) lgd[j] = 0.0;
+#pragma unroll 4
+    for (int q = 0; q < p.ks; ++q) {
+      const double *row = p.logits + ((size_t)q * p.T + t) * E;
+#pragma unroll
+      for (int j = 0; j < EPL; ++j)
+        if (lane + 32 * j < E) lgd[j] += row[lane + 32 * j];
     }
+    // the token's bound factors, loaded while the selection runs
+    int xcnt = 0;
+    double xs0 = 0.0, xs1 = 0.0, xs2 = 0.0;
+    if (p.approx) {
+      xcnt = p.xcnt[t];
+      xs0 = p.xst[(size_t)t * 4];
+      xs1 = p.xst[(size_t)t * 4 + 1];
+      xs2 = p.xst[(size_t)t * 4 + 2];
+    }
+#pragma unroll
+    for (int j = 0; j < EPL; ++j) lg[j] = (float)lgd[j];
     float score[EPL], prob[EPL];
     if (softmax) {
       float m = -INFINITY;
@@ -875,6 +854,7 @@ route_select_refine(RouteParams p) {
     uint32_t taken = 0;
     int my_e = -1;
     bool my_ok = false;
+    double my_l = 0.0;
     for (int r = 0; r < p.k; ++r) {
       int bi;
       if (p.forced) {
@@ -893,13 +873,17 @@ route_select_refine(RouteParams p) {
         warp_argmax_f(bv, bi);
       }
       bool again = false;
+      double lv = 0.0;
 #pragma unroll
       for (int j = 0; j < EPL; ++j)
         if (lane + 32 * j == bi && bi >= 0 && bi < E) {
           again = (taken >> j) & 1u;
           taken |= 1u << j;
+          lv = lgd[j];
         }
       again = __any_sync(full, again);
+      lv = __shfl_sync(full, lv, bi & 31);
+      if (lane == r) my_l = lv;
       if (p.forced && lane == 0) {
         if (bi < 0 || bi >= E) record_status(p.status, kDevBadExpertId);
         else if (again) record_status(p.status, kDevDuplicateId);
@@ -910,9 +894,46 @@ route_select_refine(RouteParams p) {
       }
     }
 
-    // exact logits of the chosen experts, eight per pass over the row
-    double my_l = 0.0;
-    for (int j0 = 0; j0 < p.k; j0 += 8) {
+    // the chosen experts' logits: with bounded logits (approx) the float64
+    // sums, the x-rounding term added exactly where listed, and an exact
+    // recomputation only where a bound exceeds tau or two chosen keys lie
+    // within their bounds; selection-grade logits are always recomputed
+    bool exact = true;
+    if (p.approx) {
+      double bnd = 0.0, key = 0.0;
+      const bool mine = lane < p.k && my_ok;
+      if (mine) {
+        const double *ws = p.wst + (size_t)my_e * 4;
+        if (xcnt <= p.round_list) {
+          const size_t o = (size_t)t * p.round_list;
+          const float *wr = p.w + (size_t)my_e * p.d;
+          double corr = 0.0;
+          for (int q = 0; q < xcnt; ++q) corr = fma(p.xdx[o + q], (double)__ldg(wr + p.xidx[o + q]), corr);
+          my_l += corr;
+        } else {
+          bnd = xs0 * ws[0];
+        }
+        bnd += xs1 * ws[1] + xs2 * ws[2];
+        const double b = p.bias ? (double)p.bias[my_e] : 0.0;
+        key = softmax ? my_l + b : 1.0 / (1.0 + exp(-my_l)) + b;
+      }
+      bool need = mine && bnd > p.tau;
+      if (!p.forced)
+        for (int j = 0; j < p.k; ++j) {
+          const double kj = __shfl_sync(full, key, j), bj = __shfl_sync(full, bnd, j);
+          const bool okj = __shfl_sync(full, my_ok, j) && j < p.k;
+          // |key error| <= bound (softmax: key = logit + bias; sigmoid: a quarter of it)
+          if (mine && okj && j != lane && fabs(kj - key) <= bj + bnd) need = true;
+        }
+      exact = __any_sync(full, need);
+      if (exact) {
+        // the provisional weights below are replaced by route_refine_listed
+        if (lane == 0) p.flag_list[atomicAdd(p.flag_count, 1)] = t;
+        exact = false;
+      }
+    }
+    if (!p.approx) my_l = 0.0;
+    for (int j0 = 0; exact && j0 < p.k; j0 += 8) {
       int ids[8];
       bool valid[8];
 #pragma unroll
@@ -974,6 +995,123 @@ route_select_refine(RouteParams p) {
   }
 }
 
+// Exact re-weighting of the listed tokens (bounded-logit plan): a block per
+// token (grid-stride over the list), every thread a share of the hidden
+// dimension for eight chosen experts at a time (bf16 x fp32 products exact in
+// float64, float64 sums reduced in a fixed order), then warp 0 weights and
+// orders the slots from the exact logits as the selection pass would.
+constexpr int RL_THREADS = 256;
+__global__ void __launch_bounds__(RL_THREADS) route_refine_listed(RouteParams p) {
+  pdl_enter();
+  __shared__ double red[RL_THREADS / 32][8];
+  __shared__ double lsh[32];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const unsigned full = 0xffffffffu;
+  const int n = *p.flag_count;
+  const bool softmax = p.router == MOE_ROUTER_SOFTMAX_TOPK;
+  for (int j = blockIdx.x; j < n; j += gridDim.x) {
+    const int t = p.flag_list[j];
+    const uint4 *xr = reinterpret_cast<const uint4 *>(static_cast<const __nv_bfloat16 *>(p.x) + (size_t)t * p.d);
+    for (int r0 = 0; r0 < p.k; r0 += 8) {
+      int ids[8];
+#pragma unroll
+      for (int s = 0; s < 8; ++s) {
+        const int e = r0 + s < p.k ? p.ids[(size_t)t * p.k + r0 + s] : -1;
+        ids[s] = e >= 0 && e < p.E ? e : -1;
+      }
+      double acc[8];
+#pragma unroll
+      for (int s = 0; s < 8; ++s) acc[s] = 0.0;
+      for (int i = threadIdx.x; i < p.d / 8; i += RL_THREADS) {
+        const uint4 xv = __ldg(xr + i);
+        const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
+        double xd[8];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          xd[2 * u] = (double)__uint_as_float(xw[u] << 16);
+          xd[2 * u + 1] = (double)__uint_as_float(xw[u] & 0xFFFF0000u);
+        }
+#pragma unroll
+        for (int s = 0; s < 8; ++s)
+          if (ids[s] >= 0) {
+            const float4 *wr = reinterpret_cast<const float4 *>(p.w + (size_t)ids[s] * p.d) + 2 * i;
+            const float4 a = __ldg(wr), b = __ldg(wr + 1);
+            acc[s] = fma(xd[0], (double)a.x, acc[s]);
+            acc[s] = fma(xd[1], (double)a.y, acc[s]);
+            acc[s] = fma(xd[2], (double)a.z, acc[s]);
+            acc[s] = fma(xd[3], (double)a.w, acc[s]);
+            acc[s] = fma(xd[4], (double)b.x, acc[s]);
+            acc[s] = fma(xd[5], (double)b.y, acc[s]);
+            acc[s] = fma(xd[6], (double)b.z, acc[s]);
+            acc[s] = fma(xd[7], (double)b.w, acc[s]);
+          }
+      }
+#pragma unroll
+      for (int s = 0; s < 8; ++s) {
+        double v = acc[s];
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(full, v, o);
+        if (lane == 0) red[warp][s] = v;
+      }
+      __syncthreads();
+      if (threadIdx.x < 8 && r0 + (int)threadIdx.x < p.k) {
+        double v = 0.0;
+        for (int w = 0; w < RL_THREADS / 32; ++w) v += red[w][threadIdx.x];
+        lsh[r0 + threadIdx.x] = v;
+      }
+      __syncthreads();
+    }
+    if (warp == 0) {
+      int my_e = lane < p.k ? p.ids[(size_t)t * p.k + lane] : -1;
+      // a slot is live when its id is in range and not taken by an earlier slot
+      bool ok = lane < p.k && my_e >= 0 && my_e < p.E;
+      for (int s = 0; s < p.k; ++s) {
+        const int es = __shfl_sync(full, my_e, s);
+        if (s < lane && es == my_e) ok = false;
+      }
+      double wv = 0.0, key = -INFINITY;
+      if (ok) {
+        const double l = lsh[lane];
+        const double b = p.bias ? (double)p.bias[my_e] : 0.0;
+        if (softmax) {
+          wv = l + b;
+          key = wv;
+        } else {
+          wv = 1.0 / (1.0 + exp(-l));
+          key = wv + b;
+        }
+      }
+      if (softmax) {
+        double m = ok ? wv : -INFINITY;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) m = fmax(m, __shfl_xor_sync(full, m, o));
+        wv = ok ? exp(wv - m) : 0.0;
+      }
+      double tot = lane < p.k ? wv : 0.0;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) tot += __shfl_xor_sync(full, tot, o);
+      double wout;
+      if (softmax) wout = p.norm ? wv / fmax(tot, 1e-12) : wv;
+      else wout = (p.norm ? wv / (tot + 1e-20) : wv) * p.scaling;
+      int slot = lane;
+      if (!p.forced) {
+        slot = 0;
+        for (int s = 0; s < p.k; ++s) {
+          const double ks = __shfl_sync(full, key, s);
+          const int es = __shfl_sync(full, my_e, s);
+          if (ks > key || (ks == key && es < my_e)) ++slot;
+        }
+      }
+      __syncwarp();
+      if (lane < p.k) {
+        p.ids[(size_t)t * p.k + slot] = my_e;
+        p.wts[(size_t)t * p.k + slot] = (float)wout;
+      }
+    }
+    __syncthreads();
+  }
+}
+
 // prob_sum[e] = sum over 32-token groups in a fixed order: a block per 32
 // experts; warp w adds groups w, w + 32, w + 64, ... with eight loads in
 // flight, then the 32 warp sums are added in warp order.  Deterministic for a
@@ -1021,19 +1159,22 @@ cudaError_t launch_tiled(const RouteParams &p, dim3 grid, cudaStream_t s) {
 }
 
 // The selection pass over float64 logits partials [ks][T][E].
-template <int EPL, int TPB>
+template <int EPL, int TPB, int WPB>
 cudaError_t launch_select_tpb(const RouteParams &p, cudaStream_t s) {
   const size_t smem = sizeof(double) * ((size_t)TPB * p.E + (size_t)TPB * kMaxExperts);
-  auto sel = route_select<EPL, TPB>;
+  auto sel = route_select<EPL, TPB, WPB>;
   cudaError_t err = cudaFuncSetAttribute(sel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (err != cudaSuccess) return err;
-  launch_pdl(sel, (p.T + TPB - 1) / TPB, 32 * TPB, smem, s, p);
+  launch_pdl(sel, (p.T + TPB - 1) / TPB, 32 * WPB, smem, s, p);
   return cudaGetLastError();
 }
 
+// 32-token blocks run 16 warps (two tokens each) so that a selecting thread
+// keeps up to 128 registers
 template <int EPL>
 cudaError_t launch_select_epl(const RouteParams &p, cudaStream_t s) {
-  return select_tokens_per_block(p.T) == 8 ? launch_select_tpb<EPL, 8>(p, s) : launch_select_tpb<EPL, 32>(p, s);
+  return select_tokens_per_block(p.T) == 8 ? launch_select_tpb<EPL, 8, 8>(p, s)
+                                           : launch_select_tpb<EPL, 32, 16>(p, s);
 }
 
 template <int EPL, bool BF16>
@@ -1063,11 +1204,11 @@ cudaError_t launch_refine_tpb(const RouteParams &p, cudaStream_t s) {
 // tokens per block as the probability-sum rows were sized (select_tokens_per_block)
 template <int EPL>
 cudaError_t launch_refine_epl(const RouteParams &p, cudaStream_t s) {
-  return select_tokens_per_block(p.T) == 8 ? launch_refine_tpb<EPL, 8, 8>(p, s) : launch_refine_tpb<EPL, 32, 16>(p, s);
+  return select_tokens_per_block(p.T) == 8 ? launch_refine_tpb<EPL, 8, 8>(p, s) : launch_refine_tpb<EPL, 32, 8>(p, s);
 }
 
 cudaError_t launch_select(const RouteParams &p, cudaStream_t s) {
-  if (p.refine) {
+  if (p.refine || p.approx) {
     if (p.E <= 32) return launch_refine_epl<1>(p, s);
     if (p.E <= 64) return launch_refine_epl<2>(p, s);
     if (p.E <= 128) return launch_refine_epl<4>(p, s);
@@ -1097,10 +1238,21 @@ cudaError_t launch_any(const RouteParams &p, const RoutePlan &plan, cudaStream_t
 
 }  // namespace
 
+// MOE_ROUTER_TC=bf16 keeps the bf16 tensor-core logits with the exact
+// re-weighting of every token (read once per process)
+static bool bf16_tc_router_requested() {
+  static const bool on = [] {
+    const char *v = getenv("MOE_ROUTER_TC");
+    return v != nullptr && strcmp(v, "bf16") == 0;
+  }();
+  return on;
+}
+
 RoutePlan route_plan(const moe_config &c, bool allow_split) {
   RoutePlan plan{};
   plan.split = false;
   plan.tc = false;
+  plan.i8 = false;
   plan.ks = 1;
   plan.kchunk = c.hidden;
   plan.tpw = 4;
@@ -1109,6 +1261,11 @@ RoutePlan route_plan(const moe_config &c, bool allow_split) {
   const bool chosen_only = c.router == MOE_ROUTER_SIGMOID_GROUP || c.norm_topk_prob;
   // (a decode-sized batch is served faster by the split CUDA-core pass)
   if (allow_split && c.act_dtype == MOE_BF16 && chosen_only && c.num_tokens >= 512) {
+    if (i8_route_supported(c) && !bf16_tc_router_requested()) {
+      plan.i8 = true;
+      plan.ks = i8_route_plan(c).ks;
+      return plan;
+    }
     const TcRoutePlan t = tc_route_plan(c);
     plan.tc = true;
     plan.ks = t.ks;
@@ -1146,8 +1303,14 @@ static size_t tc_logits_part(const moe_config &c, int ks) {
 
 size_t route_logits_bytes(const moe_config &c) {
   const RoutePlan plan = route_plan(c, true);
+  if (plan.i8) return i8_route_bytes(c, i8_route_plan(c));
   if (plan.tc) return tc_logits_part(c, plan.ks) + tc_route_plan(c).wsplit_bytes;
   return plan.split ? sizeof(double) * (size_t)plan.ks * c.num_tokens * c.num_experts : 0;
+}
+
+size_t route_logits_f64_bytes(const moe_config &c) {
+  const RoutePlan plan = route_plan(c, true);
+  return plan.tc || plan.i8 || plan.split ? sizeof(double) * (size_t)plan.ks * c.num_tokens * c.num_experts : 0;
 }
 
 cudaError_t launch_route(const moe_config &c, const void *x, const float *w_router,
@@ -1174,12 +1337,45 @@ cudaError_t launch_route(const moe_config &c, const void *x, const float *w_rout
   p.part = route_part;
   const RoutePlan plan = route_plan(c, logits != nullptr);
   p.refine = plan.tc ? 1 : 0;
+  p.approx = 0;
+  p.xst = nullptr;
+  p.wst = nullptr;
+  p.tau = 0.0;
+  p.xcnt = nullptr;
+  p.xidx = nullptr;
+  p.xdx = nullptr;
+  p.round_list = 0;
+  p.flag_count = nullptr;
+  p.flag_list = nullptr;
   p.logits = logits;
   p.ks = plan.ks;
   p.kchunk = plan.kchunk;
 
   cudaError_t err;
-  if (plan.tc) {
+  if (plan.i8) {
+    const I8RoutePlan t = i8_route_plan(c);
+    const I8RouteBuffers b = i8_route_buffers(c, t, logits);
+    p.logits = b.logits;
+    p.approx = 1;
+    p.xst = b.xst;
+    p.wst = b.wst;
+    p.xcnt = b.xcnt;
+    p.xidx = b.xidx;
+    p.xdx = b.xdx;
+    p.round_list = b.round_list;
+    // a chosen logit within 2.5e-7 moves a renormalised weight by at most
+    // about 5e-7 of itself (twice the logit error), inside the 1e-6 bound
+    p.tau = 2.5e-7;
+    p.flag_count = b.flag_count;
+    p.flag_list = b.flag_list;
+    err = launch_route_i8_logits(c, x, w_router, t, b, status, s);
+    if (err == cudaSuccess) err = launch_select(p, s);
+    if (err == cudaSuccess) {
+      const int grid = c.num_tokens < 296 ? c.num_tokens : 296;
+      launch_pdl(route_refine_listed, grid, RL_THREADS, 0, s, p);
+      err = cudaGetLastError();
+    }
+  } else if (plan.tc) {
     __nv_bfloat16 *wsplit =
         reinterpret_cast<__nv_bfloat16 *>(reinterpret_cast<char *>(logits) + tc_logits_part(c, plan.ks));
     err = launch_route_tc_logits(c, x, w_router, wsplit, logits, status, s);
@@ -1190,7 +1386,7 @@ cudaError_t launch_route(const moe_config &c, const void *x, const float *w_rout
   if (err != cudaSuccess) return err;
   // probability-sum rows: one per selection block when route_select ran,
   // else one per 32-token block of the fused router kernels
-  const int nb = plan.tc || plan.split ? (c.num_tokens + select_tokens_per_block(c.num_tokens) - 1) /
+  const int nb = plan.tc || plan.i8 || plan.split ? (c.num_tokens + select_tokens_per_block(c.num_tokens) - 1) /
                                              select_tokens_per_block(c.num_tokens)
                                        : route_blocks(c);
   launch_pdl(route_finalize, (c.num_experts + 31) / 32, 32 * FIN_WARPS, 0, s, route_part, nb, c.num_experts, prob_sum);

@@ -221,6 +221,12 @@ def test_workspace_regions(name):
         assert n == expect[region], (region, n, expect[region])
         end = off + n
         assert end <= total
+    # the router's float64 logits partials [ks][T][E] lie before the dispatch buffers
+    off, n = api.moe_workspace_region(cfg, "router_logits")
+    assert off % 256 == 0 and n % (8 * w.T * w.E) == 0
+    assert off + n <= api.moe_workspace_region(cfg, "offsets")[0]
+    if w.dtype == "bf16" and w.T >= 512 and (w.router == "sigmoid_group" or w.norm_topk_prob):
+        assert n > 0, name          # tensor-core logits live in the workspace
     with pytest.raises(L.MoEError):
         off, n = C.c_size_t(), C.c_size_t()
         L.check(L.lib().moe_workspace_region(C.byref(cfg), L.MOE_WS_REGION_COUNT, C.byref(off), C.byref(n)),

@@ -13,7 +13,7 @@ import torch
 from gpu_harness import (AUX_RTOL, Run, check_aux, check_canaries, check_dispatch, check_output, check_route,
                          forward_permutation, sample_tokens)
 from mixture_experts_layer_41_b200 import api
-from mixture_experts_layer_41_b200.inputs import workload
+from mixture_experts_layer_41_b200.inputs import to_host, workload
 from moe_cases import oracle_route
 
 pytestmark = pytest.mark.gpu
@@ -227,6 +227,51 @@ ROUTER_SHAPES = {
 # (up to about a quarter at E = 96..128 with d = 192..256); every token inside
 # the margin is still checked for a valid choice and exact weights.
 ROUTER_SHAPE_MAX_UNSAFE = 0.35
+
+
+# Integer tensor-core logits (bf16, T >= 512, renormalised softmax or sigmoid):
+# the workspace logits against the digit model of the stated arithmetic (the
+# integer sums are exact, so only the float64 slice sums may differ), then the
+# routing against the oracle.  "hard_rows" plants an outlier element, a zero
+# row and a subnormal row: their bounds force the exact recomputation.
+I8_CASES = {
+    "deepseek_d7168": workload("deepseek_v3", T=1024, F=64, shared_F=0),
+    "mixtral_d4096_e8": workload("mixtral_prefill", T=512, F=64),
+    "switch_d2048_e64": workload("switch_top1", T=1024, F=64),
+    "e40_ragged_d": ROUTER_SHAPES["tc_e40_ragged_d"],
+    "e200_sigmoid": ROUTER_SHAPES["tc_e200_sigmoid"],
+    "e16": ROUTER_SHAPES["tc_e16"],
+    "hard_rows": workload("deepseek_v3", T=640, d=1024, F=64, shared_F=0),
+}
+
+
+@pytest.mark.parametrize("name", sorted(I8_CASES))
+def test_integer_router_logits(name):
+    from router_digits import logits_and_bound
+
+    w = I8_CASES[name]
+    run = Run(w, seed=9)
+    if name == "hard_rows":
+        x = run.inp["x"]
+        x[5, 3] = 3000.0
+        x[6] = 0.0
+        x[7] = x[7] * 1e-39
+        x[8, ::2] = 0.0
+    api.moe_route(run.cfg, run.inp["x"], run.inp["w_router"], run.bias, run.ids, run.wts, run.prob_sum, run.ws)
+    torch.cuda.synchronize()
+    assert run.status() == 0
+    off, n = api.moe_workspace_region(run.cfg, "router_logits")
+    assert n > 0 and n % (8 * w.T * w.E) == 0
+    ks = n // (8 * w.T * w.E)
+    part = run.ws[off:off + n].view(torch.float64).view(ks, w.T, w.E).cpu().numpy()
+    got = np.zeros((w.T, w.E))
+    for q in range(ks):
+        got += part[q]
+    model, bound = logits_and_bound(to_host(run.inp["x"]), to_host(run.inp["w_router"]))
+    dev = np.abs(got - model).max()
+    print(f"[i8 logits] {name}: {ks} slices, |gpu - model| {dev:.2e}, max bound {bound.max():.2e}")
+    assert dev <= 1e-12 * max(1.0, np.abs(model).max())
+    check_route(run, oracle_route(w, run.inp), max_unsafe_fraction=ROUTER_SHAPE_MAX_UNSAFE)
 
 
 @pytest.mark.parametrize("name", sorted(ROUTER_SHAPES))

@@ -1,0 +1,82 @@
+"""The integer tensor-core router's arithmetic contract, on the CPU: the digit
+model of its logits (tests/router_digits.py) stays within the stated bound of
+the oracle's float64 logits, on the workloads' recipes and on rows built to
+stress the split (an outlier element, a zero row, subnormal values)."""
+import numpy as np
+import pytest
+import torch
+
+from mixture_experts_layer_41_b200.inputs import make_inputs, to_host, workload
+from oracle import moe_oracle as O
+from router_digits import logits_and_bound, rounding_correction, token_digits, weight_digits
+
+# a chosen logit within this of exact moves a renormalised weight by at most
+# twice as much relative to itself: inside the 1e-6 routing-weight bound
+TAU = 2.5e-7
+
+
+def _bf16(a: np.ndarray) -> np.ndarray:
+    return torch.from_numpy(a.astype(np.float32)).to(torch.bfloat16).float().numpy()
+
+
+@pytest.mark.parametrize("name,T", [("deepseek_v3", 384), ("mixtral_prefill", 256), ("switch_top1", 256)])
+def test_model_within_bound_on_recipes(name, T):
+    # x and the router weight are the first draws: a small F leaves them unchanged
+    w = workload(name, T=T, F=8, shared_F=0)
+    inp = make_inputs(w, seed=3)
+    x, wr = to_host(inp["x"]), to_host(inp["w_router"])
+    ref = O.router_logits(x, wr)
+    lg, bound = logits_and_bound(x, wr)
+    err = np.abs(lg - ref)
+    assert np.all(err <= bound * (1 + 1e-9) + 1e-300), f"bound violated by {np.max(err - bound):.3e}"
+    print(f"[digits] {name}: max err {err.max():.2e}, median bound {np.median(bound):.2e}, "
+          f"(t, e) with bound > tau {np.mean(bound > TAU):.4f}")
+    # the recipes' logits come out far inside the routing tolerance
+    assert err.max() < 3e-7
+    assert np.mean(bound > TAU) < 0.05
+    # with the x-rounding term added exactly, the rest of the bound holds and
+    # leaves (nearly) nothing for the exact recomputation
+    corr, rest, n_rounded = rounding_correction(x, wr)
+    err2 = np.abs(lg + corr - ref)
+    assert np.all(err2 <= rest * (1 + 1e-9) + 1e-300)
+    print(f"[digits] {name}: corrected max err {err2.max():.2e}, rest bound > tau {np.mean(rest > TAU):.5f}, "
+          f"rows with > 8 rounded elements {np.mean(n_rounded > 8):.4f}")
+    assert np.mean(rest > TAU) < 1e-3
+
+
+def test_bound_holds_on_hard_rows():
+    rng = np.random.default_rng(11)
+    d, E = 1024, 16
+    x = rng.standard_normal((6, d))
+    x[1, 7] = 3000.0                         # an outlier: the row's small values lose digits
+    x[2] = 0.0                               # a zero row
+    x[3] = rng.standard_normal(d) * 1e-39    # subnormal bf16 values
+    x[4, ::2] = 0.0
+    x[5] = rng.standard_normal(d) * 2.0 ** 40
+    x = _bf16(x)
+    w = (rng.standard_normal((E, d)) * 0.02).astype(np.float32)
+    w[3] = 0.0
+    w[4, 5] = 7.0                            # an outlier weight
+    ref = O.router_logits(x, w)
+    lg, bound = logits_and_bound(x, w)
+    err = np.abs(lg - ref)
+    assert np.all(err <= bound * (1 + 1e-9) + 1e-300)
+    assert np.all(lg[2] == 0.0) and np.all(lg[:, 3] == 0.0)
+    # the outlier row's bound is large: its chosen logits are recomputed exactly
+    assert bound[1].max() > 100 * bound[0].max()
+
+
+def test_digits_reassemble_and_fit_int8():
+    rng = np.random.default_rng(5)
+    x = _bf16(rng.standard_normal((8, 256)) * np.logspace(-3, 3, 8)[:, None])
+    w = (rng.standard_normal((4, 256)) * 0.02).astype(np.float32)
+    A, sx, vx = token_digits(x)
+    B, sw, vw = weight_digits(w)
+    for dgt in A + B:
+        assert dgt.min() >= -128 and dgt.max() <= 127
+    assert np.array_equal(A[0] * 65536 + A[1] * 256 + A[2], vx)
+    assert np.array_equal(((B[0] * 256 + B[1]) * 256 + B[2]) * 256 + B[3], vw)
+    assert np.abs(vx).max() <= 2 ** 22 and np.abs(vw).max() <= 2 ** 30
+    # bf16 values at most 2^14 below the row maximum are represented exactly
+    keep = np.abs(x) >= np.abs(x).max(1, keepdims=True) * 2.0 ** -14
+    assert np.array_equal((vx * np.ldexp(1.0, -sx)[:, None])[keep], x.astype(np.float64)[keep])
