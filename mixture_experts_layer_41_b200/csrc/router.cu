@@ -8,10 +8,14 @@
 //
 // Two ways to the logits.  bf16 batches of 512 tokens or more whose weights
 // depend on the chosen experts alone (renormalised softmax, sigmoid) take
-// the tensor-core GEMMs of router_tc.cu (float64 partials per hidden slice);
-// route_select then chooses from those logits and recomputes the k chosen
-// logits exactly (exact_logit) for the weights and the slot order.  All other
-// cases stay on the CUDA cores: fp32 products summed over runs of 8 elements,
+// the integer tensor-core GEMM of router_i8.cu (float64 partials per hidden
+// slice, each logit within a computed bound of exact; or, with
+// MOE_ROUTER_TC=bf16, the selection-grade bf16 GEMMs of router_tc.cu);
+// route_select_refine then selects from those logits in fp32 and weights the
+// k chosen experts from their float64 logits: with bounded logits after
+// adding the x-rounding term exactly, listing for route_refine_listed the
+// tokens whose bound could matter; with selection-grade ones after an exact
+// recomputation.  All other cases stay on the CUDA cores: fp32 products summed over runs of 8 elements,
 // the runs added in float64 (a straight fp32 sum over d = 7168 misses the
 // 1e-6 weight bound); scores, selection and weights are float64 and rounded
 // to float32 on the store.  CUDA-core shapes:
@@ -25,10 +29,9 @@
 //                 of the hidden dimension and writes float64 partial logits.
 //   route_select  after a SPLIT pass (8-token x 32-expert x hidden-slice
 //                 blocks, used when T is too small to fill the GPU with
-//                 whole-row blocks, e.g. decode) or the tensor-core pass: sums
-//                 the partial logits of its tokens (32, or 8 for small T) in
-//                 slice order into shared memory, then selects with one warp
-//                 per token.
+//                 whole-row blocks, e.g. decode): sums the partial logits of
+//                 its tokens (32, or 8 for small T) in slice order into shared
+//                 memory, then selects with one warp per token.
 // Every selecting block writes one float64 probability sum per (block,
 // expert); route_finalize adds the rows in order, so prob_sum is
 // deterministic.

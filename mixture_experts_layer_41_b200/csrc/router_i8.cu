@@ -27,23 +27,32 @@
 // xhat and what carried by the digits a2 and b3), bounded by
 //   |dx|_1 |w|_inf + |xhat|_2 |dw|_2 + |x2|_2 |w3|_2,
 // whose factors route_i8_prep writes per token and per expert (float64,
-// rounded up).  The selection pass recomputes a token's chosen logits
-// exactly wherever that bound could move a weight past the routing tolerance
-// or swap two chosen experts.
+// rounded up; |xhat|_2 and |x2|_2 by upper bounds).  The preparation pass also
+// lists the (few) elements of each token row that the digits round, so the
+// selection pass adds dx . w exactly for the chosen experts; the rest of the
+// bound is then about 1e-7 on the workloads' recipes.  Tokens whose bound
+// could still move a weight past the routing tolerance, or swap two chosen
+// experts, are recomputed exactly (route_refine_listed in router.cu).
 //
 // route_i8_prep   a block per expert row (scale, four digit planes
-//                 [4][e_pad][d_pad], norms), then a warp per token row (scale,
-//                 the list of elements its digits round, norms).
+//                 [4][e_pad][d_pad], norms), then a warp per token row held in
+//                 registers (scale, |x|_2, the list of rounded elements).
 // route_i8_gemm   grid (N-expert tile, 128-token tile, hidden slice), one CTA
 //                 per SM:
 //   warp 0        TMA producer: the bf16 token tile (128 x 64, 128-byte
 //                 swizzle) and the four weight digit tiles (N x 64 bytes,
-//                 64-byte swizzle);
-//   warp 1        TMEM owner and single-thread MMA issuer (kind::i8, M = 128,
-//                 N, K = 32; 11 pair products per K-block, 2 K-steps each);
-//   warps 2-9     digit converters: each K-block's token tile into three
-//                 digit planes in the 64-byte-swizzled K-major layout the MMA
-//                 reads; after the last K-block, the epilogue.
+//                 64-byte swizzle), stored one after another so that they
+//                 read as one 4N-row operand;
+//   warp 1        TMEM owner and single-thread MMA issuer: per 32-element K
+//                 step three kind::i8 MMAs (M = 128), token digit i (from
+//                 TMEM) against the weight digits side by side (N' = 4N, 4N,
+//                 3N) into the class columns i N ..., which adds every kept
+//                 pair (i, j) to class i + j;
+//   warps 2-9     digit converters: each K-block's token tile into the three
+//                 digit planes, stored into TMEM (lane = token row, four int8
+//                 of K per column; three stages); after the last K-block, the
+//                 epilogue (int64 combination, float64 scale, rows staged in
+//                 shared memory for coalesced stores).
 // Every mbarrier wait is bounded by %globaltimer (moe_set_wait_timeout_ns); on
 // expiry the CTA records a status, drains its own copies and MMAs, frees TMEM
 // and exits.
