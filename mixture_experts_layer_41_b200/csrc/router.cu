@@ -801,36 +801,51 @@ route_select_refine(RouteParams p) {
       float sum = 0.f;
 #pragma unroll
       for (int j = 0; j < EPL; ++j) {
-        prob[j] = (lane + 32 * j) < E ? expf(score[j] - m) : 0.f;
+        prob[j] = (lane + 32 * j) < E ? __expf(score[j] - m) : 0.f;
         sum += prob[j];
       }
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(full, sum, o);
 #pragma unroll
-      for (int j = 0; j < EPL; ++j) prob[j] /= sum;
+      for (int j = 0; j < EPL; ++j) prob[j] = __fdividef(prob[j], sum);
     } else {
 #pragma unroll
       for (int j = 0; j < EPL; ++j) {
         const int e = lane + 32 * j;
         if (e < E) {
-          prob[j] = 1.f / (1.f + expf(-lg[j]));
+          prob[j] = __fdividef(1.f, 1.f + __expf(-lg[j]));
           score[j] = prob[j] + (p.bias ? p.bias[e] : 0.f);
-          scr[e] = score[j];
+          if (G != 32) scr[e] = score[j];
         } else {
           prob[j] = 0.f;
           score[j] = -INFINITY;
         }
       }
-      __syncwarp();
       // group score: the sum of the group's two largest selection scores
       float gs = -INFINITY;
-      if (lane < p.n_group) {
-        float b1 = -INFINITY, b2 = -INFINITY;
-        for (int q = 0; q < G; ++q) {
-          const float v = scr[lane * G + q];
-          if (v > b1) { b2 = b1; b1 = v; } else if (v > b2) { b2 = v; }
+      if (G == 32) {
+        // group g is column g of the lanes' scores: two warp arg-max reductions
+#pragma unroll
+        for (int g = 0; g < EPL; ++g)
+          if (g < p.n_group) {
+            float v1 = score[g];
+            int i1 = lane;
+            warp_argmax_f(v1, i1);
+            float v2 = lane == i1 ? -INFINITY : score[g];
+            int i2 = lane;
+            warp_argmax_f(v2, i2);
+            if (lane == g) gs = v1 + v2;
+          }
+      } else {
+        __syncwarp();
+        if (lane < p.n_group) {
+          float b1 = -INFINITY, b2 = -INFINITY;
+          for (int q = 0; q < G; ++q) {
+            const float v = scr[lane * G + q];
+            if (v > b1) { b2 = b1; b1 = v; } else if (v > b2) { b2 = v; }
+          }
+          gs = b1 + b2;
         }
-        gs = b1 + b2;
       }
       __syncwarp();
       uint32_t keep = 0;
@@ -1003,7 +1018,7 @@ route_select_refine(RouteParams p) {
 // dimension for eight chosen experts at a time (bf16 x fp32 products exact in
 // float64, float64 sums reduced in a fixed order), then warp 0 weights and
 // orders the slots from the exact logits as the selection pass would.
-constexpr int RL_THREADS = 256;
+constexpr int RL_THREADS = 1024;
 __global__ void __launch_bounds__(RL_THREADS) route_refine_listed(RouteParams p) {
   pdl_enter();
   __shared__ double red[RL_THREADS / 32][8];
@@ -1374,7 +1389,7 @@ cudaError_t launch_route(const moe_config &c, const void *x, const float *w_rout
     err = launch_route_i8_logits(c, x, w_router, t, b, status, s);
     if (err == cudaSuccess) err = launch_select(p, s);
     if (err == cudaSuccess) {
-      const int grid = c.num_tokens < 296 ? c.num_tokens : 296;
+      const int grid = c.num_tokens < 148 ? c.num_tokens : 148;
       launch_pdl(route_refine_listed, grid, RL_THREADS, 0, s, p);
       err = cudaGetLastError();
     }

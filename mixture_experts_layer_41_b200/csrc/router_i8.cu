@@ -35,8 +35,8 @@
 // experts, are recomputed exactly (route_refine_listed in router.cu).
 //
 // route_i8_prep   a block per expert row (scale, four digit planes
-//                 [4][e_pad][d_pad], norms), then a warp per token row held in
-//                 registers (scale, |x|_2, the list of rounded elements).
+//                 [4][e_pad][d_pad], norms), then two warps per token row held
+//                 in registers (scale, |x|_2, the list of rounded elements).
 // route_i8_gemm   grid (N-expert tile, 128-token tile, hidden slice), one CTA
 //                 per SM:
 //   warp 0        TMA producer: the bf16 token tile (128 x 64, 128-byte
@@ -339,59 +339,137 @@ __device__ __forceinline__ void token_chunk_scan(uint4 v, __nv_bfloat162 &mx, __
 }
 __device__ __forceinline__ uint32_t bf16x2_bits(__nv_bfloat162 v) { return *reinterpret_cast<uint32_t *>(&v); }
 
-// One token row per warp.  NC > 0: the row (d <= 256 NC) is loaded into
-// registers at once, all loads in flight together; NC = 0: streamed twice.
+// Shared by the two warps of a token row (half-row mode).
+struct HalfRowShared {
+  uint32_t mb[2], ml[2];
+  float l2[2];
+  double l1[2];
+  int cnt0;
+};
+
+// Pass 2 over one warp's chunks (indices base + lane + 32 c): the rounded
+// elements listed from slot cnt on, |dx| added to l1.
 template <int NC>
-__device__ __forceinline__ void token_row(const PrepParams &p, int t, int lane) {
-  const unsigned full = 0xffffffffu;
-  const uint4 *xr = reinterpret_cast<const uint4 *>(p.x + (size_t)t * p.d);
-  const int nv = p.d / 8;
-  const uint4 zero = make_uint4(0u, 0u, 0u, 0u);
-  uint4 reg[NC > 0 ? NC : 1];
-  // pass 1: the row's largest and smallest magnitude and |x|_2^2 (fp32)
-  const uint32_t lo0 = 0u, hi0 = 0x7F7F7F7Fu;
-  __nv_bfloat162 mx = *reinterpret_cast<const __nv_bfloat162 *>(&lo0);
-  __nv_bfloat162 mn = *reinterpret_cast<const __nv_bfloat162 *>(&hi0);
-  float l2 = 0.f;
-  if constexpr (NC > 0) {
+__device__ __forceinline__ void list_rounded(const PrepParams &p, int t, const uint4 (&reg)[NC], int base, int nv,
+                                             bool all, int ethr, double scale_d, double inv, int lane, double &l1,
+                                             int &cnt) {
 #pragma unroll
-    for (int c = 0; c < NC; ++c) reg[c] = lane + 32 * c < nv ? __ldg(xr + lane + 32 * c) : zero;
-#pragma unroll
-    for (int c = 0; c < NC; ++c)
-      if (lane + 32 * c < nv) token_chunk_scan(reg[c], mx, mn, l2);
-  } else {
-#pragma unroll 4
-    for (int i = lane; i < nv; i += 32) token_chunk_scan(__ldg(xr + i), mx, mn, l2);
-  }
-  uint32_t mb = bf16x2_bits(mx), ml = bf16x2_bits(mn);
-  // lanes past the row end kept the initial values, which the reductions ignore
-  mb = warp_max_u(max(mb & 0xFFFFu, mb >> 16));
-  ml = min(ml & 0xFFFFu, ml >> 16);
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) ml = min(ml, __shfl_xor_sync(full, ml, o));
+  for (int c = 0; c < NC; ++c)
+    if (base + 32 * c < nv && __any_sync(0xffffffffu, chunk_may_round(reg[c], all, ethr)))
+      token_chunk_rounding(p, t, base + lane + 32 * c, reg[c], scale_d, inv, lane, l1, cnt);
+}
+
+// The row statistics from its largest / smallest magnitude bits and sums.
+__device__ __forceinline__ void row_scale(uint32_t mb, int &sx, int &emax, bool &all, int &ethr) {
   // |x| < 2^e over the row (e = 0 for an all-zero row)
   int e = 0;
   if (mb >= 0x80u) e = (int)(mb >> 7) - 126;
   else if (mb != 0) e = (31 - __clz((int)mb)) - 132;
-  const int sx = min(22 - e, 127);
-  // pass 2: the elements the digits round.  x 2^sx = M 2^(E - Emax + 14)
-  // for a bf16 significand M, so only exponent fields below Emax - 14 can
-  // round -- unless the scale was clamped (Emax < 21), when any can
-  const int emax = max((int)(mb >> 7), 1);
-  const bool all = emax < 21;
-  const int ethr = emax - 14;
+  sx = min(22 - e, 127);
+  // x 2^sx = M 2^(E - Emax + 14) for a bf16 significand M, so only exponent
+  // fields below Emax - 14 can round -- unless the scale was clamped
+  // (Emax < 21), when any can
+  emax = max((int)(mb >> 7), 1);
+  all = emax < 21;
+  ethr = emax - 14;
+}
+
+__device__ __forceinline__ void write_row_stats(const PrepParams &p, int t, int sx, int cnt, double l1, double l2) {
+  const double inv = pow2d(-sx);
+  p.sx[t] = sx;
+  p.xcnt[t] = cnt;
+  double *o = p.xst + (size_t)t * 4;
+  o[0] = l1 * kRoundUp;
+  o[1] = sqrt(l2) * kRoundUp32 + l1 * kRoundUp;        // |xhat|_2 <= |x|_2 + |dx|_1
+  o[2] = 128.0 * sqrt((double)p.d) * inv * kRoundUp;   // |x2|_2 <= 128 sqrt(d) 2^-sx
+  o[3] = 0.0;
+}
+
+// A token row held in the registers of two warps (half h of d <= 512 NC:
+// chunks NC h .. NC h + NC - 1 of 32 lanes), all loads in flight at once.
+// Both halves meet in shared memory for the scale; half 0 lists its rounded
+// elements first, then half 1 continues the list.
+template <int NC>
+__device__ __forceinline__ void token_half_row(const PrepParams &p, int t, int h, int lane, HalfRowShared &sh) {
+  const unsigned full = 0xffffffffu;
+  const bool live = t < p.T;
+  const uint4 *xr = reinterpret_cast<const uint4 *>(p.x + (size_t)(live ? t : 0) * p.d);
+  const int nv = live ? p.d / 8 : 0;
+  const int base = 32 * NC * h;
+  const uint4 zero = make_uint4(0u, 0u, 0u, 0u);
+  uint4 reg[NC];
+  const uint32_t lo0 = 0u, hi0 = 0x7F7F7F7Fu;
+  __nv_bfloat162 mx = *reinterpret_cast<const __nv_bfloat162 *>(&lo0);
+  __nv_bfloat162 mn = *reinterpret_cast<const __nv_bfloat162 *>(&hi0);
+  float l2 = 0.f;
+#pragma unroll
+  for (int c = 0; c < NC; ++c) reg[c] = base + lane + 32 * c < nv ? __ldg(xr + base + lane + 32 * c) : zero;
+#pragma unroll
+  for (int c = 0; c < NC; ++c)
+    if (base + lane + 32 * c < nv) token_chunk_scan(reg[c], mx, mn, l2);
+  uint32_t mb = bf16x2_bits(mx), ml = bf16x2_bits(mn);
+  mb = warp_max_u(max(mb & 0xFFFFu, mb >> 16));
+  ml = min(ml & 0xFFFFu, ml >> 16);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    ml = min(ml, __shfl_xor_sync(full, ml, o));
+    l2 += __shfl_xor_sync(full, l2, o);
+  }
+  if (lane == 0) {
+    sh.mb[h] = mb;
+    sh.ml[h] = ml;
+    sh.l2[h] = l2;
+  }
+  __syncthreads();
+  mb = max(sh.mb[0], sh.mb[1]);
+  ml = min(sh.ml[0], sh.ml[1]);
+  int sx, emax, ethr;
+  bool all;
+  row_scale(mb, sx, emax, all, ethr);
+  const double scale_d = pow2d(sx), inv = pow2d(-sx);
+  // (the smallest magnitude tells whether any element can round at all)
+  const bool any_round = live && (all || max((int)(ml >> 7), 1) < ethr);
+  double l1 = 0.0;
+  int cnt = 0;
+  if (any_round && h == 0) list_rounded<NC>(p, t, reg, base, nv, all, ethr, scale_d, inv, lane, l1, cnt);
+  if (lane == 0 && h == 0) sh.cnt0 = cnt;
+  __syncthreads();
+  if (any_round && h == 1) {
+    cnt = sh.cnt0;
+    list_rounded<NC>(p, t, reg, base, nv, all, ethr, scale_d, inv, lane, l1, cnt);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) l1 += __shfl_xor_sync(full, l1, o);
+  if (lane == 0) sh.l1[h] = l1;
+  __syncthreads();
+  if (live && h == 1 && lane == 0)
+    write_row_stats(p, t, sx, cnt, sh.l1[0] + sh.l1[1], (double)sh.l2[0] + (double)sh.l2[1]);
+}
+
+// A token row per warp, streamed twice (rows longer than the register halves hold).
+__device__ __forceinline__ void token_row_stream(const PrepParams &p, int t, int lane) {
+  const unsigned full = 0xffffffffu;
+  const uint4 *xr = reinterpret_cast<const uint4 *>(p.x + (size_t)t * p.d);
+  const int nv = p.d / 8;
+  const uint4 zero = make_uint4(0u, 0u, 0u, 0u);
+  const uint32_t lo0 = 0u, hi0 = 0x7F7F7F7Fu;
+  __nv_bfloat162 mx = *reinterpret_cast<const __nv_bfloat162 *>(&lo0);
+  __nv_bfloat162 mn = *reinterpret_cast<const __nv_bfloat162 *>(&hi0);
+  float l2 = 0.f;
+#pragma unroll 4
+  for (int i = lane; i < nv; i += 32) token_chunk_scan(__ldg(xr + i), mx, mn, l2);
+  uint32_t mb = bf16x2_bits(mx), ml = bf16x2_bits(mn);
+  mb = warp_max_u(max(mb & 0xFFFFu, mb >> 16));
+  ml = min(ml & 0xFFFFu, ml >> 16);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) ml = min(ml, __shfl_xor_sync(full, ml, o));
+  int sx, emax, ethr;
+  bool all;
+  row_scale(mb, sx, emax, all, ethr);
   const double scale_d = pow2d(sx), inv = pow2d(-sx);
   double l1 = 0.0;
   int cnt = 0;
-  // (the smallest magnitude tells whether any element can round at all)
-  if (!all && max((int)(ml >> 7), 1) >= ethr) {
-    // nothing to list
-  } else if constexpr (NC > 0) {
-#pragma unroll
-    for (int c = 0; c < NC; ++c)
-      if (32 * c < nv && __any_sync(full, chunk_may_round(reg[c], all, ethr)))
-        token_chunk_rounding(p, t, lane + 32 * c, reg[c], scale_d, inv, lane, l1, cnt);
-  } else {
+  if (all || max((int)(ml >> 7), 1) < ethr) {
     for (int base = 0; base < nv; base += 32) {
       const int i = base + lane;
       const uint4 v = i < nv ? __ldg(xr + i) : zero;
@@ -405,15 +483,7 @@ __device__ __forceinline__ void token_row(const PrepParams &p, int t, int lane) 
     l1 += __shfl_xor_sync(full, l1, o);
     dl2 += __shfl_xor_sync(full, dl2, o);
   }
-  if (lane == 0) {
-    p.sx[t] = sx;
-    p.xcnt[t] = cnt;
-    double *o = p.xst + (size_t)t * 4;
-    o[0] = l1 * kRoundUp;
-    o[1] = sqrt(dl2) * kRoundUp32 + l1 * kRoundUp;        // |xhat|_2 <= |x|_2 + |dx|_1
-    o[2] = 128.0 * sqrt((double)p.d) * inv * kRoundUp;   // |x2|_2 <= 128 sqrt(d) 2^-sx
-    o[3] = 0.0;
-  }
+  if (lane == 0) write_row_stats(p, t, sx, cnt, l1, dl2);
 }
 
 __global__ void __launch_bounds__(32 * PREP_WARPS) route_i8_prep(PrepParams p) {
@@ -421,14 +491,20 @@ __global__ void __launch_bounds__(32 * PREP_WARPS) route_i8_prep(PrepParams p) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   if (blockIdx.x == 0 && threadIdx.x == 0) *p.flag_count = 0;
   if ((int)blockIdx.x >= p.e_pad) {
-    // ---------------------------------------------------------- token row
-    const int t = (blockIdx.x - p.e_pad) * PREP_WARPS + warp;
-    if (t >= p.T) return;
-    const int nc = (p.d / 8 + 31) / 32;
-    if (nc <= 8) token_row<8>(p, t, lane);
-    else if (nc <= 16) token_row<16>(p, t, lane);
-    else if (nc <= 32) token_row<32>(p, t, lane);
-    else token_row<0>(p, t, lane);
+    // ---------------------------------------------------------- token rows
+    const int nc = (p.d / 8 + 31) / 32;      // 32-lane chunks of a row
+    if (nc <= 32) {
+      // two warps per row, PREP_WARPS / 2 rows per block
+      __shared__ HalfRowShared sh[PREP_WARPS / 2];
+      const int t = (blockIdx.x - p.e_pad) * (PREP_WARPS / 2) + (warp >> 1);
+      const int h = warp & 1;
+      if (nc <= 8) token_half_row<4>(p, t, h, lane, sh[warp >> 1]);
+      else if (nc <= 16) token_half_row<8>(p, t, h, lane, sh[warp >> 1]);
+      else token_half_row<16>(p, t, h, lane, sh[warp >> 1]);
+    } else {
+      const int t = (blockIdx.x - p.e_pad) * PREP_WARPS + warp;
+      if (t < p.T) token_row_stream(p, t, lane);
+    }
     return;
   }
   // ------------------------------------------------------------ expert row: a block per row
@@ -885,7 +961,9 @@ cudaError_t launch_route_i8_logits(const moe_config &c, const void *x, const flo
   pp.E = c.num_experts;
   pp.e_pad = t.e_pad;
   pp.d_pad = t.d_pad;
-  pp.x_blocks = (c.num_tokens + PREP_WARPS - 1) / PREP_WARPS;
+  // two warps per token row while a row fits their registers (d <= 8192), else one
+  const int rows_per_block = (c.hidden / 8 + 31) / 32 <= 32 ? PREP_WARPS / 2 : PREP_WARPS;
+  pp.x_blocks = (c.num_tokens + rows_per_block - 1) / rows_per_block;
   pp.wdig = b.wdig;
   pp.sx = b.sx;
   pp.sw = b.sw;
