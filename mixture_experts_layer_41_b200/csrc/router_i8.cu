@@ -67,7 +67,7 @@ namespace {
 
 constexpr int TM = 128;                 // tokens per tile (MMA M)
 constexpr int BK = 64;                  // hidden elements per K-block
-constexpr int XS = 6, AS = 3, WS = 6;   // ring depths: token tiles, token digit planes (TMEM), weight digit planes
+constexpr int XS = 3, AS = 3, WS = 3;   // ring depths: token tiles, token digit planes (TMEM), weight digit planes
 constexpr int XD = 3, WD = 4;           // digit planes of a token row and of a weight row
 constexpr int NCLS = 5;                 // accumulator classes i + j = 0..4
 constexpr int CONV_WARPS = 8;
@@ -101,7 +101,8 @@ struct I8Shape {
   }
   static constexpr uint32_t IDESC4 = idesc(WD * N), IDESC3 = idesc((WD - 1) * N);
   static_assert(WD * N <= 256, "an MMA spans at most 256 columns");
-  static_assert(CONV_WARPS * 32 * (CPW + 1) * 8 <= XS * X_BYTES, "epilogue staging exceeds the token ring");
+  static_assert(CONV_WARPS * 32 * (CPW + 1) * 8 <= XS * X_BYTES + WS * W_BYTES,
+                "epilogue staging exceeds the rings");
   static_assert(COLS_USED <= 512, "accumulators and token digits exceed TMEM");
 };
 
@@ -120,6 +121,8 @@ struct I8Shared {
   uint64_t a_full[AS], a_empty[AS];
   uint64_t w_full[WS], w_empty[WS];
   uint64_t acc_full, drain;
+  uint64_t tmem_full;   // the accumulators are allocated (warp 1)
+  uint64_t acc_read;    // every converter warp has read them (warp 1 frees TMEM)
   uint32_t tmem_base;
   int abort_flag;
 };
@@ -598,7 +601,7 @@ __global__ void __launch_bounds__(32 * PREP_WARPS) route_i8_prep(PrepParams p) {
 
 // ---------------------------------------------------------------- the GEMM
 template <int N>
-__global__ void __launch_bounds__(THREADS, 1)
+__global__ void __launch_bounds__(THREADS, 2)
 route_i8_gemm(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ CUtensorMap mapW,
               const I8Params p) {
   pdl_enter();
@@ -629,21 +632,17 @@ route_i8_gemm(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ 
     }
     mbar_init(&st->acc_full, 1);
     mbar_init(&st->drain, 1);
+    mbar_init(&st->tmem_full, 1);
+    mbar_init(&st->acc_read, CONV_WARPS);
     st->abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
   }
-  if (warp == 1) {
-    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&st->tmem_base)),
-                 "r"(S::TMEM_COLS)
-                 : "memory");
-    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
-  }
-  tc_fence_before();
   __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem_base = st->tmem_base;
   volatile int *abort_flag = &st->abort_flag;
+  // Two CTAs share an SM: the copies start at once, while the tensor memory
+  // may still belong to the other CTA (its allocation waits until that one
+  // has read its accumulators and freed it).
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
@@ -683,7 +682,15 @@ route_i8_gemm(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ 
     }
     __syncwarp();
   } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
+    // ------------------------------------------------------------ TMEM owner and MMA issuer
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&st->tmem_base)),
+                 "r"(S::TMEM_COLS)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&st->tmem_full);
+    const uint32_t tmem_base = st->tmem_base;
     if (lane == 0) {
       bool ok = true;
       for (int it = 0; it < kb_n && ok; ++it) {
@@ -709,8 +716,15 @@ route_i8_gemm(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ 
       if (ok) tc_commit(&st->acc_full);
       tc_commit(&st->drain);
       if (!wait_drain(&st->drain, 0u)) record_status(p.status, kDevTimeoutDrain);
+      // the converters read the accumulators (or gave up): then TMEM is free
+      // for the other CTA on this SM while this one stores the logits
+      if (!wait_bounded(&st->acc_read, 0u, abort_flag, p.status, kDevTimeoutMma, p.timeout_ns))
+        wait_drain(&st->acc_read, 0u);
     }
     __syncwarp();
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(S::TMEM_COLS)
+                 : "memory");
   } else {
     // ------------------------------------------------------------ digit converters, then the epilogue
     // warp (quarter q, half h): lane = token row 32 q + lane of the tile, the
@@ -719,10 +733,14 @@ route_i8_gemm(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ 
     const int cw = warp - 2;
     const int q = warp & 3, h = cw >> 2;
     const int r = q * 32 + lane;
+    const bool have_tmem =
+        wait_bounded(&st->tmem_full, 0u, abort_flag, p.status, kDevTimeoutEpilogue, p.timeout_ns);
+    tc_fence_after();
+    const uint32_t tmem_base = st->tmem_base;
     // (the row's scale is read here, so the copies start without waiting for it)
     const float sc = t0 + r < p.T ? pow2f(p.sx[t0 + r]) : 1.0f;
     const uint32_t lane_base = tmem_base + ((uint32_t)(q * 32) << 16);
-    {
+    if (have_tmem) {
       // zero this quarter's half of the class accumulators (made visible to
       // the MMAs by the first K-block's wait and fence below)
       const uint32_t z[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
@@ -730,8 +748,8 @@ route_i8_gemm(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ 
 #pragma unroll 1
       for (int c0 = 0; c0 < HALF; c0 += 8) tmem_st8(lane_base + (uint32_t)(h * HALF + c0), z);
     }
-    bool ok = true;
-    for (int it = 0; it < kb_n; ++it) {
+    bool ok = have_tmem;
+    for (int it = 0; ok && it < kb_n; ++it) {
       const int xs = it % XS, as = it % AS;
       if (!wait_bounded(&st->x_full[xs], (it / XS) & 1, abort_flag, p.status, kDevTimeoutEpilogue, p.timeout_ns) ||
           !wait_bounded(&st->a_empty[as], ((it / AS) & 1) ^ 1, abort_flag, p.status, kDevTimeoutEpilogue,
@@ -775,8 +793,16 @@ route_i8_gemm(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ 
       }
     }
     // ---------------------------------------------------------- epilogue
-    if (ok && kb_n > 0 &&
-        wait_bounded(&st->acc_full, 0u, abort_flag, p.status, kDevTimeoutEpilogue, p.timeout_ns)) {
+    const bool acc_ok = ok && kb_n > 0 &&
+                        wait_bounded(&st->acc_full, 0u, abort_flag, p.status, kDevTimeoutEpilogue, p.timeout_ns);
+    if (!acc_ok) {
+      if (have_tmem) {
+        tmem_wait_st();
+        tc_fence_before();
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&st->acc_read);   // nothing to read: TMEM may go
+    } else {
       tc_fence_after();
       // each warp's 32 rows x CPW logits go through its own slice of the
       // (now idle) token-tile ring, so the global stores run along rows
@@ -798,7 +824,10 @@ route_i8_gemm(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ 
           stage[lane * (S::CPW + 1) + cc + m] = (double)s * pow2d(8 - sxt - __ldg(p.sw + e0 + col0 + cc + m));
         }
       }
+      // the accumulators are read: TMEM goes to the other CTA on this SM
+      tc_fence_before();
       __syncwarp();
+      if (lane == 0) mbar_arrive(&st->acc_read);
       // row i of the warp: lanes take consecutive experts
       const int ne = min(S::CPW, p.E - (e0 + col0));
       for (int i = 0; i < 32; ++i) {
@@ -810,13 +839,6 @@ route_i8_gemm(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ 
     }
   }
 
-  tc_fence_before();
-  __syncthreads();
-  if (warp == 1) {
-    tc_fence_after();
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(S::TMEM_COLS)
-                 : "memory");
-  }
 }
 
 // ---------------------------------------------------------------- host side
