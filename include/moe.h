@@ -203,7 +203,8 @@ const char *moe_last_error(void);
 int64_t moe_kernel_launches(void);
 
 /* Bound on every on-chip barrier wait of the tensor-core kernels (grouped
- * GEMMs, the tensor-core router logits), in nanoseconds of the GPU's global
+ * GEMMs, the 4-bit tcgen05 FFN, the router's integer and bf16 tensor-core
+ * logits), in nanoseconds of the GPU's global
  * timer, for the launches that follow (process-wide, all threads).  When a
  * wait runs out, the kernel records where in the workspace status word
  * (moe_workspace_status: MOE_ERR_DEVICE, "... wait timed out"), lets the

@@ -26,10 +26,10 @@ enum DeviceStatus : int {
   kDevOk = 0,
   kDevBadExpertId = 1,       // dispatch: topk id outside [0, E)
   kDevDuplicateId = 2,       // dispatch: a token names the same expert twice
-  kDevTimeoutProducer = 10,  // grouped GEMM: TMA producer waited too long
-  kDevTimeoutMma = 11,       // grouped GEMM: MMA issuer waited too long
-  kDevTimeoutEpilogue = 12,  // grouped GEMM: epilogue waited too long
-  kDevTimeoutDrain = 13,     // grouped GEMM: in-flight work did not drain after an abort
+  kDevTimeoutProducer = 10,  // tensor-core kernel: TMA producer waited too long
+  kDevTimeoutMma = 11,       // tensor-core kernel: MMA issuer waited too long
+  kDevTimeoutEpilogue = 12,  // tensor-core kernel: epilogue / converter waited too long
+  kDevTimeoutDrain = 13,     // tensor-core kernel: in-flight work did not drain after an abort
   kDevBadOffsets = 20,       // grouped FFN: expert_offsets not 0-based / non-decreasing / in range
 };
 

@@ -377,10 +377,10 @@ moe_status moe_workspace_status(const void *ws, moe_stream_t stream) {
   switch (code) {
     case kDevBadExpertId: what = "dispatch: expert id outside [0, E)"; break;
     case kDevDuplicateId: what = "dispatch: a token names the same expert twice"; break;
-    case kDevTimeoutProducer: what = "grouped GEMM: TMA producer wait timed out"; break;
-    case kDevTimeoutMma: what = "grouped GEMM: MMA issuer wait timed out"; break;
-    case kDevTimeoutEpilogue: what = "grouped GEMM: epilogue wait timed out"; break;
-    case kDevTimeoutDrain: what = "grouped GEMM: in-flight work did not drain after an abort"; break;
+    case kDevTimeoutProducer: what = "tensor-core kernel: TMA producer wait timed out"; break;
+    case kDevTimeoutMma: what = "tensor-core kernel: MMA issuer wait timed out"; break;
+    case kDevTimeoutEpilogue: what = "tensor-core kernel: epilogue / converter wait timed out"; break;
+    case kDevTimeoutDrain: what = "tensor-core kernel: in-flight work did not drain after an abort"; break;
     case kDevBadOffsets: what = "grouped FFN: expert_offsets not 0-based, non-decreasing and within T*k"; break;
   }
   char num[32];

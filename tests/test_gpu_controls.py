@@ -394,3 +394,28 @@ def test_barrier_wait_timeout_reports_and_recovers(kernel, monkeypatch):
     run.staged()
     assert run.status() == 0
     check_output(run, routing="gpu")
+
+
+def test_router_wait_timeout_reports_and_recovers():
+    """The same failure path in the integer tensor-core router (two CTAs per
+    SM sharing the tensor memory): with a 1 ns bound the router GEMM gives up,
+    frees its tensor memory, and the call reports MOE_ERR_DEVICE; with the
+    default bound restored the same workspace routes as the oracle does."""
+    from gpu_harness import check_route
+    from moe_cases import oracle_route
+    w = workload("deepseek_v3", T=1024, d=2048, F=64, shared_F=0)
+    run = Run(w, seed=4)
+    c = run.cfg
+    try:
+        api.moe_set_wait_timeout_ns(1)
+        api.moe_route(c, run.inp["x"], run.inp["w_router"], run.bias, run.ids, run.wts, run.prob_sum, run.ws)
+        st = run.status()
+        text = L.lib().moe_last_error().decode()
+    finally:
+        api.moe_set_wait_timeout_ns(0)
+    assert st == L.MOE_ERR_DEVICE, st
+    assert "timed out" in text, text
+    api.moe_route(c, run.inp["x"], run.inp["w_router"], run.bias, run.ids, run.wts, run.prob_sum, run.ws)
+    torch.cuda.synchronize()
+    assert run.status() == 0
+    check_route(run, oracle_route(w, run.inp))
