@@ -926,7 +926,11 @@ route_select_refine(RouteParams p) {
           const size_t o = (size_t)t * p.round_list;
           const float *wr = p.w + (size_t)my_e * p.d;
           double corr = 0.0;
-          for (int q = 0; q < xcnt; ++q) corr = fma(p.xdx[o + q], (double)__ldg(wr + p.xidx[o + q]), corr);
+          for (int q = 0; q < xcnt; ++q) {
+            // (an index outside the row, left by a preparation pass that gave up, adds nothing)
+            const int ix = p.xidx[o + q];
+            if ((unsigned)ix < (unsigned)p.d) corr = fma(p.xdx[o + q], (double)__ldg(wr + ix), corr);
+          }
           my_l += corr;
         } else {
           bnd = xs0 * ws[0];

@@ -62,6 +62,8 @@
 #include <cudaTypedefs.h>
 #include <stdlib.h>
 
+#include <algorithm>
+
 namespace moe {
 namespace {
 
@@ -234,11 +236,6 @@ __device__ __forceinline__ double warp_sum_d(double v) {
   for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
   return v;
 }
-__device__ __forceinline__ double warp_max_d(double v) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) v = fmax(v, __shfl_xor_sync(0xffffffffu, v, o));
-  return v;
-}
 __device__ __forceinline__ uint32_t warp_max_u(uint32_t v) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v = max(v, __shfl_xor_sync(0xffffffffu, v, o));
@@ -254,7 +251,10 @@ struct PrepParams {
   const __nv_bfloat16 *x;
   const float *w;
   int T, d, E, e_pad, d_pad;
-  int x_blocks;          // blocks [0, e_pad) take expert rows (first: the longest), the next x_blocks token rows
+  int cw;                // warps per block
+  int nseg;              // ring segments of one token row (PREP_SEG bytes each, the last one shorter)
+  uint64_t timeout_ns;
+  int *status;
   int8_t *wdig;          // [WD][e_pad][d_pad]
   int *sx;               // [T]
   int *sw;               // [e_pad]
@@ -266,10 +266,30 @@ struct PrepParams {
   double *xdx;           // [T][kRoundList] their dx
 };
 
-constexpr int PREP_WARPS = 4;
+constexpr int PREP_CW_MAX = 16;   // consumer warps per block
+constexpr int PREP_SPW = 3;       // ring slots per warp: one segment read while the next two land
+constexpr int PREP_SEG = 4096;    // bytes of a token row per slot: 8 chunks of 16 bytes per lane
 // fp32 sums of n < 2^16 non-negative terms (each rounded once) are within a
 // factor (1 + 2^-7) of exact; the bound norms are rounded up by it
 constexpr double kRoundUp32 = 1.0 + 0x1p-7;
+
+struct PrepShared {
+  uint64_t full[PREP_CW_MAX * PREP_SPW];
+  double red[3][PREP_CW_MAX];
+  uint32_t redm[PREP_CW_MAX];
+  int abort_flag;
+};
+
+// Barrier 1 joins the block's warps (the expert rows' reductions).
+__device__ __forceinline__ void prep_bar(int nt) { asm volatile("bar.sync 1, %0;" ::"r"(nt) : "memory"); }
+
+// One contiguous copy global -> shared memory completing on an mbarrier
+// (16-byte aligned addresses, size a multiple of 16).
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void *src, uint32_t bytes, uint32_t bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+               "l"((uint64_t)src), "r"(bytes), "r"(bar)
+               : "memory");
+}
 
 // Whether an 8-element chunk of a token row holds an element the digits can
 // round: only exponent fields below ethr can, unless the scale was clamped
@@ -326,40 +346,33 @@ __device__ __noinline__ void token_chunk_rounding(const PrepParams &p, int t, in
   cnt += total;
 }
 
-// Pass 1 on one 8-element chunk: the largest and smallest magnitude (as
-// bf16 pairs: non-negative bf16 values order as their bits) and |x|^2 in fp32.
-__device__ __forceinline__ void token_chunk_scan(uint4 v, __nv_bfloat162 &mx, __nv_bfloat162 &mn, float &l2) {
-  const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-  for (int q = 0; q < 4; ++q) {
-    const uint32_t m = w4[q] & 0x7FFF7FFFu;
-    const __nv_bfloat162 mb = *reinterpret_cast<const __nv_bfloat162 *>(&m);
-    mx = __hmax2(mx, mb);
-    mn = __hmin2(mn, mb);
-    const float lo = __uint_as_float(w4[q] << 16), hi = __uint_as_float(w4[q] & 0xFFFF0000u);
-    l2 = fmaf(lo, lo, fmaf(hi, hi, l2));
-  }
+// The squares of the two bf16 values of w added into the two fp32 lanes of
+// acc (one packed fused multiply-add: each lane rounded once).
+__device__ __forceinline__ void sq_acc2(uint32_t w, unsigned long long &acc) {
+  asm("{\n\t.reg .b64 t;\n\t"
+      "mov.b64 t, {%1, %2};\n\t"
+      "fma.rn.f32x2 %0, t, t, %0;\n\t}\n"
+      : "+l"(acc)
+      : "r"(w << 16), "r"(w & 0xFFFF0000u));
 }
 __device__ __forceinline__ uint32_t bf16x2_bits(__nv_bfloat162 v) { return *reinterpret_cast<uint32_t *>(&v); }
 
-// Shared by the two warps of a token row (half-row mode).
-struct HalfRowShared {
-  uint32_t mb[2], ml[2];
-  float l2[2];
-  double l1[2];
-  int cnt0;
-};
-
-// Pass 2 over one warp's chunks (indices base + lane + 32 c): the rounded
-// elements listed from slot cnt on, |dx| added to l1.
-template <int NC>
-__device__ __forceinline__ void list_rounded(const PrepParams &p, int t, const uint4 (&reg)[NC], int base, int nv,
-                                             bool all, int ethr, double scale_d, double inv, int lane, double &l1,
-                                             int &cnt) {
-#pragma unroll
-  for (int c = 0; c < NC; ++c)
-    if (base + 32 * c < nv && __any_sync(0xffffffffu, chunk_may_round(reg[c], all, ethr)))
-      token_chunk_rounding(p, t, base + lane + 32 * c, reg[c], scale_d, inv, lane, l1, cnt);
+// Pass 1 on one 8-element chunk: the largest and smallest magnitude (as
+// bf16 pairs: non-negative bf16 values order as their bits), |x|^2 in fp32,
+// and the exponent field of the chunk's smallest magnitude (returned).
+__device__ __forceinline__ uint32_t chunk_scan(uint4 v, __nv_bfloat162 &mx, __nv_bfloat162 &mn,
+                                               unsigned long long &acc) {
+  const uint32_t w4[4] = {v.x & 0x7FFF7FFFu, v.y & 0x7FFF7FFFu, v.z & 0x7FFF7FFFu, v.w & 0x7FFF7FFFu};
+  const __nv_bfloat162 *b = reinterpret_cast<const __nv_bfloat162 *>(w4);
+  const __nv_bfloat162 lo = __hmin2(__hmin2(b[0], b[1]), __hmin2(b[2], b[3]));
+  mx = __hmax2(mx, __hmax2(__hmax2(b[0], b[1]), __hmax2(b[2], b[3])));
+  mn = __hmin2(mn, lo);
+  sq_acc2(v.x, acc);
+  sq_acc2(v.y, acc);
+  sq_acc2(v.z, acc);
+  sq_acc2(v.w, acc);
+  const uint32_t lb = bf16x2_bits(lo);
+  return min(lb & 0xFFFFu, lb >> 16) >> 7;
 }
 
 // The row statistics from its largest / smallest magnitude bits and sums.
@@ -388,79 +401,56 @@ __device__ __forceinline__ void write_row_stats(const PrepParams &p, int t, int 
   o[3] = 0.0;
 }
 
-// A token row held in the registers of two warps (half h of d <= 512 NC:
-// chunks NC h .. NC h + NC - 1 of 32 lanes), all loads in flight at once.
-// Both halves meet in shared memory for the scale; half 0 lists its rounded
-// elements first, then half 1 continues the list.
-template <int NC>
-__device__ __forceinline__ void token_half_row(const PrepParams &p, int t, int h, int lane, HalfRowShared &sh) {
-  const unsigned full = 0xffffffffu;
-  const bool live = t < p.T;
-  const uint4 *xr = reinterpret_cast<const uint4 *>(p.x + (size_t)(live ? t : 0) * p.d);
-  const int nv = live ? p.d / 8 : 0;
-  const int base = 32 * NC * h;
-  const uint4 zero = make_uint4(0u, 0u, 0u, 0u);
-  uint4 reg[NC];
-  const uint32_t lo0 = 0u, hi0 = 0x7F7F7F7Fu;
-  __nv_bfloat162 mx = *reinterpret_cast<const __nv_bfloat162 *>(&lo0);
-  __nv_bfloat162 mn = *reinterpret_cast<const __nv_bfloat162 *>(&hi0);
-  float l2 = 0.f;
-#pragma unroll
-  for (int c = 0; c < NC; ++c) reg[c] = base + lane + 32 * c < nv ? __ldg(xr + base + lane + 32 * c) : zero;
-#pragma unroll
-  for (int c = 0; c < NC; ++c)
-    if (base + lane + 32 * c < nv) token_chunk_scan(reg[c], mx, mn, l2);
-  uint32_t mb = bf16x2_bits(mx), ml = bf16x2_bits(mn);
-  mb = warp_max_u(max(mb & 0xFFFFu, mb >> 16));
-  ml = min(ml & 0xFFFFu, ml >> 16);
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    ml = min(ml, __shfl_xor_sync(full, ml, o));
-    l2 += __shfl_xor_sync(full, l2, o);
-  }
-  if (lane == 0) {
-    sh.mb[h] = mb;
-    sh.ml[h] = ml;
-    sh.l2[h] = l2;
-  }
-  __syncthreads();
-  mb = max(sh.mb[0], sh.mb[1]);
-  ml = min(sh.ml[0], sh.ml[1]);
-  int sx, emax, ethr;
-  bool all;
-  row_scale(mb, sx, emax, all, ethr);
-  const double scale_d = pow2d(sx), inv = pow2d(-sx);
-  // (the smallest magnitude tells whether any element can round at all)
-  const bool any_round = live && (all || max((int)(ml >> 7), 1) < ethr);
-  double l1 = 0.0;
-  int cnt = 0;
-  if (any_round && h == 0) list_rounded<NC>(p, t, reg, base, nv, all, ethr, scale_d, inv, lane, l1, cnt);
-  if (lane == 0 && h == 0) sh.cnt0 = cnt;
-  __syncthreads();
-  if (any_round && h == 1) {
-    cnt = sh.cnt0;
-    list_rounded<NC>(p, t, reg, base, nv, all, ethr, scale_d, inv, lane, l1, cnt);
-  }
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) l1 += __shfl_xor_sync(full, l1, o);
-  if (lane == 0) sh.l1[h] = l1;
-  __syncthreads();
-  if (live && h == 1 && lane == 0)
-    write_row_stats(p, t, sx, cnt, sh.l1[0] + sh.l1[1], (double)sh.l2[0] + (double)sh.l2[1]);
+// A warp's ring: PREP_SPW slots of its own; segment q of the warp's work
+// (row j = w + (q / nseg) cw of the block, segment q mod nseg of it) lands in
+// slot q mod PREP_SPW.  The warp copies its own segments in, PREP_SPW - 1
+// ahead of the one it reads.
+struct PrepRing {
+  uint8_t *slots;               // this warp's [PREP_SPW][PREP_SEG]
+  uint64_t *full;               // this warp's [PREP_SPW] barriers
+  volatile int *abort_flag;
+  int w, cw;                    // this warp, warps per block
+  uint32_t nq;                  // segments of this warp's rows
+};
+
+__device__ __forceinline__ void seg_issue(const PrepParams &p, const PrepRing &r, uint32_t q, int lane) {
+  if (lane != 0 || q >= r.nq) return;
+  const int j = r.w + (int)(q / (uint32_t)p.nseg) * r.cw;
+  const uint32_t off = (q % (uint32_t)p.nseg) * PREP_SEG;
+  const uint32_t bytes = min((uint32_t)PREP_SEG, (uint32_t)p.d * 2u - off);
+  const char *src = reinterpret_cast<const char *>(p.x + (size_t)(blockIdx.x + (size_t)j * gridDim.x) * p.d) + off;
+  uint64_t *bar = r.full + q % PREP_SPW;
+  mbar_expect_tx(bar, bytes);
+  bulk_load(smem_u32(r.slots + (size_t)(q % PREP_SPW) * PREP_SEG), src, bytes, smem_u32(bar));
 }
 
-// A token row per warp, streamed twice (rows longer than the register halves hold).
-__device__ __forceinline__ void token_row_stream(const PrepParams &p, int t, int lane) {
+// The warp's q-th segment once it has landed (nullptr: the block gave up).
+__device__ __forceinline__ const uint4 *seg_acquire(const PrepParams &p, const PrepRing &r, uint32_t q, int lane) {
+  uint64_t *bar = r.full + q % PREP_SPW;
+  const uint32_t par = (q / PREP_SPW) & 1u;
+  int good = 1;
+  if (lane == 0) good = wait_bounded(bar, par, r.abort_flag, p.status, kDevTimeoutEpilogue, p.timeout_ns);
+  if (!__shfl_sync(0xffffffffu, good, 0)) return nullptr;
+  // every lane observes the completed phase itself (it stays complete until
+  // the slot is refilled by this warp, so this returns at once)
+  wait_drain(bar, par);
+  return reinterpret_cast<const uint4 *>(r.slots + (size_t)(q % PREP_SPW) * PREP_SEG);
+}
+// Done with segment q: its slot takes segment q + PREP_SPW.
+__device__ __forceinline__ void seg_release(const PrepParams &p, const PrepRing &r, uint32_t q, int lane) {
+  __syncwarp();
+  seg_issue(p, r, q + PREP_SPW, lane);
+}
+
+// The row scale and statistics from the warp's pass-1 partials; then pass 2
+// lists the rounded elements, reading again (from global memory) only the
+// chunks that can round: those whose smallest exponent field (eb: a byte per
+// chunk lane + 32 k) selects them when use_eb, else every chunk.
+__device__ __forceinline__ void finish_row(const PrepParams &p, int t, int lane, __nv_bfloat162 mx,
+                                           __nv_bfloat162 mn, double dl2, bool use_eb, const uint32_t (&eb)[8],
+                                           uint32_t valid) {
   const unsigned full = 0xffffffffu;
-  const uint4 *xr = reinterpret_cast<const uint4 *>(p.x + (size_t)t * p.d);
   const int nv = p.d / 8;
-  const uint4 zero = make_uint4(0u, 0u, 0u, 0u);
-  const uint32_t lo0 = 0u, hi0 = 0x7F7F7F7Fu;
-  __nv_bfloat162 mx = *reinterpret_cast<const __nv_bfloat162 *>(&lo0);
-  __nv_bfloat162 mn = *reinterpret_cast<const __nv_bfloat162 *>(&hi0);
-  float l2 = 0.f;
-#pragma unroll 4
-  for (int i = lane; i < nv; i += 32) token_chunk_scan(__ldg(xr + i), mx, mn, l2);
   uint32_t mb = bf16x2_bits(mx), ml = bf16x2_bits(mn);
   mb = warp_max_u(max(mb & 0xFFFFu, mb >> 16));
   ml = min(ml & 0xFFFFu, ml >> 16);
@@ -470,17 +460,38 @@ __device__ __forceinline__ void token_row_stream(const PrepParams &p, int t, int
   bool all;
   row_scale(mb, sx, emax, all, ethr);
   const double scale_d = pow2d(sx), inv = pow2d(-sx);
+  const uint4 *xg = reinterpret_cast<const uint4 *>(p.x + (size_t)t * p.d);
   double l1 = 0.0;
   int cnt = 0;
+  // (the smallest magnitude tells whether any element can round at all)
   if (all || max((int)(ml >> 7), 1) < ethr) {
-    for (int base = 0; base < nv; base += 32) {
-      const int i = base + lane;
-      const uint4 v = i < nv ? __ldg(xr + i) : zero;
-      if (__any_sync(full, chunk_may_round(v, all, ethr)))
+    if (use_eb) {
+      // chunk k can round when max(its smallest exponent field, 1) < ethr
+      const uint32_t th = ethr > 0 ? (uint32_t)ethr * 0x01010101u : 0u;
+      uint32_t sel = 0;
+#pragma unroll
+      for (int r = 0; r < 8; ++r) {
+        const uint32_t f = __vcmpltu4(__vmaxu4(eb[r], 0x01010101u), th);   // 0xFF per selected byte
+        sel |= ((f & 1u) | ((f >> 7) & 2u) | ((f >> 14) & 4u) | ((f >> 21) & 8u)) << (4 * r);
+      }
+      sel = (all ? 0xFFFFFFFFu : sel) & valid;
+      uint32_t any = __reduce_or_sync(full, sel);
+      while (any) {
+        const int k = __ffs(any) - 1;
+        any &= any - 1;
+        const int i = lane + 32 * k;
+        const uint4 v = (sel >> k) & 1u ? __ldg(xg + i) : make_uint4(0u, 0u, 0u, 0u);
         token_chunk_rounding(p, t, i, v, scale_d, inv, lane, l1, cnt);
+      }
+    } else {
+      for (int base = 0; base < nv; base += 32) {
+        const int i = base + lane;
+        const uint4 v = i < nv ? __ldg(xg + i) : make_uint4(0u, 0u, 0u, 0u);
+        if (__any_sync(full, chunk_may_round(v, all, ethr)))
+          token_chunk_rounding(p, t, i, v, scale_d, inv, lane, l1, cnt);
+      }
     }
   }
-  double dl2 = (double)l2;
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) {
     l1 += __shfl_xor_sync(full, l1, o);
@@ -489,38 +500,65 @@ __device__ __forceinline__ void token_row_stream(const PrepParams &p, int t, int
   if (lane == 0) write_row_stats(p, t, sx, cnt, l1, dl2);
 }
 
-__global__ void __launch_bounds__(32 * PREP_WARPS) route_i8_prep(PrepParams p) {
-  pdl_enter();
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  if (blockIdx.x == 0 && threadIdx.x == 0) *p.flag_count = 0;
-  if ((int)blockIdx.x >= p.e_pad) {
-    // ---------------------------------------------------------- token rows
-    const int nc = (p.d / 8 + 31) / 32;      // 32-lane chunks of a row
-    if (nc <= 32) {
-      // two warps per row, PREP_WARPS / 2 rows per block
-      __shared__ HalfRowShared sh[PREP_WARPS / 2];
-      const int t = (blockIdx.x - p.e_pad) * (PREP_WARPS / 2) + (warp >> 1);
-      const int h = warp & 1;
-      if (nc <= 8) token_half_row<4>(p, t, h, lane, sh[warp >> 1]);
-      else if (nc <= 16) token_half_row<8>(p, t, h, lane, sh[warp >> 1]);
-      else token_half_row<16>(p, t, h, lane, sh[warp >> 1]);
-    } else {
-      const int t = (blockIdx.x - p.e_pad) * PREP_WARPS + warp;
-      if (t < p.T) token_row_stream(p, t, lane);
-    }
-    return;
+// One token row by one warp, its segments taken from the ring in order
+// (lane: chunks lane + 32 k).  For rows of at most 4 segments each chunk's
+// smallest exponent field is kept (a byte per chunk in eight registers), so
+// pass 2 reads only the chunks that can round; longer rows check every chunk
+// in pass 2.  Returns false when the block gave up.
+__device__ __forceinline__ bool token_row(const PrepParams &p, const PrepRing &r, uint32_t &seq, int t, int lane) {
+  const int nv = p.d / 8;
+  const bool short_row = p.nseg <= 4;
+  const uint32_t lo0 = 0u, hi0 = 0x7F7F7F7Fu;
+  __nv_bfloat162 mx[2], mn[2];
+  unsigned long long acc[2] = {0ull, 0ull};
+#pragma unroll
+  for (int a = 0; a < 2; ++a) {
+    mx[a] = *reinterpret_cast<const __nv_bfloat162 *>(&lo0);
+    mn[a] = *reinterpret_cast<const __nv_bfloat162 *>(&hi0);
   }
-  // ------------------------------------------------------------ expert row: a block per row
-  const int e = blockIdx.x;
-  constexpr int NT = 32 * PREP_WARPS;
-  __shared__ double red[3][PREP_WARPS];
-  __shared__ uint32_t redm[PREP_WARPS];
-  const int tid = threadIdx.x;
+  uint32_t eb[8];
+#pragma unroll
+  for (int q = 0; q < 8; ++q) eb[q] = 0xFFFFFFFFu;           // absent chunks: never selected
+  uint32_t valid = 0;
+#pragma unroll 1
+  for (int s = 0; s < p.nseg; ++s) {
+    const uint4 *seg = seg_acquire(p, r, seq, lane);
+    if (!seg) return false;
+    uint32_t w2[2] = {0xFFFFFFFFu, 0xFFFFFFFFu}, vb = 0;
+#pragma unroll
+    for (int kk = 0; kk < 8; ++kk) {
+      if (lane + 32 * kk + 256 * s < nv) {
+        const uint32_t e = chunk_scan(seg[lane + 32 * kk], mx[kk & 1], mn[kk & 1], acc[(kk >> 1) & 1]);
+        const int sh = 8 * (kk & 3);
+        w2[kk >> 2] = (w2[kk >> 2] & ~(0xFFu << sh)) | (e << sh);
+        vb |= 1u << kk;
+      }
+    }
+    seg_release(p, r, seq, lane);
+    ++seq;
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+      if (s == q) {
+        eb[2 * q] = w2[0];
+        eb[2 * q + 1] = w2[1];
+      }
+    if (s < 4) valid |= vb << (8 * s);
+  }
+  const float2 a0 = *reinterpret_cast<const float2 *>(&acc[0]), a1 = *reinterpret_cast<const float2 *>(&acc[1]);
+  const double dl2 = ((double)a0.x + (double)a0.y) + ((double)a1.x + (double)a1.y);
+  finish_row(p, t, lane, __hmax2(mx[0], mx[1]), __hmin2(mn[0], mn[1]), dl2, short_row, eb, valid);
+  return true;
+}
+
+// One expert row (scale, four digit planes, norms) by the block's consumer
+// threads (tid in [0, nt)).
+__device__ __noinline__ void expert_row(const PrepParams &p, int e, int tid, int nt, PrepShared *sh) {
+  const int lane = tid & 31, warp = tid >> 5, nw = nt >> 5;
   const size_t plane = (size_t)p.e_pad * p.d_pad;
   uint32_t *dst = reinterpret_cast<uint32_t *>(p.wdig + (size_t)e * p.d_pad);
   const int n4 = p.d / 4, nq = p.d_pad / 4;
   if (e >= p.E) {
-    for (int i = tid; i < nq; i += NT)
+    for (int i = tid; i < nq; i += nt)
 #pragma unroll
       for (int j = 0; j < WD; ++j) dst[j * plane / 4 + i] = 0u;
     if (tid == 0) {
@@ -532,70 +570,118 @@ __global__ void __launch_bounds__(32 * PREP_WARPS) route_i8_prep(PrepParams p) {
   const float4 *wr = reinterpret_cast<const float4 *>(p.w + (size_t)e * p.d);
   uint32_t mb = 0;
 #pragma unroll 4
-  for (int i = tid; i < n4; i += NT) {
+  for (int i = tid; i < n4; i += nt) {
     const float4 v = __ldg(wr + i);
     mb = max(max(mb, __float_as_uint(v.x) & 0x7FFFFFFFu), __float_as_uint(v.y) & 0x7FFFFFFFu);
     mb = max(max(mb, __float_as_uint(v.z) & 0x7FFFFFFFu), __float_as_uint(v.w) & 0x7FFFFFFFu);
   }
   mb = warp_max_u(mb);
-  if (lane == 0) redm[warp] = mb;
-  __syncthreads();
+  if (lane == 0) sh->redm[warp] = mb;
+  prep_bar(nt);
   mb = 0;
-  for (int w = 0; w < PREP_WARPS; ++w) mb = max(mb, redm[w]);
+  for (int w = 0; w < nw; ++w) mb = max(mb, sh->redm[w]);
   int ew = 0;
   if (mb >= 0x800000u) ew = (int)(mb >> 23) - 126;
   else if (mb != 0) ew = (31 - __clz((int)mb)) - 148;
   const int sw = 30 - ew;
-  const double scale = pow2d(sw), inv = pow2d(-sw);
-  double winf = 0.0, dw2 = 0.0, w3n = 0.0;
+  // v = rne(w 2^sw) from the fp32 fields in integer arithmetic: w 2^sw =
+  // m 2^sh (m the 24-bit significand); the part rounded off, r = m - v 2^k
+  // (k = -sh), gives dw 2^sw = r 2^-k exactly
+  float dw2f = 0.f;                  // sum of (dw 2^sw)^2, each term and sum rounded once in fp32
+  int w3s = 0;                       // sum of b3^2 (exact)
 #pragma unroll 2
-  for (int i = tid; i < nq; i += NT) {
+  for (int i = tid; i < nq; i += nt) {
     const float4 v4 = i < n4 ? __ldg(wr + i) : make_float4(0.f, 0.f, 0.f, 0.f);
-    const float wv[4] = {v4.x, v4.y, v4.z, v4.w};
+    const uint32_t wb[4] = {__float_as_uint(v4.x), __float_as_uint(v4.y), __float_as_uint(v4.z),
+                            __float_as_uint(v4.w)};
     uint32_t packed[WD] = {0, 0, 0, 0};
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
-      const double w = (double)wv[q];
-      const long long v = __double2ll_rn(w * scale);      // |v| <= 2^30, exact scaling
-      const long long u = v + 0x808080;
-      const int b0 = (int)(u >> 24);
-      const int b1 = (int)((u >> 16) & 0xFF) - 128;
-      const int b2 = (int)((u >> 8) & 0xFF) - 128;
-      const int b3 = (int)(u & 0xFF) - 128;
-      packed[0] |= (uint32_t)(b0 & 0xFF) << (8 * q);
-      packed[1] |= (uint32_t)(b1 & 0xFF) << (8 * q);
-      packed[2] |= (uint32_t)(b2 & 0xFF) << (8 * q);
-      packed[3] |= (uint32_t)(b3 & 0xFF) << (8 * q);
-      const double what = (double)v * inv;
-      const double w3 = (double)b3 * inv;
-      winf = fmax(winf, fabs(w));
-      dw2 += (w - what) * (w - what);
-      w3n += w3 * w3;
+      const uint32_t fe = (wb[q] >> 23) & 0xFFu, mant = wb[q] & 0x7FFFFFu;
+      const uint32_t m = fe ? (mant | 0x800000u) : mant;
+      const int sh = (int)max(fe, 1u) - 150 + sw;     // <= 6: |v| <= 2^30
+      uint32_t v = 0;
+      float dws = 0.f;
+      if (sh >= 0) {
+        v = m << sh;
+      } else if (sh >= -25) {
+        const int k = -sh;
+        const uint32_t rem = m & ((1u << k) - 1u), half = 1u << (k - 1);
+        v = m >> k;
+        v += (rem > half || (rem == half && (v & 1u))) ? 1u : 0u;   // ties to even
+        dws = (float)((int)m - (int)(v << k)) * pow2f(-k);           // exact: |m - v 2^k| <= 2^24
+      } else if (m != 0) {
+        dws = 0.5f;                                                  // v = 0 and |w 2^sw| < 1/2
+      }
+      const int vs = (wb[q] >> 31) ? -(int)v : (int)v;
+      const uint32_t u = (uint32_t)(vs + 0x808080);
+      packed[0] |= ((u >> 24) & 0xFFu) << (8 * q);
+      packed[1] |= (((u >> 16) & 0xFFu) ^ 0x80u) << (8 * q);
+      packed[2] |= (((u >> 8) & 0xFFu) ^ 0x80u) << (8 * q);
+      packed[3] |= ((u & 0xFFu) ^ 0x80u) << (8 * q);
+      const int b3 = (int)(u & 0xFFu) - 128;
+      w3s += b3 * b3;
+      dw2f = fmaf(dws, dws, dw2f);
     }
 #pragma unroll
     for (int j = 0; j < WD; ++j) dst[j * plane / 4 + i] = packed[j];
   }
-  winf = warp_max_d(winf);
-  dw2 = warp_sum_d(dw2);
-  w3n = warp_sum_d(w3n);
+  double dw2 = warp_sum_d((double)dw2f);
+  double w3n = warp_sum_d((double)w3s);
   if (lane == 0) {
-    red[0][warp] = winf;
-    red[1][warp] = dw2;
-    red[2][warp] = w3n;
+    sh->red[1][warp] = dw2;
+    sh->red[2][warp] = w3n;
   }
-  __syncthreads();
+  prep_bar(nt);
   if (tid == 0) {
-    for (int w = 1; w < PREP_WARPS; ++w) {
-      winf = fmax(winf, red[0][w]);
-      dw2 += red[1][w];
-      w3n += red[2][w];
+    for (int w = 1; w < nw; ++w) {
+      dw2 += sh->red[1][w];
+      w3n += sh->red[2][w];
     }
     p.sw[e] = sw;
     double *o = p.wst + (size_t)e * 4;
-    o[0] = winf;
-    o[1] = sqrt(dw2) * kRoundUp;
-    o[2] = sqrt(w3n) * kRoundUp;
+    o[0] = (double)__uint_as_float(mb);                             // |w|_inf
+    o[1] = sqrt(dw2) * pow2d(-sw) * (kRoundUp32 * kRoundUp);        // |dw|_2 (fp32 partial sums)
+    o[2] = sqrt(w3n) * pow2d(-sw) * kRoundUp;                       // |w3|_2 (exact sum)
     o[3] = 0.0;
+  }
+}
+
+// One block per SM.  Block b takes the expert rows b, b + G, ... (all its
+// warps together), then the token rows b, b + G, ...: warp w the block's rows
+// j = w, w + cw, ..., segment by segment through its own ring, whose first
+// copies start before the expert rows.
+__global__ void __launch_bounds__(32 * PREP_CW_MAX, 1) route_i8_prep(PrepParams p) {
+  pdl_enter();
+  extern __shared__ __align__(128) uint8_t prep_smem[];
+  const int cw = p.cw, nslots = cw * PREP_SPW;
+  PrepShared *sh = reinterpret_cast<PrepShared *>(prep_smem + (size_t)nslots * PREP_SEG);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < nslots; ++i) mbar_init(&sh->full[i], 1);
+    sh->abort_flag = 0;
+    if (blockIdx.x == 0) *p.flag_count = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  }
+  __syncthreads();
+  const int G = gridDim.x;
+  const int n_rows = p.T > (int)blockIdx.x ? (p.T - 1 - (int)blockIdx.x) / G + 1 : 0;
+  const int my_rows = n_rows > warp ? (n_rows - 1 - warp) / cw + 1 : 0;
+  const PrepRing ring{prep_smem + (size_t)warp * PREP_SPW * PREP_SEG, sh->full + warp * PREP_SPW, &sh->abort_flag,
+                      warp, cw, (uint32_t)my_rows * (uint32_t)p.nseg};
+  for (uint32_t q = 0; q < PREP_SPW; ++q) seg_issue(p, ring, q, lane);
+  for (int e = blockIdx.x; e < p.e_pad; e += G) expert_row(p, e, threadIdx.x, 32 * cw, sh);
+  uint32_t seq = 0;
+  bool ok = true;
+  for (int j = warp; j < n_rows && ok; j += cw) {
+    const int t = blockIdx.x + j * G;
+    ok = token_row(p, ring, seq, t, lane);
+  }
+  if (!ok && lane == 0) {
+    // let this warp's copies in flight land before the block goes away
+    for (uint32_t q = seq; q < seq + PREP_SPW && q < ring.nq; ++q)
+      if (!wait_drain(ring.full + q % PREP_SPW, (q / PREP_SPW) & 1u)) record_status(p.status, kDevTimeoutDrain);
   }
 }
 
@@ -867,6 +953,12 @@ cudaError_t make_map(CUtensorMap *m, CUtensorMapDataType dt, const void *ptr, ui
   return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
+int prep_sm_count() {
+  int dev = 0, n = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  return n > 0 ? n : 148;
+}
+
 template <int N>
 cudaError_t run_gemm(const moe_config &c, const void *x, const I8RoutePlan &t, const I8RouteBuffers &b,
                      int *status, cudaStream_t s) {
@@ -983,9 +1075,11 @@ cudaError_t launch_route_i8_logits(const moe_config &c, const void *x, const flo
   pp.E = c.num_experts;
   pp.e_pad = t.e_pad;
   pp.d_pad = t.d_pad;
-  // two warps per token row while a row fits their registers (d <= 8192), else one
-  const int rows_per_block = (c.hidden / 8 + 31) / 32 <= 32 ? PREP_WARPS / 2 : PREP_WARPS;
-  pp.x_blocks = (c.num_tokens + rows_per_block - 1) / rows_per_block;
+  // one block per SM: 16 warps with three ring segments each
+  pp.cw = PREP_CW_MAX;
+  pp.nseg = (int)((2 * (size_t)c.hidden + PREP_SEG - 1) / PREP_SEG);
+  pp.timeout_ns = wait_timeout_ns();
+  pp.status = status;
   pp.wdig = b.wdig;
   pp.sx = b.sx;
   pp.sw = b.sw;
@@ -995,9 +1089,11 @@ cudaError_t launch_route_i8_logits(const moe_config &c, const void *x, const flo
   pp.flag_count = b.flag_count;
   pp.xidx = b.xidx;
   pp.xdx = b.xdx;
-  const int blocks = pp.x_blocks + t.e_pad;
-  launch_pdl(route_i8_prep, blocks, 32 * PREP_WARPS, 0, s, pp);
-  cudaError_t err = cudaGetLastError();
+  const size_t smem = (size_t)pp.cw * PREP_SPW * PREP_SEG + sizeof(PrepShared);
+  cudaError_t err = cudaFuncSetAttribute(route_i8_prep, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (err != cudaSuccess) return err;
+  launch_pdl(route_i8_prep, std::min(prep_sm_count(), std::max(1, c.num_tokens)), 32 * pp.cw, smem, s, pp);
+  err = cudaGetLastError();
   if (err != cudaSuccess) return err;
   switch (t.n) {
     case 16: return run_gemm<16>(c, x, t, b, status, s);

@@ -242,6 +242,9 @@ I8_CASES = {
     "e200_sigmoid": ROUTER_SHAPES["tc_e200_sigmoid"],
     "e16": ROUTER_SHAPES["tc_e16"],
     "hard_rows": workload("deepseek_v3", T=640, d=1024, F=64, shared_F=0),
+    # rows too long for a consumer warp per 7 KB of ring: fewer consumer warps per block
+    "wide_d12288_e64": workload("switch_top1", T=520, d=12288, F=64, E=64),
+    "wide_d40960_e16": workload("mixtral_prefill", T=512, d=40960, F=64, E=16, k=4),
 }
 
 
