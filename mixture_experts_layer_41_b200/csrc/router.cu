@@ -1017,6 +1017,196 @@ route_select_refine(RouteParams p) {
   }
 }
 
+// Sigmoid group-limited selection over bounded logits (the integer plan),
+// for E <= 256 experts (E a multiple of 8) in groups of G = 8 LG experts, LG a
+// power of two: lane l holds experts 8 l .. 8 l + 7, so a group is LG
+// adjacent lanes.  A group's two largest selection scores come from each
+// lane's own top two and log2(LG) butterfly merges; the kept groups from one
+// rank count over the n_group group scores; the top k from each lane's
+// scores sorted once (keys: score, then the lower expert), k rounds taking
+// the largest head over the warp.  Same choices, weights, bound checks and
+// listing as route_select_refine (ties to the lower index throughout).
+__device__ __forceinline__ uint32_t score_key(float v) {
+  const uint32_t u = __float_as_uint(v);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+__device__ __forceinline__ void cas_desc(unsigned long long &a, unsigned long long &b) {
+  const unsigned long long hi = a > b ? a : b, lo = a > b ? b : a;
+  a = hi;
+  b = lo;
+}
+
+template <int TPB>
+__global__ void __launch_bounds__(256, 2) route_select_group8(RouteParams p) {
+  pdl_enter();
+  constexpr int WPB = 8;
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  const int E = p.E;
+  float *pr = reinterpret_cast<float *>(smem_raw);        // [TPB][E] per-token probabilities
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const unsigned full = 0xffffffffu;
+  const int LG = E / p.n_group / 8;                        // lanes per group
+  const int e0 = 8 * lane;
+  const bool live = e0 < E;
+  float bias[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) bias[j] = live && p.bias ? p.bias[e0 + j] : 0.f;
+
+  for (int i = 0; i < TPB / WPB; ++i) {
+    const int tl = warp * (TPB / WPB) + i;
+    const int t = blockIdx.x * TPB + tl;
+    float4 *prow = reinterpret_cast<float4 *>(pr + (size_t)tl * E + e0);
+    if (t >= p.T) {
+      if (live) prow[0] = prow[1] = make_float4(0.f, 0.f, 0.f, 0.f);
+      continue;
+    }
+    // the logits: the hidden slices added in order; the token's bound factors
+    // loaded while the selection runs
+    double lgd[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) lgd[j] = 0.0;
+    if (live) {
+#pragma unroll 2
+      for (int q = 0; q < p.ks; ++q) {
+        const double2 *row = reinterpret_cast<const double2 *>(p.logits + ((size_t)q * p.T + t) * E + e0);
+#pragma unroll
+        for (int h = 0; h < 4; ++h) {
+          const double2 v = row[h];
+          lgd[2 * h] += v.x;
+          lgd[2 * h + 1] += v.y;
+        }
+      }
+    }
+    const int xcnt = p.xcnt[t];
+    const double xs0 = p.xst[(size_t)t * 4], xs1 = p.xst[(size_t)t * 4 + 1], xs2 = p.xst[(size_t)t * 4 + 2];
+    float prob[8], score[8];
+    float a1 = -INFINITY, a2 = -INFINITY;                  // this lane's two largest scores
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      if (live) {
+        prob[j] = __fdividef(1.f, 1.f + __expf(-(float)lgd[j]));
+        score[j] = prob[j] + bias[j];
+      } else {
+        prob[j] = 0.f;
+        score[j] = -INFINITY;
+      }
+      a2 = fmaxf(a2, fminf(a1, score[j]));
+      a1 = fmaxf(a1, score[j]);
+    }
+    if (live) {
+      prow[0] = make_float4(prob[0], prob[1], prob[2], prob[3]);
+      prow[1] = make_float4(prob[4], prob[5], prob[6], prob[7]);
+    }
+    // the group's two largest: merge the lanes' pairs
+    for (int o = 1; o < LG; o <<= 1) {
+      const float b1 = __shfl_xor_sync(full, a1, o), b2 = __shfl_xor_sync(full, a2, o);
+      a2 = fmaxf(fminf(a1, b1), fmaxf(a2, b2));
+      a1 = fmaxf(a1, b1);
+    }
+    const float gs = a1 + a2;
+    // kept groups: rank of this lane's group among the group scores
+    const int g = lane / LG;
+    int rank = 0;
+    for (int h = 0; h < p.n_group; ++h) {
+      const float gh = __shfl_sync(full, gs, (h * LG) & 31);
+      rank += (gh > gs || (gh == gs && h < g)) ? 1 : 0;
+    }
+    const bool keep = live && g < p.n_group && rank < p.topk_group;
+    // this lane's candidates, sorted: key (score, then the lower expert) in
+    // the high word, 7 - j in the low one; absent experts sort last (0)
+    unsigned long long c[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+      c[j] = live ? ((unsigned long long)score_key(keep ? score[j] : -INFINITY) << 32) | (unsigned)(7 - j) : 0ull;
+    // Batcher's odd-even merge sort on 8 keys, largest first
+    cas_desc(c[0], c[1]); cas_desc(c[2], c[3]); cas_desc(c[4], c[5]); cas_desc(c[6], c[7]);
+    cas_desc(c[0], c[2]); cas_desc(c[1], c[3]); cas_desc(c[4], c[6]); cas_desc(c[5], c[7]);
+    cas_desc(c[1], c[2]); cas_desc(c[5], c[6]);
+    cas_desc(c[0], c[4]); cas_desc(c[1], c[5]); cas_desc(c[2], c[6]); cas_desc(c[3], c[7]);
+    cas_desc(c[2], c[4]); cas_desc(c[3], c[5]);
+    cas_desc(c[1], c[2]); cas_desc(c[3], c[4]); cas_desc(c[5], c[6]);
+    // the k choices (lane r keeps choice r): the largest head, ties to the
+    // lower lane (the lower experts); that lane pops it
+    int my_e = -1;
+    double my_l = 0.0;
+    for (int r = 0; r < p.k; ++r) {
+      const uint32_t hk = (uint32_t)(c[0] >> 32);
+      const uint32_t best = __reduce_max_sync(full, hk);
+      const int wl = (int)__reduce_min_sync(full, hk == best ? (uint32_t)lane : 32u);
+      const int jw = 7 - (int)__shfl_sync(full, (uint32_t)c[0] & 7u, wl);
+      double lv = lgd[0];
+#pragma unroll
+      for (int j = 1; j < 8; ++j)
+        if (jw == j) lv = lgd[j];
+      lv = __shfl_sync(full, lv, wl);
+      if (lane == r) {
+        my_e = 8 * wl + jw;
+        my_l = lv;
+      }
+      if (lane == wl) {
+#pragma unroll
+        for (int j = 0; j < 7; ++j) c[j] = c[j + 1];
+        c[7] = 0ull;
+      }
+    }
+    // the chosen logits with the x-rounding term added where listed; the
+    // token is listed for the exact pass when a chosen bound exceeds tau or
+    // two chosen keys lie within their bounds of each other
+    double bnd = 0.0, key = 0.0, sig = 0.0;
+    const bool mine = lane < p.k;
+    if (mine) {
+      const double *ws = p.wst + (size_t)my_e * 4;
+      if (xcnt <= p.round_list) {
+        const size_t o = (size_t)t * p.round_list;
+        const float *wr = p.w + (size_t)my_e * p.d;
+        double corr = 0.0;
+        for (int q = 0; q < xcnt; ++q) {
+          // (an index outside the row, left by a preparation pass that gave up, adds nothing)
+          const int ix = p.xidx[o + q];
+          if ((unsigned)ix < (unsigned)p.d) corr = fma(p.xdx[o + q], (double)__ldg(wr + ix), corr);
+        }
+        my_l += corr;
+      } else {
+        bnd = xs0 * ws[0];
+      }
+      bnd += xs1 * ws[1] + xs2 * ws[2];
+      sig = 1.0 / (1.0 + exp(-my_l));
+      key = sig + (p.bias ? (double)p.bias[my_e] : 0.0);
+    }
+    bool need = mine && bnd > p.tau;
+    for (int j = 0; j < p.k; ++j) {
+      const double kj = __shfl_sync(full, key, j), bj = __shfl_sync(full, bnd, j);
+      // |key error| <= a quarter of the logit bound
+      if (mine && j != lane && fabs(kj - key) <= bj + bnd) need = true;
+    }
+    if (__any_sync(full, need) && lane == 0) p.flag_list[atomicAdd(p.flag_count, 1)] = t;
+    // weights from these logits (replaced by route_refine_listed for a listed
+    // token); key = the selection score that orders the slots
+    double tot = mine ? sig : 0.0;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) tot += __shfl_xor_sync(full, tot, o);
+    const double wout = (p.norm ? sig / (tot + 1e-20) : sig) * p.scaling;
+    if (!mine) key = -INFINITY;
+    int slot = 0;
+    for (int j = 0; j < p.k; ++j) {
+      const double kj = __shfl_sync(full, key, j);
+      const int ej = __shfl_sync(full, my_e, j);
+      if (kj > key || (kj == key && ej < my_e)) ++slot;
+    }
+    if (mine) {
+      p.ids[(size_t)t * p.k + slot] = my_e;
+      p.wts[(size_t)t * p.k + slot] = (float)wout;
+    }
+  }
+  // the block's probability sums, tokens added in order
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += 32 * WPB) {
+    double sum = 0.0;
+    for (int tl = 0; tl < TPB; ++tl) sum += (double)pr[tl * E + e];
+    p.part[(size_t)blockIdx.x * E + e] = sum;
+  }
+}
+
 // Exact re-weighting of the listed tokens (bounded-logit plan): a block per
 // token (grid-stride over the list), every thread a share of the hidden
 // dimension for eight chosen experts at a time (bf16 x fp32 products exact in
@@ -1229,7 +1419,27 @@ cudaError_t launch_refine_epl(const RouteParams &p, cudaStream_t s) {
   return select_tokens_per_block(p.T) == 8 ? launch_refine_tpb<EPL, 8, 8>(p, s) : launch_refine_tpb<EPL, 32, 8>(p, s);
 }
 
+// The lane-per-8-experts selection for sigmoid group routing over bounded logits
+bool group8_select(const RouteParams &p) {
+  if (!p.approx || p.forced || p.router != MOE_ROUTER_SIGMOID_GROUP || p.E > 256 || p.E % 8 != 0) return false;
+  if (p.n_group < 1 || p.E % p.n_group != 0 || (p.E / p.n_group) % 8 != 0) return false;
+  const int lg = p.E / p.n_group / 8;
+  return (lg & (lg - 1)) == 0 && p.k <= 32;
+}
+
+template <int TPB>
+cudaError_t launch_group8_tpb(const RouteParams &p, cudaStream_t s) {
+  const size_t smem = sizeof(float) * (size_t)TPB * p.E;
+  auto kern = route_select_group8<TPB>;
+  cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (err != cudaSuccess) return err;
+  launch_pdl(kern, (p.T + TPB - 1) / TPB, 256, smem, s, p);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_select(const RouteParams &p, cudaStream_t s) {
+  if (group8_select(p))
+    return select_tokens_per_block(p.T) == 8 ? launch_group8_tpb<8>(p, s) : launch_group8_tpb<32>(p, s);
   if (p.refine || p.approx) {
     if (p.E <= 32) return launch_refine_epl<1>(p, s);
     if (p.E <= 64) return launch_refine_epl<2>(p, s);

@@ -70,6 +70,7 @@ namespace {
 constexpr int TM = 128;                 // tokens per tile (MMA M)
 constexpr int BK = 64;                  // hidden elements per K-block
 constexpr int XS = 3, AS = 3, WS = 3;   // ring depths: token tiles, token digit planes (TMEM), weight digit planes
+static_assert(AS == WS, "one barrier releases a stage of both digit rings");
 constexpr int XD = 3, WD = 4;           // digit planes of a token row and of a weight row
 constexpr int NCLS = 5;                 // accumulator classes i + j = 0..4
 constexpr int CONV_WARPS = 8;
@@ -120,8 +121,8 @@ struct I8Params {
 
 struct I8Shared {
   uint64_t x_full[XS], x_empty[XS];
-  uint64_t a_full[AS], a_empty[AS];
-  uint64_t w_full[WS], w_empty[WS];
+  uint64_t a_full[AS], w_full[WS];
+  uint64_t k_empty[AS];   // stage it % AS of both the token digits and the weight digits is free again
   uint64_t acc_full, drain;
   uint64_t tmem_full;   // the accumulators are allocated (warp 1)
   uint64_t acc_read;    // every converter warp has read them (warp 1 frees TMEM)
@@ -710,11 +711,10 @@ route_i8_gemm(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ 
     }
     for (int s = 0; s < AS; ++s) {
       mbar_init(&st->a_full[s], CONV_WARPS);
-      mbar_init(&st->a_empty[s], 1);
+      mbar_init(&st->k_empty[s], 1);
     }
     for (int s = 0; s < WS; ++s) {
       mbar_init(&st->w_full[s], 1);
-      mbar_init(&st->w_empty[s], 1);
     }
     mbar_init(&st->acc_full, 1);
     mbar_init(&st->drain, 1);
@@ -747,7 +747,7 @@ route_i8_gemm(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ 
         tma_load_2d(smem_u32(xt + xs * S::X_BYTES), &mapX, smem_u32(&st->x_full[xs]), kx, t0);
         ix = it + 1;
         const int ws = it % WS;
-        if (!wait_bounded(&st->w_empty[ws], ((it / WS) & 1) ^ 1, abort_flag, p.status, kDevTimeoutProducer,
+        if (!wait_bounded(&st->k_empty[ws], ((it / WS) & 1) ^ 1, abort_flag, p.status, kDevTimeoutProducer,
                           p.timeout_ns)) {
           ok = false;
           break;
@@ -796,8 +796,7 @@ route_i8_gemm(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ 
           for (int i = 0; i < XD; ++i)
             tc_mma_i8_ts(tmem_base + (uint32_t)(i * N), ta + (uint32_t)(i * (BK / 4) + kk * 8), db + (uint64_t)(kk * 2),
                          i < XD - 1 ? S::IDESC4 : S::IDESC3, 1u);
-        tc_commit(&st->a_empty[as]);
-        tc_commit(&st->w_empty[ws]);
+        tc_commit(&st->k_empty[as]);   // one commit frees both operands' stage
       }
       if (ok) tc_commit(&st->acc_full);
       tc_commit(&st->drain);
@@ -838,7 +837,7 @@ route_i8_gemm(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ 
     for (int it = 0; ok && it < kb_n; ++it) {
       const int xs = it % XS, as = it % AS;
       if (!wait_bounded(&st->x_full[xs], (it / XS) & 1, abort_flag, p.status, kDevTimeoutEpilogue, p.timeout_ns) ||
-          !wait_bounded(&st->a_empty[as], ((it / AS) & 1) ^ 1, abort_flag, p.status, kDevTimeoutEpilogue,
+          !wait_bounded(&st->k_empty[as], ((it / AS) & 1) ^ 1, abort_flag, p.status, kDevTimeoutEpilogue,
                         p.timeout_ns)) {
         ok = false;
         break;

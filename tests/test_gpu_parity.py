@@ -242,7 +242,14 @@ I8_CASES = {
     "e200_sigmoid": ROUTER_SHAPES["tc_e200_sigmoid"],
     "e16": ROUTER_SHAPES["tc_e16"],
     "hard_rows": workload("deepseek_v3", T=640, d=1024, F=64, shared_F=0),
-    # rows too long for a consumer warp per 7 KB of ring: fewer consumer warps per block
+    # sigmoid groups of 8, 16 and 64 experts: 1, 2 and 8 lanes per group in the selection
+    "sigmoid_e64_g8": workload("deepseek_v3", T=600, d=256, F=64, E=64, n_group=8, topk_group=3, k=6,
+                               shared_F=0),
+    "sigmoid_e96_g6": workload("deepseek_v3", T=530, d=320, F=64, E=96, n_group=6, topk_group=2, k=5,
+                               shared_F=0),
+    "sigmoid_e256_g4": workload("deepseek_v3", T=520, d=512, F=64, E=256, n_group=4, topk_group=2, k=8,
+                                shared_F=0),
+    # long token rows: many ring segments per row
     "wide_d12288_e64": workload("switch_top1", T=520, d=12288, F=64, E=64),
     "wide_d40960_e16": workload("mixtral_prefill", T=512, d=40960, F=64, E=16, k=4),
 }
