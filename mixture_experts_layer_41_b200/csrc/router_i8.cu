@@ -252,7 +252,7 @@ struct PrepParams {
   const __nv_bfloat16 *x;
   const float *w;
   int T, d, E, e_pad, d_pad;
-  int cw;                // warps per block
+  int cw;                // token-row warps per block (PREP_EW expert-row warps follow)
   int nseg;              // ring segments of one token row (PREP_SEG bytes each, the last one shorter)
   uint64_t timeout_ns;
   int *status;
@@ -267,7 +267,8 @@ struct PrepParams {
   double *xdx;           // [T][kRoundList] their dx
 };
 
-constexpr int PREP_CW_MAX = 16;   // consumer warps per block
+constexpr int PREP_CW_MAX = 16;   // token-row warps per block
+constexpr int PREP_EW = 4;        // expert-row warps per block
 constexpr int PREP_SPW = 3;       // ring slots per warp: one segment read while the next two land
 constexpr int PREP_SEG = 4096;    // bytes of a token row per slot: 8 chunks of 16 bytes per lane
 // fp32 sums of n < 2^16 non-negative terms (each rounded once) are within a
@@ -276,12 +277,12 @@ constexpr double kRoundUp32 = 1.0 + 0x1p-7;
 
 struct PrepShared {
   uint64_t full[PREP_CW_MAX * PREP_SPW];
-  double red[3][PREP_CW_MAX];
-  uint32_t redm[PREP_CW_MAX];
+  double red[3][PREP_EW];
+  uint32_t redm[PREP_EW];
   int abort_flag;
 };
 
-// Barrier 1 joins the block's warps (the expert rows' reductions).
+// Barrier 1 joins the expert-row warps (their reductions).
 __device__ __forceinline__ void prep_bar(int nt) { asm volatile("bar.sync 1, %0;" ::"r"(nt) : "memory"); }
 
 // One contiguous copy global -> shared memory completing on an mbarrier
@@ -551,8 +552,8 @@ __device__ __forceinline__ bool token_row(const PrepParams &p, const PrepRing &r
   return true;
 }
 
-// One expert row (scale, four digit planes, norms) by the block's consumer
-// threads (tid in [0, nt)).
+// One expert row (scale, four digit planes, norms) by the block's
+// expert-row warps (tid in [0, nt)).
 __device__ __noinline__ void expert_row(const PrepParams &p, int e, int tid, int nt, PrepShared *sh) {
   const int lane = tid & 31, warp = tid >> 5, nw = nt >> 5;
   const size_t plane = (size_t)p.e_pad * p.d_pad;
@@ -648,11 +649,11 @@ __device__ __noinline__ void expert_row(const PrepParams &p, int e, int tid, int
   }
 }
 
-// One block per SM.  Block b takes the expert rows b, b + G, ... (all its
-// warps together), then the token rows b, b + G, ...: warp w the block's rows
-// j = w, w + cw, ..., segment by segment through its own ring, whose first
-// copies start before the expert rows.
-__global__ void __launch_bounds__(32 * PREP_CW_MAX, 1) route_i8_prep(PrepParams p) {
+// One block per SM: warps 0 .. cw - 1 take the block's token rows (block b:
+// rows b, b + G, ...; warp w the block's rows j = w, w + cw, ...), segment by
+// segment through their own rings, while warps cw .. cw + PREP_EW - 1 take
+// the expert rows b, b + G, ... together.
+__global__ void __launch_bounds__(32 * (PREP_CW_MAX + PREP_EW), 1) route_i8_prep(PrepParams p) {
   pdl_enter();
   extern __shared__ __align__(128) uint8_t prep_smem[];
   const int cw = p.cw, nslots = cw * PREP_SPW;
@@ -667,12 +668,17 @@ __global__ void __launch_bounds__(32 * PREP_CW_MAX, 1) route_i8_prep(PrepParams 
   }
   __syncthreads();
   const int G = gridDim.x;
+  if (warp >= cw) {
+    // ------------------------------------------------------------ expert rows
+    for (int e = blockIdx.x; e < p.e_pad; e += G) expert_row(p, e, threadIdx.x - 32 * cw, 32 * PREP_EW, sh);
+    return;
+  }
+  // -------------------------------------------------------------- token rows
   const int n_rows = p.T > (int)blockIdx.x ? (p.T - 1 - (int)blockIdx.x) / G + 1 : 0;
   const int my_rows = n_rows > warp ? (n_rows - 1 - warp) / cw + 1 : 0;
   const PrepRing ring{prep_smem + (size_t)warp * PREP_SPW * PREP_SEG, sh->full + warp * PREP_SPW, &sh->abort_flag,
                       warp, cw, (uint32_t)my_rows * (uint32_t)p.nseg};
   for (uint32_t q = 0; q < PREP_SPW; ++q) seg_issue(p, ring, q, lane);
-  for (int e = blockIdx.x; e < p.e_pad; e += G) expert_row(p, e, threadIdx.x, 32 * cw, sh);
   uint32_t seq = 0;
   bool ok = true;
   for (int j = warp; j < n_rows && ok; j += cw) {
@@ -1074,7 +1080,8 @@ cudaError_t launch_route_i8_logits(const moe_config &c, const void *x, const flo
   pp.E = c.num_experts;
   pp.e_pad = t.e_pad;
   pp.d_pad = t.d_pad;
-  // one block per SM: 16 warps with three ring segments each
+  // one block per SM: 16 token-row warps with three ring segments each, and
+  // the expert-row warps
   pp.cw = PREP_CW_MAX;
   pp.nseg = (int)((2 * (size_t)c.hidden + PREP_SEG - 1) / PREP_SEG);
   pp.timeout_ns = wait_timeout_ns();
@@ -1091,7 +1098,7 @@ cudaError_t launch_route_i8_logits(const moe_config &c, const void *x, const flo
   const size_t smem = (size_t)pp.cw * PREP_SPW * PREP_SEG + sizeof(PrepShared);
   cudaError_t err = cudaFuncSetAttribute(route_i8_prep, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (err != cudaSuccess) return err;
-  launch_pdl(route_i8_prep, std::min(prep_sm_count(), std::max(1, c.num_tokens)), 32 * pp.cw, smem, s, pp);
+  launch_pdl(route_i8_prep, prep_sm_count(), 32 * (pp.cw + PREP_EW), smem, s, pp);
   err = cudaGetLastError();
   if (err != cudaSuccess) return err;
   switch (t.n) {
