@@ -1329,7 +1329,7 @@ __global__ void __launch_bounds__(RL_THREADS) route_refine_listed(RouteParams p)
 // flight, then the 32 warp sums are added in warp order.  Deterministic for a
 // given T and E.
 constexpr int FIN_WARPS = 32;
-constexpr int FIN_UNROLL = 8;
+constexpr int FIN_UNROLL = 16;
 __global__ void __launch_bounds__(32 * FIN_WARPS) route_finalize(const double *part, int nb, int E, float *prob_sum) {
   pdl_enter();
   __shared__ double ws[FIN_WARPS][32];
