@@ -11,11 +11,12 @@
 // the integer tensor-core GEMM of router_i8.cu (float64 partials per hidden
 // slice, each logit within a computed bound of exact; or, with
 // MOE_ROUTER_TC=bf16, the selection-grade bf16 GEMMs of router_tc.cu);
-// route_select_refine then selects from those logits in fp32 and weights the
-// k chosen experts from their float64 logits: with bounded logits after
-// adding the x-rounding term exactly, listing for route_refine_listed the
-// tokens whose bound could matter; with selection-grade ones after an exact
-// recomputation.  All other cases stay on the CUDA cores: fp32 products summed over runs of 8 elements,
+// route_select_refine (or route_select_group8, a lane per eight experts, for
+// sigmoid groups of 8, 16, 32, ... experts over bounded logits) then selects
+// from those logits in fp32 and weights the k chosen experts from their
+// float64 logits: with bounded logits after adding the x-rounding term
+// exactly, listing for route_refine_listed the tokens whose bound could
+// matter; with selection-grade ones after an exact recomputation.  All other cases stay on the CUDA cores: fp32 products summed over runs of 8 elements,
 // the runs added in float64 (a straight fp32 sum over d = 7168 misses the
 // 1e-6 weight bound); scores, selection and weights are float64 and rounded
 // to float32 on the store.  CUDA-core shapes:

@@ -34,9 +34,11 @@
 // could still move a weight past the routing tolerance, or swap two chosen
 // experts, are recomputed exactly (route_refine_listed in router.cu).
 //
-// route_i8_prep   a block per expert row (scale, four digit planes
-//                 [4][e_pad][d_pad], norms), then two warps per token row held
-//                 in registers (scale, |x|_2, the list of rounded elements).
+// route_i8_prep   one block per SM: sixteen warps stream the token rows
+//                 (scale, |x|_2, the list of rounded elements) through ring
+//                 slots of their own filled by bulk copies; four warps split
+//                 the expert rows (scale, four digit planes [4][e_pad][d_pad],
+//                 norms) in integer arithmetic.
 // route_i8_gemm   grid (N-expert tile, 128-token tile, hidden slice), one CTA
 //                 per SM:
 //   warp 0        TMA producer: the bf16 token tile (128 x 64, 128-byte
