@@ -154,6 +154,18 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
+// Non-blocking test of the phase with the given parity.
+__device__ __forceinline__ bool mbar_test_wait(uint64_t *bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
 __device__ __forceinline__ uint64_t global_ns() {
   uint64_t t;
   asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
@@ -741,31 +753,45 @@ route_i8_gemm(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
+      // The two rings are filled independently, each as soon as its next
+      // stage is free, so the token tiles run up to XS K-blocks ahead of the
+      // MMAs whatever the weight ring waits for.
       int ix = 0, iw = 0;   // K-blocks issued on each ring
       bool ok = true;
-      for (int it = 0; it < kb_n && ok; ++it) {
-        const int kx = (kb0 + it) * BK;
-        const int xs = it % XS;
-        if (!wait_bounded(&st->x_empty[xs], ((it / XS) & 1) ^ 1, abort_flag, p.status, kDevTimeoutProducer,
-                          p.timeout_ns)) {
-          ok = false;
-          break;
+      uint64_t t_idle = 0;  // start of the current wait without progress (0: none)
+      uint32_t spins = 0;
+      while (ok && (ix < kb_n || iw < kb_n)) {
+        bool progressed = false;
+        if (ix < kb_n && mbar_test_wait(&st->x_empty[ix % XS], ((ix / XS) & 1) ^ 1)) {
+          mbar_expect_tx(&st->x_full[ix % XS], S::X_BYTES);
+          tma_load_2d(smem_u32(xt + (ix % XS) * S::X_BYTES), &mapX, smem_u32(&st->x_full[ix % XS]),
+                      (kb0 + ix) * BK, t0);
+          ++ix;
+          progressed = true;
         }
-        mbar_expect_tx(&st->x_full[xs], S::X_BYTES);
-        tma_load_2d(smem_u32(xt + xs * S::X_BYTES), &mapX, smem_u32(&st->x_full[xs]), kx, t0);
-        ix = it + 1;
-        const int ws = it % WS;
-        if (!wait_bounded(&st->k_empty[ws], ((it / WS) & 1) ^ 1, abort_flag, p.status, kDevTimeoutProducer,
-                          p.timeout_ns)) {
-          ok = false;
-          break;
-        }
-        mbar_expect_tx(&st->w_full[ws], S::W_BYTES);
+        if (iw < kb_n && mbar_test_wait(&st->k_empty[iw % WS], ((iw / WS) & 1) ^ 1)) {
+          const int ws = iw % WS;
+          mbar_expect_tx(&st->w_full[ws], S::W_BYTES);
 #pragma unroll
-        for (int j = 0; j < WD; ++j)
-          tma_load_2d(smem_u32(wt + ws * S::W_BYTES + j * S::W_PLANE), &mapW, smem_u32(&st->w_full[ws]), kx,
-                      j * e_pad + e0);
-        iw = it + 1;
+          for (int j = 0; j < WD; ++j)
+            tma_load_2d(smem_u32(wt + ws * S::W_BYTES + j * S::W_PLANE), &mapW, smem_u32(&st->w_full[ws]),
+                        (kb0 + iw) * BK, j * e_pad + e0);
+          ++iw;
+          progressed = true;
+        }
+        if (progressed) {
+          t_idle = 0;
+          continue;
+        }
+        if (*abort_flag) {
+          ok = false;
+        } else if (t_idle == 0) {
+          t_idle = global_ns();
+        } else if ((++spins & 31u) == 0 && global_ns() - t_idle > p.timeout_ns) {
+          *abort_flag = 1;
+          record_status(p.status, kDevTimeoutProducer);
+          ok = false;
+        }
       }
       if (!ok) {
         for (int i = ix > XS ? ix - XS : 0; i < ix; ++i)
