@@ -1214,15 +1214,14 @@ __global__ void __launch_bounds__(256, 2) route_select_group8(RouteParams p) {
 // float64, float64 sums reduced in a fixed order), then warp 0 weights and
 // orders the slots from the exact logits as the selection pass would.
 constexpr int RL_THREADS = 1024;
-__global__ void __launch_bounds__(RL_THREADS) route_refine_listed(RouteParams p) {
-  pdl_enter();
+__device__ __forceinline__ void refine_listed(const RouteParams &p, int bx, int nbx) {
   __shared__ double red[RL_THREADS / 32][8];
   __shared__ double lsh[32];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const unsigned full = 0xffffffffu;
   const int n = *p.flag_count;
   const bool softmax = p.router == MOE_ROUTER_SOFTMAX_TOPK;
-  for (int j = blockIdx.x; j < n; j += gridDim.x) {
+  for (int j = bx; j < n; j += nbx) {
     const int t = p.flag_list[j];
     const uint4 *xr = reinterpret_cast<const uint4 *>(static_cast<const __nv_bfloat16 *>(p.x) + (size_t)t * p.d);
     for (int r0 = 0; r0 < p.k; r0 += 8) {
@@ -1331,11 +1330,10 @@ __global__ void __launch_bounds__(RL_THREADS) route_refine_listed(RouteParams p)
 // given T and E.
 constexpr int FIN_WARPS = 32;
 constexpr int FIN_UNROLL = 16;
-__global__ void __launch_bounds__(32 * FIN_WARPS) route_finalize(const double *part, int nb, int E, float *prob_sum) {
-  pdl_enter();
+__device__ __forceinline__ void finalize_block(const double *part, int nb, int E, float *prob_sum, int bx) {
   __shared__ double ws[FIN_WARPS][32];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int e = blockIdx.x * 32 + lane;
+  const int e = bx * 32 + lane;
   double s = 0.0;
   if (e < E) {
     for (int b0 = warp; b0 < nb; b0 += FIN_WARPS * FIN_UNROLL) {
@@ -1357,6 +1355,22 @@ __global__ void __launch_bounds__(32 * FIN_WARPS) route_finalize(const double *p
     for (int w = 0; w < FIN_WARPS; ++w) t += ws[w][lane];
     prob_sum[e] = (float)t;
   }
+}
+
+__global__ void __launch_bounds__(32 * FIN_WARPS) route_finalize(const double *part, int nb, int E, float *prob_sum) {
+  pdl_enter();
+  finalize_block(part, nb, E, prob_sum, blockIdx.x);
+}
+
+// The bounded-logit plan's last launch: blocks [0, fin_blocks) add the
+// probability-sum rows (route_finalize), the rest re-weight the listed tokens
+// exactly (both only read what the selection wrote).
+static_assert(RL_THREADS == 32 * FIN_WARPS, "one block shape for both halves");
+__global__ void __launch_bounds__(RL_THREADS) route_finish_listed(RouteParams p, const double *part, int nb,
+                                                                  float *prob_sum, int fin_blocks) {
+  pdl_enter();
+  if ((int)blockIdx.x < fin_blocks) finalize_block(part, nb, p.E, prob_sum, blockIdx.x);
+  else refine_listed(p, blockIdx.x - fin_blocks, gridDim.x - fin_blocks);
 }
 
 template <int EPL, int TPW, bool BF16, bool SPLIT>
@@ -1603,11 +1617,6 @@ cudaError_t launch_route(const moe_config &c, const void *x, const float *w_rout
     p.flag_list = b.flag_list;
     err = launch_route_i8_logits(c, x, w_router, t, b, status, s);
     if (err == cudaSuccess) err = launch_select(p, s);
-    if (err == cudaSuccess) {
-      const int grid = c.num_tokens < 148 ? c.num_tokens : 148;
-      launch_pdl(route_refine_listed, grid, RL_THREADS, 0, s, p);
-      err = cudaGetLastError();
-    }
   } else if (plan.tc) {
     __nv_bfloat16 *wsplit =
         reinterpret_cast<__nv_bfloat16 *>(reinterpret_cast<char *>(logits) + tc_logits_part(c, plan.ks));
@@ -1622,7 +1631,15 @@ cudaError_t launch_route(const moe_config &c, const void *x, const float *w_rout
   const int nb = plan.tc || plan.i8 || plan.split ? (c.num_tokens + select_tokens_per_block(c.num_tokens) - 1) /
                                              select_tokens_per_block(c.num_tokens)
                                        : route_blocks(c);
-  launch_pdl(route_finalize, (c.num_experts + 31) / 32, 32 * FIN_WARPS, 0, s, route_part, nb, c.num_experts, prob_sum);
+  const int fin_blocks = (c.num_experts + 31) / 32;
+  if (plan.i8) {
+    // the listed tokens' exact re-weighting shares the launch
+    const int listed_blocks = c.num_tokens < 148 ? c.num_tokens : 148;
+    launch_pdl(route_finish_listed, fin_blocks + listed_blocks, RL_THREADS, 0, s, p, (const double *)route_part, nb,
+               prob_sum, fin_blocks);
+  } else {
+    launch_pdl(route_finalize, fin_blocks, 32 * FIN_WARPS, 0, s, route_part, nb, c.num_experts, prob_sum);
+  }
   return cudaGetLastError();
 }
 
