@@ -15,7 +15,7 @@
 // sigmoid groups of 8, 16, 32, ... experts over bounded logits) then selects
 // from those logits in fp32 and weights the k chosen experts from their
 // float64 logits: with bounded logits after adding the x-rounding term
-// exactly, listing for route_refine_listed the tokens whose bound could
+// exactly, listing for route_finish_listed the tokens whose bound could
 // matter; with selection-grade ones after an exact recomputation.  All other cases stay on the CUDA cores: fp32 products summed over runs of 8 elements,
 // the runs added in float64 (a straight fp32 sum over d = 7168 misses the
 // 1e-6 weight bound); scores, selection and weights are float64 and rounded
@@ -35,7 +35,8 @@
 //                 memory, then selects with one warp per token.
 // Every selecting block writes one float64 probability sum per (block,
 // expert); route_finalize adds the rows in order, so prob_sum is
-// deterministic.
+// deterministic (on the bounded-logit plan route_finish_listed does it, in
+// the same launch as the listed tokens' exact re-weighting).
 #include "common.cuh"
 
 #include <math.h>
@@ -79,7 +80,7 @@ struct RouteParams {
   const double *xdx;
   int round_list;
   // tokens whose chosen logits need the exact recomputation are appended
-  // here (the count zeroed by the preparation pass) for route_refine_listed
+  // here (the count zeroed by the preparation pass) for route_finish_listed
   int *flag_count, *flag_list;
 };
 
@@ -950,7 +951,7 @@ route_select_refine(RouteParams p) {
         }
       exact = __any_sync(full, need);
       if (exact) {
-        // the provisional weights below are replaced by route_refine_listed
+        // the provisional weights below are replaced by route_finish_listed
         if (lane == 0) p.flag_list[atomicAdd(p.flag_count, 1)] = t;
         exact = false;
       }
@@ -1181,7 +1182,7 @@ __global__ void __launch_bounds__(256, 2) route_select_group8(RouteParams p) {
       if (mine && j != lane && fabs(kj - key) <= bj + bnd) need = true;
     }
     if (__any_sync(full, need) && lane == 0) p.flag_list[atomicAdd(p.flag_count, 1)] = t;
-    // weights from these logits (replaced by route_refine_listed for a listed
+    // weights from these logits (replaced by route_finish_listed for a listed
     // token); key = the selection score that orders the slots
     double tot = mine ? sig : 0.0;
 #pragma unroll

@@ -32,7 +32,7 @@
 // selection pass adds dx . w exactly for the chosen experts; the rest of the
 // bound is then about 1e-7 on the workloads' recipes.  Tokens whose bound
 // could still move a weight past the routing tolerance, or swap two chosen
-// experts, are recomputed exactly (route_refine_listed in router.cu).
+// experts, are recomputed exactly (route_finish_listed in router.cu).
 //
 // route_i8_prep   one block per SM: sixteen warps stream the token rows
 //                 (scale, |x|_2, the list of rounded elements) through ring
