@@ -204,7 +204,7 @@ int64_t moe_kernel_launches(void);
 
 /* Bound on every on-chip barrier wait of the tensor-core kernels (grouped
  * GEMMs, the 4-bit tcgen05 FFN, the router's integer and bf16 tensor-core
- * logits), in nanoseconds of the GPU's global
+ * logits and the integer plan's token-row streaming), in nanoseconds of the GPU's global
  * timer, for the launches that follow (process-wide, all threads).  When a
  * wait runs out, the kernel records where in the workspace status word
  * (moe_workspace_status: MOE_ERR_DEVICE, "... wait timed out"), lets the
