@@ -47,6 +47,7 @@ namespace moe {
 namespace {
 
 constexpr int KC = 32;      // hidden-dimension chunk staged in shared memory
+constexpr int kMaxSplitSlices = 16;   // hidden slices of the split pass (their sums are read at once)
 constexpr int RUN = 8;      // fp32 run length before the float64 add
 constexpr int WARPS = kRouteThreads / 32;
 
@@ -88,13 +89,18 @@ __device__ __forceinline__ void argmax_merge(double &v, int &i, double ov, int o
   if (ov > v || (ov == v && oi < i)) { v = ov; i = oi; }
 }
 
+// Warp arg-max of (v, i), ties to the lower index (i >= 0): three warp
+// reductions on the order-preserving 64-bit image of v.
 __device__ __forceinline__ void warp_argmax(double &v, int &i) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    const double ov = __shfl_xor_sync(0xffffffffu, v, o);
-    const int oi = __shfl_xor_sync(0xffffffffu, i, o);
-    argmax_merge(v, i, ov, oi);
-  }
+  const unsigned full = 0xffffffffu;
+  const unsigned long long u = (unsigned long long)__double_as_longlong(v);
+  const unsigned long long key = (u >> 63) ? ~u : (u | 0x8000000000000000ull);
+  const uint32_t hi = (uint32_t)(key >> 32), lo = (uint32_t)key;
+  const uint32_t mhi = __reduce_max_sync(full, hi);
+  const uint32_t mlo = __reduce_max_sync(full, hi == mhi ? lo : 0u);
+  i = (int)__reduce_min_sync(full, hi == mhi && lo == mlo ? (uint32_t)i : 0xFFFFFFFFu);
+  const unsigned long long mk = ((unsigned long long)mhi << 32) | mlo;
+  v = __longlong_as_double((long long)((mk >> 63) ? (mk & 0x7FFFFFFFFFFFFFFFull) : ~mk));
 }
 
 __device__ __forceinline__ double warp_sum(double v) {
@@ -650,27 +656,22 @@ __device__ __forceinline__ void select_tile(const RouteParams &p, int tile, unsi
   const int E = p.E;
   const int tb = tile * TPB;
   constexpr int NT = 32 * WPB;
-  // every thread sums the slices of 4 (token, expert) logits at a time, in
-  // slice order, with the loads of a slice in flight together
+  // every thread sums the slices of its (token, expert) logits in slice
+  // order, the loads of all slices of one logit in flight together
   const int n = TPB * E;
-  for (int o0 = threadIdx.x; o0 < n; o0 += 4 * NT) {
-    double sacc[4];
+  for (int o = threadIdx.x; o < n; o += NT) {
+    // all of the entry's slices (at most 16) in flight at once, then added in order
+    const int t = tb + o / E;
+    const bool live = t < p.T;
+    const double *src = p.logits + (size_t)(live ? t : 0) * E + o % E;
+    double v[kMaxSplitSlices];
 #pragma unroll
-    for (int u = 0; u < 4; ++u) sacc[u] = 0.0;
-#pragma unroll 4
-    for (int q = 0; q < p.ks; ++q) {
+    for (int q = 0; q < kMaxSplitSlices; ++q) v[q] = live && q < p.ks ? src[(size_t)q * p.T * E] : 0.0;
+    double acc = 0.0;
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int o = o0 + u * NT;
-        const int t = tb + o / E;
-        if (o < n && t < p.T) sacc[u] += p.logits[((size_t)q * p.T + t) * E + o % E];
-      }
-    }
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const int o = o0 + u * NT;
-      if (o < n) lgs[o] = sacc[u];
-    }
+    for (int q = 0; q < kMaxSplitSlices; ++q)
+      if (q < p.ks) acc += v[q];
+    lgs[o] = acc;
   }
   __syncthreads();
   double psum[EPL];
@@ -1528,7 +1529,7 @@ RoutePlan route_plan(const moe_config &c, bool allow_split) {
     // (each a multiple of 32 elements, at most 16) as it takes to fill the GPU
     const int base = ((c.num_tokens + 7) / 8) * ((c.num_experts + 31) / 32);
     int ks = (sms + base - 1) / base;
-    const int max_ks = c.hidden / KC < 16 ? c.hidden / KC : 16;
+    const int max_ks = c.hidden / KC < kMaxSplitSlices ? c.hidden / KC : kMaxSplitSlices;
     ks = ks < max_ks ? ks : max_ks;
     ks = ks < 1 ? 1 : ks;
     int kchunk = (c.hidden + ks - 1) / ks;
