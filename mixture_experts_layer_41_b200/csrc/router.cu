@@ -1526,9 +1526,11 @@ RoutePlan route_plan(const moe_config &c, bool allow_split) {
   const bool vec_ok = c.act_dtype == MOE_BF16 ? (c.hidden % 8 == 0) : (c.hidden % 4 == 0);
   if (allow_split && vec_ok && whole_row_blocks < sms) {
     // 8-token tiles x 32-expert slices, then as many hidden-dimension slices
-    // (each a multiple of 32 elements, at most 16) as it takes to fill the GPU
+    // (each a multiple of 32 elements, at most 16) as it takes to give every
+    // SM four blocks: a block's chain of staged 32-element chunks is what
+    // takes the time at these sizes, so shorter slices finish sooner
     const int base = ((c.num_tokens + 7) / 8) * ((c.num_experts + 31) / 32);
-    int ks = (sms + base - 1) / base;
+    int ks = (4 * sms + base - 1) / base;
     const int max_ks = c.hidden / KC < kMaxSplitSlices ? c.hidden / KC : kMaxSplitSlices;
     ks = ks < max_ks ? ks : max_ks;
     ks = ks < 1 ? 1 : ks;
