@@ -60,7 +60,7 @@ typedef enum moe_status {
   MOE_ERR_INVALID_ARG = 1,         /* shape, null or misaligned pointer, bad enum */
   MOE_ERR_INVALID_TOPK = 2,        /* top_k outside [1, num_experts] (blog: InvalidTopK) */
   MOE_ERR_CAPACITY_TOO_TIGHT = 3,  /* 0 < capacity_factor < 1 (blog: CapacityTooTight) */
-  MOE_ERR_UNSUPPORTED = 4,         /* valid MoE, but a shape/dtype this build has no kernel for */
+  MOE_ERR_UNSUPPORTED = 4,         /* valid MoE, but a shape/dtype this library has no kernel for */
   MOE_ERR_WORKSPACE = 5,           /* ws NULL or smaller than moe_workspace_size() */
   MOE_ERR_CUDA = 6,                /* CUDA runtime error; text in moe_last_error() */
   MOE_ERR_DEVICE = 7               /* a kernel recorded a device-side failure (moe_workspace_status) */

@@ -347,7 +347,7 @@ const char *moe_status_string(moe_status s) {
     case MOE_ERR_INVALID_ARG: return "invalid argument";
     case MOE_ERR_INVALID_TOPK: return "top_k outside [1, num_experts]";
     case MOE_ERR_CAPACITY_TOO_TIGHT: return "capacity_factor below 1.0 drops tokens under perfectly uniform routing";
-    case MOE_ERR_UNSUPPORTED: return "configuration not supported by this build";
+    case MOE_ERR_UNSUPPORTED: return "configuration not supported by this library";
     case MOE_ERR_WORKSPACE: return "workspace missing or smaller than moe_workspace_size()";
     case MOE_ERR_CUDA: return "CUDA error";
     case MOE_ERR_DEVICE: return "device-side failure recorded in the workspace";
