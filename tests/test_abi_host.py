@@ -231,3 +231,17 @@ def test_workspace_regions(name):
         off, n = C.c_size_t(), C.c_size_t()
         L.check(L.lib().moe_workspace_region(C.byref(cfg), L.MOE_WS_REGION_COUNT, C.byref(off), C.byref(n)),
                 "region")
+
+
+@pytest.mark.parametrize("T,d,E,ks", [
+    (64, 2048, 128, 16),   # decode-sized: 8 x 4 tiles, four blocks per SM asks 19 slices, capped at 16
+    (256, 1024, 64, 8),    # 64 tiles ask 10 slices of 103 elements, rounded up to 128: 8 slices
+    (200, 256, 48, 8),     # 25 x 2 tiles ask 12 slices, capped at d / 32 = 8
+])
+def test_split_router_slice_count(T, d, E, ks):
+    """Small batches take the CUDA-core split pass: 8-token x 32-expert tiles
+    times as many hidden slices (multiples of 32 elements, at most 16) as give
+    148 SMs four blocks each; the workspace holds their float64 partials."""
+    cfg = _cfg(num_tokens=T, hidden=d, num_experts=E, top_k=4)
+    off, n = api.moe_workspace_region(cfg, "router_logits")
+    assert n == ks * T * E * 8, (n // (T * E * 8), ks)
