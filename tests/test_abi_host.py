@@ -245,3 +245,15 @@ def test_split_router_slice_count(T, d, E, ks):
     cfg = _cfg(num_tokens=T, hidden=d, num_experts=E, top_k=4)
     off, n = api.moe_workspace_region(cfg, "router_logits")
     assert n == ks * T * E * 8, (n // (T * E * 8), ks)
+
+
+@pytest.mark.parametrize("T,ks", [(16384, 2), (8192, 4), (1024, 4), (512, 9)])
+def test_integer_router_slice_count(T, ks):
+    """The integer tensor-core plan (bf16, T >= 512) splits the hidden
+    dimension (112 K-blocks of 64 at d = 7168) into the slice count whose
+    rounds of 148 CTAs times K-blocks per CTA, plus four K-blocks of fixed
+    cost, are fewest; the workspace holds the float64 partials."""
+    cfg = _cfg(num_tokens=T, hidden=7168, num_experts=256, top_k=8, router="sigmoid_group", n_group=8,
+               topk_group=4, routed_scaling=2.5)
+    off, n = api.moe_workspace_region(cfg, "router_logits")
+    assert n == ks * T * 256 * 8, (n // (T * 256 * 8), ks)
