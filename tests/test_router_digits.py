@@ -80,3 +80,45 @@ def test_digits_reassemble_and_fit_int8():
     # bf16 values at most 2^14 below the row maximum are represented exactly
     keep = np.abs(x) >= np.abs(x).max(1, keepdims=True) * 2.0 ** -14
     assert np.array_equal((vx * np.ldexp(1.0, -sx)[:, None])[keep], x.astype(np.float64)[keep])
+
+
+def _integer_rne_digits(w: np.ndarray, sw: int) -> np.ndarray:
+    """rne(w 2^sw) the way the preparation pass computes it: from the fp32
+    fields with integer shifts, ties to even, no float conversion."""
+    bits = w.astype(np.float32).view(np.uint32).astype(np.int64)
+    fe = (bits >> 23) & 0xFF
+    mant = bits & 0x7FFFFF
+    m = np.where(fe > 0, mant | 0x800000, mant)
+    sh = np.maximum(fe, 1) - 150 + sw
+    v = np.zeros_like(m)
+    up = sh >= 0
+    v[up] = m[up] << sh[up]
+    mid = (sh < 0) & (sh >= -25)
+    k = -sh[mid]
+    q = m[mid] >> k
+    rem = m[mid] & ((1 << k) - 1)
+    half = 1 << (k - 1)
+    q = q + ((rem > half) | ((rem == half) & (q & 1 == 1)))
+    v[mid] = q
+    return np.where(bits >> 31 == 1, -v, v)
+
+
+def test_weight_digit_integer_rounding_matches_rint():
+    """The integer rounding of the router weights to their 30-bit digits
+    equals round-half-even of w 2^sw in float64 over normal, subnormal, tie
+    and far-below-the-row-maximum values."""
+    rng = np.random.default_rng(13)
+    w = (rng.standard_normal(20000) * np.exp2(rng.integers(-40, 10, 20000))).astype(np.float32)
+    w[:8] = np.array([0.0, -0.0, 1e-45, -3e-42, 0.75, -0.75, 1.5, 2.5], dtype=np.float32)
+    for scale in (1.0, 2.0 ** -100, 3.0e4):
+        row = (w.astype(np.float64) * scale).astype(np.float32)
+        _, sw, vref = weight_digits(row[None, :])
+        got = _integer_rne_digits(row, int(sw[0]))
+        assert np.array_equal(got, vref[0])
+        # ties exercised: values exactly half a unit of 2^-sw away from an integer
+        t = (np.arange(1, 200) + 0.5) * np.ldexp(1.0, -int(sw[0]))
+        t = t[np.abs(t) <= np.abs(row).max()].astype(np.float32)
+        t = t[t.astype(np.float64) == (np.arange(1, 200) + 0.5)[: len(t)] * np.ldexp(1.0, -int(sw[0]))]
+        if len(t):
+            assert np.array_equal(_integer_rne_digits(t, int(sw[0])),
+                                  np.rint(t.astype(np.float64) * np.ldexp(1.0, int(sw[0]))).astype(np.int64))
