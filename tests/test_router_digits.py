@@ -122,3 +122,32 @@ def test_weight_digit_integer_rounding_matches_rint():
         if len(t):
             assert np.array_equal(_integer_rne_digits(t, int(sw[0])),
                                   np.rint(t.astype(np.float64) * np.ldexp(1.0, int(sw[0]))).astype(np.int64))
+
+
+def test_chunk_selection_covers_every_rounded_element():
+    """The preparation pass reads again only the 8-element chunks whose
+    smallest exponent field e (taken as 1 for zeros and subnormals) lies below
+    the row's largest minus 14 (all chunks when the scale is clamped).  Every
+    element that the digits round lies in such a chunk."""
+    rng = np.random.default_rng(17)
+    d = 1024
+    rows = [rng.standard_normal(d), rng.standard_normal(d) * 1e-3, np.zeros(d),
+            rng.standard_normal(d) * 1e-39, rng.standard_normal(d) * 2.0 ** 60]
+    r = rng.standard_normal(d)
+    r[5] = 4000.0                              # an outlier: far-below elements round
+    rows.append(r)
+    r = rng.standard_normal(d)
+    r[::3] = 0.0
+    rows.append(r)
+    x = _bf16(np.stack(rows))
+    _, sx, v = token_digits(x)
+    bits = torch.from_numpy(x.astype(np.float32)).to(torch.bfloat16).view(torch.int16).numpy().astype(np.int64)
+    mag = bits & 0x7FFF
+    rounded = x.astype(np.float64) != v * np.ldexp(1.0, -sx)[:, None]
+    for t in range(x.shape[0]):
+        emax = max(int(mag[t].max()) >> 7, 1)
+        clamped = emax < 21                    # the scale 2^sx was capped at 2^127
+        ethr = emax - 14
+        chunk_min_e = np.maximum(mag[t].reshape(-1, 8).min(axis=1) >> 7, 1)
+        selected = np.ones(d // 8, bool) if clamped else chunk_min_e < ethr
+        assert np.all(selected[np.nonzero(rounded[t])[0] // 8]), t
