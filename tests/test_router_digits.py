@@ -151,3 +151,51 @@ def test_chunk_selection_covers_every_rounded_element():
         chunk_min_e = np.maximum(mag[t].reshape(-1, 8).min(axis=1) >> 7, 1)
         selected = np.ones(d // 8, bool) if clamped else chunk_min_e < ethr
         assert np.all(selected[np.nonzero(rounded[t])[0] // 8]), t
+
+
+def _group8_select(sel: np.ndarray, n_group: int, topk_group: int, top_k: int) -> np.ndarray:
+    """The lane-per-eight-experts selection, step for step: lane l holds
+    experts 8 l .. 8 l + 7; a group's two largest scores from each lane's own
+    pair merged over the group's lanes by xor partners; kept groups by a rank
+    count (ties to the lower group); the top k as k rounds taking the largest
+    head of each lane's sorted candidates (ties to the lower lane)."""
+    E = sel.shape[0]
+    lanes = E // 8
+    lg = E // n_group // 8
+    s = sel.reshape(lanes, 8)
+    a = np.sort(s, axis=1)[:, ::-1][:, :2].copy()          # (a1, a2) per lane
+    o = 1
+    while o < lg:
+        b = a[np.arange(lanes) ^ o]
+        a = np.stack([np.maximum(a[:, 0], b[:, 0]),
+                      np.maximum(np.minimum(a[:, 0], b[:, 0]), np.maximum(a[:, 1], b[:, 1]))], axis=1)
+        o <<= 1
+    gs = a[:, 0] + a[:, 1]                                  # every lane of a group holds its score
+    g = np.arange(lanes) // lg
+    gscore = gs[np.arange(n_group) * lg]
+    rank = np.array([np.sum((gscore > gscore[gi]) | ((gscore == gscore[gi]) & (np.arange(n_group) < gi)))
+                     for gi in g])
+    keep = rank < topk_group
+    cand = np.where(keep[:, None], s, -np.inf)
+    heads = [sorted([(-cand[l, j], j) for j in range(8)]) for l in range(lanes)]   # largest first, lower j
+    chosen = []
+    for _ in range(top_k):
+        best = max(range(lanes), key=lambda l: (-heads[l][0][0], -l))
+        chosen.append(8 * best + heads[best].pop(0)[1])
+        heads[best].append((np.inf, 99))                     # an emptied slot sorts last
+    return np.array(chosen)
+
+
+@pytest.mark.parametrize("E,n_group,topk_group,top_k", [(256, 8, 4, 8), (64, 8, 3, 6), (96, 6, 2, 5),
+                                                        (256, 4, 2, 8), (128, 1, 1, 8)])
+def test_group8_selection_matches_group_routing(E, n_group, topk_group, top_k):
+    """The lane-per-eight-experts selection chooses the oracle's experts, in
+    its order, also when scores tie (logits on a coarse grid)."""
+    rng = np.random.default_rng(E + n_group)
+    for trial in range(40):
+        logits = rng.integers(-8, 9, (4, E)) * 0.25 if trial % 2 else rng.standard_normal((4, E))
+        bias = rng.integers(-2, 3, E) * 0.01 if trial % 3 else None
+        ids, _, s, _ = O.route_sigmoid_group(logits, top_k, n_group, topk_group, 1.0, expert_bias=bias)
+        sel = s + (bias if bias is not None else 0.0)
+        for t in range(logits.shape[0]):
+            assert np.array_equal(_group8_select(sel[t], n_group, topk_group, top_k), ids[t]), (trial, t)
