@@ -257,3 +257,32 @@ def test_integer_router_slice_count(T, ks):
                topk_group=4, routed_scaling=2.5)
     off, n = api.moe_workspace_region(cfg, "router_logits")
     assert n == ks * T * 256 * 8, (n // (T * 256 * 8), ks)
+
+
+def _router_plan_sizes(env_extra):
+    """Workspace size and router-logits region of two bf16 configurations,
+    in a fresh process (the router switch is read once per process)."""
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    code = (
+        "import sys; sys.path.insert(0, %r)\n"
+        "from mixture_experts_layer_41_b200 import api\n"
+        "for T, d, E, k, kw in [(1024, 1024, 256, 8, dict(router='sigmoid_group', n_group=8, topk_group=4)),\n"
+        "                       (600, 512, 8, 2, {})]:\n"
+        "    cfg = api.make_config(num_tokens=T, hidden=d, intermediate=64, num_experts=E, top_k=k, **kw)\n"
+        "    print(api.moe_workspace_size(cfg), api.moe_workspace_region(cfg, 'router_logits')[1])\n" % root)
+    env = {k: v for k, v in os.environ.items() if k != "MOE_ROUTER_TC"}
+    env.update(env_extra)
+    r = subprocess.run([sys.executable, "-c", code], env=env, capture_output=True, text=True, timeout=300)
+    assert r.returncode == 0, r.stderr
+    return [tuple(int(v) for v in line.split()) for line in r.stdout.split("\n") if line.strip()]
+
+
+def test_bf16_router_switch_changes_the_plan():
+    """MOE_ROUTER_TC=bf16 puts bf16 batches of 512 tokens or more on the bf16
+    selection-grade tensor-core logits instead of the integer ones: the
+    workspace the plan sizes differs (its own weight slices and slice count)."""
+    default = _router_plan_sizes({})
+    bf16 = _router_plan_sizes({"MOE_ROUTER_TC": "bf16"})
+    assert len(default) == len(bf16) == 2
+    assert all(a[0] != b[0] for a, b in zip(default, bf16))

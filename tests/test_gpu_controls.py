@@ -419,3 +419,34 @@ def test_router_wait_timeout_reports_and_recovers():
     torch.cuda.synchronize()
     assert run.status() == 0
     check_route(run, oracle_route(w, run.inp))
+
+
+# ---------------------------------------------------------------- bf16 tensor-core router (opt-in)
+def test_bf16_tensor_core_router_routes_as_the_oracle():
+    """MOE_ROUTER_TC=bf16 (read once per process, so run in a fresh one)
+    routes bf16 batches of 512 tokens or more with the bf16 selection-grade
+    tensor-core logits and an exact re-weighting of every token's chosen
+    experts; ids, weights and probability sums match the oracle."""
+    import os
+    import subprocess
+    import sys
+    tests = os.path.dirname(os.path.abspath(__file__))
+    code = (
+        "import sys; sys.path[:0] = [%r, %r]\n"
+        "import torch\n"
+        "from gpu_harness import Run, check_route\n"
+        "from moe_cases import oracle_route\n"
+        "from mixture_experts_layer_41_b200 import api\n"
+        "from mixture_experts_layer_41_b200.inputs import workload\n"
+        "for w in (workload('deepseek_v3', T=1024, d=1024, F=64, shared_F=0),\n"
+        "          workload('mixtral_prefill', T=600, d=512, F=64)):\n"
+        "    run = Run(w, seed=7)\n"
+        "    api.moe_route(run.cfg, run.inp['x'], run.inp['w_router'], run.bias, run.ids, run.wts,\n"
+        "                  run.prob_sum, run.ws)\n"
+        "    torch.cuda.synchronize()\n"
+        "    assert run.status() == 0\n"
+        "    check_route(run, oracle_route(w, run.inp))\n"
+        "print('routed')\n" % (os.path.dirname(tests), tests))
+    env = dict(os.environ, MOE_ROUTER_TC="bf16")
+    r = subprocess.run([sys.executable, "-c", code], env=env, capture_output=True, text=True, timeout=900)
+    assert r.returncode == 0 and "routed" in r.stdout, r.stdout[-2000:] + r.stderr[-4000:]
